@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA prefill hot path on B200 (one JSON line on rank 0).
+
+A step is one pass of the whole hot path over one batch of synthetic input.  For the default
+workload (one 131072-token sequence, 32 value heads, dk = dv = 128, bf16 q/k/v, fp32 gates and
+state, cut into 16 segments of 8192) a step is the context-parallel prefill:
+  1. kda_segment_summarize_and_scan: per-segment transition M_i and contribution U_i for every
+     head, then the exclusive affine scan (incoming / outgoing / final states);
+  2. kda_chunk_fwd over the 16 segments as independent sequences, each starting from its
+     incoming state -- every output row of the sequence plus the final state.
+Other workloads (``--workload``) time one kda_chunk_fwd call over the whole batch; their
+state pool carries over from step to step (each step resumes from the previous final states,
+as a split prefill would), so the timed work never includes a pool restore.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload (the
+oracle is the only reference implementation there is).  Under torchrun every rank runs its
+own replica of the workload (weak scaling, no data-path collective); timings are device
+times, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kda_workloads as W  # noqa: E402
+
+METRIC = "KDA prefill tokens/s (H=32,dk=dv=128,bf16) and % of roofline on 1 B200"
+DEFAULT_WORKLOAD = "long_T131072_H32_cp16"
+
+
+# ------------------------------------------------------------------------------------------
+# algorithmic traffic and work (per launch), see the design notes for the derivation
+# ------------------------------------------------------------------------------------------
+
+def io_bytes_per_token_head(qkv_bytes=2, out_bytes=2, dk=128, dv=128, group=1):
+    # q and k are read once per key head; for Hv = Hk each value head reads its own q, k
+    return (2 * dk * qkv_bytes) / group + dv * qkv_bytes + dk * 4 + 4 + dv * out_bytes
+
+
+def chunk_fwd_bytes(w, num_seqs, dk=128, dv=128):
+    th = w.total_tokens * w.num_v_heads
+    group = w.num_v_heads // w.num_k_heads
+    qkv = 2 if w.q.dtype == torch.bfloat16 else 4
+    ob = 2 if w.output_dtype == torch.bfloat16 else 4
+    return th * io_bytes_per_token_head(qkv, ob, dk, dv, group) + num_seqs * w.num_v_heads * 2 * dk * dv * 4
+
+
+def segment_bytes(w, N, dk=128, dv=128):
+    th = w.total_tokens * w.num_v_heads
+    qkv = 2 if w.q.dtype == torch.bfloat16 else 4
+    reads = th * (dk * qkv + dv * qkv + dk * 4 + 4)
+    summaries = N * w.num_v_heads * (dk * dk + dk * dv) * 4
+    scan = N * w.num_v_heads * dk * dv * 4 * 2 + summaries  # incoming + outgoing written, M/U re-read
+    return reads + summaries + scan
+
+
+def chunk_fwd_flops(w, C=64, dk=128, dv=128):
+    # 6 d^2 (W S, (Q o Gamma) S, K'^T Delta) + 5 C d (A, P, W, U, P Delta) + C^2/3 (inverse)
+    th = w.total_tokens * w.num_v_heads
+    return th * (2 * 3 * dk * dv + 2 * 2.5 * C * dk + C * C / 3)
+
+
+# ------------------------------------------------------------------------------------------
+# helpers
+# ------------------------------------------------------------------------------------------
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kimi_delta_attention_23_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from a committed ncu summary, only if the kernel is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index=0):
+        self.proc = None
+        self.path = os.path.join("/tmp", f"kda_clocks_{os.getpid()}.csv")
+        sel = []
+        try:
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            sel = ["-i", bus] if bus else []
+        except Exception:
+            sel = []
+        self.cmd = ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(self.cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(float(r[2]) for r in rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit()),
+                "samples": len(rows), "reasons": reasons}
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+# ------------------------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ------------------------------------------------------------------------------------------
+
+def oracle_time_sample(w, n_tokens):
+    """Run the oracle over the first n_tokens of every (sequence, head) chain's token range."""
+    import oracle
+    cu = w.cu_seqlens.cpu().tolist()
+    # take a prefix of the packed batch, cutting sequence boundaries where they fall
+    n = min(n_tokens, w.total_tokens)
+    cu_s = [c for c in cu if c < n] + [n]
+    B = len(cu_s) - 1
+    cpu = lambda t: t.detach().cpu()  # noqa: E731
+    t0 = time.perf_counter()
+    oracle.kda_forward(cpu(w.q)[:n], cpu(w.k)[:n], cpu(w.v)[:n], cpu(w.raw_gate)[:n], cpu(w.beta_logits)[:n],
+                       cpu(w.a_log), cpu(w.dt_bias), torch.tensor(cu_s, dtype=torch.int32),
+                       cpu(w.state_pool), cpu(w.state_indices)[:B], gate_mode=w.gate_mode, beta_mode=w.beta_mode,
+                       state_layout=w.state_layout, gate_lower_bound=w.gate_lower_bound)
+    return time.perf_counter() - t0, n
+
+
+def calibrate_oracle(w, target_s):
+    n = 256
+    while True:
+        dt, n_done = oracle_time_sample(w, n)
+        if dt >= target_s / 4 or n_done >= w.total_tokens:
+            scale = target_s / max(dt, 1e-6)
+            return max(1, min(w.total_tokens, int(n_done * scale)))
+        n *= 4
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    w = W.make(args.workload, device="cpu")
+    n = calibrate_oracle(w, target_s=args.ref_step_seconds)
+    for _ in range(args.warmup):
+        oracle_time_sample(w, n)
+    times = [oracle_time_sample(w, n)[0] for _ in range(args.steps)]
+    total = sum(times)
+    value = n * args.steps / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload, "tokens_per_step": n,
+                                            "num_v_heads": w.num_v_heads, "dk": w.dk, "dv": w.dv},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"first {n} tokens of the workload, all {w.num_v_heads} heads, per step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------
+
+class Step:
+    """One pass of the hot path on device-resident inputs; records per-call CUDA events."""
+
+    def __init__(self, w, stream):
+        import kimi_delta_attention_23_b200 as kda
+        self.kda, self.w, self.stream = kda, w, stream
+        dev = w.q.device
+        self.cp = w.seg_offsets is not None
+        T, Hv, dv, dk = w.total_tokens, w.num_v_heads, w.dv, w.dk
+        self.out = torch.empty((T, Hv, dv), dtype=w.output_dtype, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        if self.cp:
+            N = w.seg_offsets.numel() - 1
+            st = (dk, dv) if w.state_layout == "K_FIRST" else (dv, dk)
+            self.N = N
+            # single-sequence workload whose state sits in pool slot 0 (a view: it follows the pool)
+            self.init = w.state_pool[0]
+            self.M = torch.empty((N, Hv, dk, dk), device=dev)
+            self.U = torch.empty((N, Hv, *st), device=dev)
+            self.inc = torch.empty((N, Hv, *st), device=dev)
+            self.outg = torch.empty((N, Hv, *st), device=dev)
+            self.fin = torch.empty((Hv, *st), device=dev)
+            self.seg_idx = torch.arange(N, dtype=torch.int32, device=dev)
+        self.pool = None if self.cp else w.state_pool.clone()
+        self.events = []
+
+    def kw(self):
+        w = self.w
+        return dict(gate_mode=w.gate_mode, beta_mode=w.beta_mode, state_layout=w.state_layout,
+                    gate_lower_bound=w.gate_lower_bound, device_status=self.status, stream=self.stream)
+
+    def launches(self):
+        return 4 if self.cp else 1  # transition build, contribution build, scan, chunk pass
+
+    def __call__(self, record=False):
+        w, kda = self.w, self.kda
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if record else None
+        if ev:
+            ev[0].record(self.stream)
+        if self.cp:
+            kda.kda_segment_summarize_and_scan(w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias,
+                                               w.seg_offsets, self.init, M=self.M, U=self.U, incoming=self.inc,
+                                               outgoing=self.outg, final_state=self.fin, **self.kw())
+            if ev:
+                ev[1].record(self.stream)
+            kda.kda_chunk_fwd(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.seg_offsets,
+                              self.inc, self.seg_idx, self.out, **self.kw())
+        else:
+            if ev:
+                ev[1].record(self.stream)
+            kda.kda_chunk_fwd(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens,
+                              self.pool, w.state_indices, self.out, **self.kw())
+        if ev:
+            ev[2].record(self.stream)
+            self.events.append(ev)
+
+
+def run_ours(args):
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        pg = dist
+    from kimi_delta_attention_23_b200 import build as kbuild
+    kbuild.build()
+    w = W.make(args.workload, device=dev, seed=None if rank == 0 else 1000 * rank + W.WORKLOADS.index(args.workload))
+    stream = torch.cuda.current_stream(dev)
+    step = Step(w, stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {int(step.status.item())} during warm-up")
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    # timed region: K steps, events per API call plus the bracketing pair
+    step.events.clear()
+    barrier()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        start.record(stream)
+        for _ in range(args.steps):
+            step(record=True)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = start.elapsed_time(stop)
+    seg_ms = [e[0].elapsed_time(e[1]) for e in step.events]
+    pass_ms = [e[1].elapsed_time(e[2]) for e in step.events]
+    if pg is not None:
+        t = torch.tensor([ms_total], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    tokens = w.total_tokens
+    value = tokens * world / (ms_total / args.steps / 1e3)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(w, args, stream, pg)
+
+    if rank != 0:
+        if pg is not None:
+            pg.destroy_process_group()
+        return 0
+    pk = peaks()
+    n_seq = (step.N if step.cp else w.batch)
+    bytes_pass = chunk_fwd_bytes(w, n_seq)
+    ms_pass = statistics.mean(pass_ms)
+    ms_seg = statistics.mean(seg_ms) if step.cp else 0.0
+    achieved = bytes_pass / (ms_pass / 1e3) / 1e9
+    dom = "kda_chunk_fwd"
+    roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / pk["hbm_gbs"], "traffic": recorded_traffic(dom),
+            "algorithmic_bytes_per_launch": bytes_pass, "ms_per_launch": ms_pass,
+            "peak_source": pk["source"]}
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.q.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+            "config": {"workload": args.workload, "tokens": tokens, "num_v_heads": w.num_v_heads,
+                       "num_k_heads": w.num_k_heads, "dk": w.dk, "dv": w.dv, "batch": w.batch,
+                       "segments": step.N if step.cp else None, "gate_mode": w.gate_mode,
+                       "state_layout": w.state_layout, "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (%.2f GB read per step), no flush" % (bytes_pass / 1e9)},
+            "breakdown_ms": {"segment_summarize_and_scan": ms_seg, "chunk_fwd": ms_pass},
+            "roofline": roof, "gpu_launches": step.launches() * args.steps, "clocks": clocks.summary()}
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args)
+    print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+def measure_e2e(w, args, stream, pg):
+    """Same step through the public API with pinned host buffers: H2D of every input, the step,
+    D2H of the output rows and the final state, all inside the timed region."""
+    dev = w.q.device
+    names = ["q", "k", "v", "raw_gate", "beta_logits", "a_log", "dt_bias", "cu_seqlens", "state_pool",
+             "state_indices"] + (["seg_offsets"] if w.seg_offsets is not None else [])
+    host = {n: getattr(w, n).cpu().pin_memory() for n in names}
+    wd = W.Workload(**{k: getattr(w, k) for k in w.__dataclass_fields__})
+    for n in names:
+        setattr(wd, n, torch.empty_like(getattr(w, n)))
+    step = Step(wd, stream)
+    out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    fin_src = step.fin if step.cp else step.pool
+    fin_host = torch.empty(fin_src.shape, dtype=fin_src.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size() + fin_host.numel() * fin_host.element_size()
+
+    def one():
+        for n in names:
+            getattr(wd, n).copy_(host[n], non_blocking=True)
+        if not step.cp:
+            step.pool.copy_(wd.state_pool)
+        step()
+        out_host.copy_(step.out, non_blocking=True)
+        fin_host.copy_(fin_src, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        one()
+    torch.cuda.synchronize()
+    if pg is not None:
+        pg.barrier()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(1, min(args.steps, 5))
+    start.record(stream)
+    for _ in range(n):
+        one()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(stop)
+    if pg is not None:
+        t = torch.tensor([ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    world = pg.get_world_size() if pg is not None else 1
+    return {"value": w.total_tokens * world / (ms / n / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n}
+
+
+def cpu_baseline(w, args):
+    import oracle
+    wc = w.to("cpu")
+    n = calibrate_oracle(wc, target_s=args.cpu_seconds)
+    dt, n = oracle_time_sample(wc, n)
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {n} tokens of the workload, all {w.num_v_heads} heads (fp64 token-by-token)",
+            "seconds": dt}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=W.WORKLOADS, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

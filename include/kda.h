@@ -1,0 +1,165 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention prefill library (libkda.so).
+ *
+ * Two operations:
+ *
+ *  kda_chunk_fwd
+ *    The chunk-parallel KDA prefill ("max.nn.state_space.kda_chunk": the same recurrence as
+ *    single-token decode, evaluated in parallel over fixed-size chunks, mutating the state
+ *    pool).  For every sequence b, value head h and token t of that sequence:
+ *        g_t  = -exp(a_log[h]) * softplus(raw_gate[t,h,:] + dt_bias[h,:])   (per key channel)
+ *               ("safe" gate mode: g_t = max(g_t, gate_lower_bound))
+ *        b_t  = sigmoid(beta_logits[t,h])   (or beta_logits[t,h] itself in probability mode)
+ *        S    = Diag(exp(g_t)) S                          decay each key row
+ *        S    = S + k_t (b_t (v_t - k_t^T S))^T           delta-rule write (predicts from the
+ *                                                          decayed state; overwrites along k)
+ *        o_t  = q_t^T S                                   readout after the write
+ *    ("nx_nofloat_kda.nx source": gate, then delta write, then read, per token.)
+ *    S (dk x dv, fp32) starts as state_pool[state_indices[b], h] and is written back there
+ *    when the sequence ends.  The key head used by value head h is h / (Hv / Hk).  No query
+ *    scaling is applied (GStar Assignment 2: the formulas omit it; scale = 1).
+ *
+ *  kda_segment_summarize_and_scan
+ *    Context-parallel segment summary and exclusive scan ("KDA Context Parallelism"): a
+ *    single sequence is cut into N segments; each is reduced to the affine map
+ *    F_i(S) = M_i S + U_i (M_i: how the segment transforms its incoming state, dk x dk;
+ *    U_i: the state it creates from zero, dk x dv); the maps are applied in sequence order
+ *    (an exclusive prefix), giving every segment its incoming and outgoing state and the
+ *    final state.  A later kda_chunk_fwd call with cu_seqlens = segment offsets, the incoming
+ *    stack as the state pool and state_indices = 0..N-1 then produces every segment's
+ *    outputs in parallel; afterwards that pool holds the outgoing states.
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major and densely
+ *    packed in the stated shapes.  The library allocates no device memory.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *    default stream).  The returned status covers the host-side checks and the launch only.
+ *  - Host-side checks are always on: null pointers, extents, Hv % Hk == 0, dtype groupings
+ *    that bind no kernel, flag combinations.  A failed check returns before any launch and
+ *    writes nothing.
+ *  - device_status (nullable, device int32): kernels record the first device-side finding
+ *    there (KDA_ERR_DEVICE_CHECK for a state slot outside [0, max_slots) or decreasing
+ *    offsets -- that sequence is skipped and its slot and outputs are left untouched;
+ *    KDA_ERR_DEVICE_TIMEOUT if a bounded wait gave up).  The caller zeroes it beforehand and
+ *    reads it after synchronising.  Kernels never trap.
+ *  - Inputs must not alias outputs.  Two sequences naming the same pool slot is a caller
+ *    error with an unspecified result.  Pool slots not named by state_indices are never
+ *    touched.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1,    /* null pointer, bad extent, Hv % Hk != 0, bad flags          */
+  KDA_ERR_UNSUPPORTED = 2,    /* the dtype grouping / head dims bind no kernel               */
+  KDA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than kda_workspace_size()      */
+  KDA_ERR_CUDA = 4,           /* a CUDA runtime call (attribute set, launch) failed          */
+  KDA_ERR_DEVICE_CHECK = 5,   /* device_status value: bad slot or decreasing offsets         */
+  KDA_ERR_DEVICE_TIMEOUT = 6  /* device_status value: a bounded wait gave up                 */
+} kda_status_t;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
+
+/* flags (bitwise OR) -- the kda_chunk keyword arguments gate_mode, beta_mode, state_layout
+ * and use_computebound */
+enum {
+  KDA_GATE_SAFE = 1u << 0,     /* gate_mode="safe": g = max(g, gate_lower_bound); else "original" */
+  KDA_BETA_PROB = 1u << 1,     /* beta_mode="probability": beta used as given; else sigmoid(logits) */
+  KDA_STATE_V_FIRST = 1u << 2, /* state_layout="V_FIRST": a slot stores S^T as [dv][dk]; else [dk][dv] */
+  KDA_FUSED = 1u << 3,         /* use_computebound: accepted; the bf16 path is always the fused kernel */
+  KDA_SEG_SCAN_ONLY = 1u << 4, /* segment call: M and U are inputs, only the scan runs           */
+  KDA_FORCE_SIMT = 1u << 5     /* run the fp32 CUDA-core chunk kernel even for bf16 inputs       */
+};
+
+/*
+ * kda_chunk_fwd -- chunk-parallel KDA prefill over a varlen batch (kda_chunk, all parameters).
+ *
+ *   q, k          [total_tokens, num_k_heads, dk]   qkv_dtype
+ *   v             [total_tokens, num_v_heads, dv]   qkv_dtype
+ *   raw_gate      [total_tokens, num_v_heads, dk]   fp32, forget-gate pre-activation before dt_bias
+ *   beta_logits   [total_tokens, num_v_heads]       fp32 (logits, or probabilities with KDA_BETA_PROB)
+ *   a_log         [num_v_heads]                     fp32
+ *   dt_bias       [num_v_heads, dk]                 fp32
+ *   cu_seqlens    [batch + 1]                       int32 exclusive prefix offsets, cu_seqlens[batch]
+ *                                                   <= total_tokens; zero-length sequences allowed
+ *   state_pool    [max_slots, num_v_heads, dk, dv]  fp32 (K_FIRST) or [.., dv, dk] (V_FIRST); read
+ *                                                   and written in place
+ *   state_indices [batch]                           int32 pool slot of each sequence
+ *   out           [total_tokens, num_v_heads, dv]   out_dtype; rows outside every sequence untouched
+ *   gate_lower_bound                                used only with KDA_GATE_SAFE
+ *   workspace     unused by the current kernels (kda_workspace_size() returns 0); may be NULL
+ *
+ * Supported groupings: (qkv F32, out F32) for any 1 <= dk, dv <= 128 on the fp32 CUDA-core
+ * kernel; (qkv BF16, out BF16 or F32) with dk = dv = 128 on the fused tensor-core kernel, or on
+ * the fp32 kernel with KDA_FORCE_SIMT.  Anything else returns KDA_ERR_UNSUPPORTED.
+ */
+KDA_API kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                           const float *raw_gate, const float *beta_logits, const float *a_log,
+                           const float *dt_bias, const int32_t *cu_seqlens, int32_t batch,
+                           int64_t total_tokens, int32_t num_k_heads, int32_t num_v_heads,
+                           int32_t dk, int32_t dv, float *state_pool, int32_t max_slots,
+                           const int32_t *state_indices, void *out, kda_dtype_t out_dtype,
+                           uint32_t flags, float gate_lower_bound, void *workspace,
+                           size_t workspace_bytes, int32_t *device_status, void *stream);
+
+/*
+ * kda_segment_summarize_and_scan -- segment summaries and the exclusive affine scan of ONE
+ * sequence ("KDA Context Parallelism": Theory; Compose segments in sequence order; Incoming
+ * and outgoing states; Implementation order; Requirements).
+ *
+ *   k             [T, num_k_heads, dk]    kv_dtype      (ignored with KDA_SEG_SCAN_ONLY)
+ *   v             [T, num_v_heads, dv]    kv_dtype      (ignored with KDA_SEG_SCAN_ONLY)
+ *   raw_gate, beta_logits, a_log, dt_bias  as in kda_chunk_fwd (ignored with KDA_SEG_SCAN_ONLY)
+ *   seg_offsets   [num_segments + 1]       int32 device, seg_offsets[0] = 0 ... = T, non-decreasing
+ *   initial_state [num_v_heads, <state>]   fp32, <state> = [dk][dv] (K_FIRST) or [dv][dk] (V_FIRST)
+ *   M             [num_segments, num_v_heads, dk, dk]   fp32, row-major, F_i(S) = M_i S + U_i
+ *                                          (written; read-only input with KDA_SEG_SCAN_ONLY)
+ *   U             [num_segments, num_v_heads, <state>]  fp32 (written; input with SCAN_ONLY)
+ *   incoming      [num_segments, num_v_heads, <state>]  fp32 out: state entering segment i
+ *   outgoing      [num_segments, num_v_heads, <state>]  fp32 out: state leaving segment i
+ *   final_state   [num_v_heads, <state>]                fp32 out: outgoing of the last segment
+ *
+ * num_segments >= 1.  M_i is the segment's transition (the recurrence run from S = I with zero
+ * values); U_i is its local contribution (the recurrence from S = 0).  Left multiplication:
+ * out_i = M_i in_i + U_i.  initial_state, M and U (in SCAN_ONLY mode) are never written.
+ * Summaries need dk <= 128 and dv <= 128 (fp32 or bf16 k/v).
+ */
+KDA_API kda_status_t kda_segment_summarize_and_scan(
+    const void *k, const void *v, kda_dtype_t kv_dtype, const float *raw_gate,
+    const float *beta_logits, const float *a_log, const float *dt_bias, int64_t T,
+    int32_t num_k_heads, int32_t num_v_heads, int32_t dk, int32_t dv, const int32_t *seg_offsets,
+    int32_t num_segments, const float *initial_state, float *M, float *U, float *incoming,
+    float *outgoing, float *final_state, uint32_t flags, float gate_lower_bound, void *workspace,
+    size_t workspace_bytes, int32_t *device_status, void *stream);
+
+/* Bytes of workspace kda_chunk_fwd / kda_segment_summarize_and_scan need for these extents
+ * (0 for the current kernels). */
+KDA_API size_t kda_workspace_size(int64_t total_tokens, int32_t batch, int32_t num_k_heads,
+                          int32_t num_v_heads, int32_t dk, int32_t dv, int32_t num_segments,
+                          uint32_t flags);
+
+/* Static, human-readable name of a status code. */
+KDA_API const char *kda_status_string(kda_status_t status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+KDA_API int32_t kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,272 @@
+"""Python binding of libkda.so, the sm_100a KDA prefill library (argument marshalling only).
+
+Every step of the computation runs in the CUDA kernels behind the C ABI in ``include/kda.h``;
+this module only turns torch tensors into pointers and extents.  PyTorch supplies device
+memory and streams.  There is no CPU path: if ``libkda.so`` is missing, every call raises.
+
+Public calls (same names as the C ABI):
+  kda_chunk_fwd(...)                      chunk-parallel prefill, mutates state_pool in place
+  kda_segment_summarize_and_scan(...)     segment (M_i, U_i) summaries + exclusive scan
+  kda_context_parallel(M, U, initial)     the scan alone, returning exactly incoming_states,
+                                          outgoing_states and final_state
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["kda_chunk_fwd", "kda_segment_summarize_and_scan", "kda_context_parallel",
+           "kda_workspace_size", "kda_status_string", "load_library", "KdaError", "LIB_PATH"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkda.so")
+
+# flag bits of include/kda.h
+GATE_SAFE = 1 << 0
+BETA_PROB = 1 << 1
+STATE_V_FIRST = 1 << 2
+FUSED = 1 << 3
+SEG_SCAN_ONLY = 1 << 4
+FORCE_SIMT = 1 << 5
+
+_F32, _BF16 = 0, 1
+_DTYPES = {torch.float32: _F32, torch.bfloat16: _BF16}
+
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {kda_status_string(code)} (status {code})")
+
+
+def load_library():
+    """Load libkda.so (built in-tree by ``build.py``); raise loudly if it is absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libkda.so is not built at {LIB_PATH}; run kimi_delta_attention_23_b200/build.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, fp, ip = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+    i32, i64, u32, f32, sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float, ctypes.c_size_t
+    lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_chunk_fwd.argtypes = [vp, vp, vp, ctypes.c_int, fp, fp, fp, fp, ip, i32, i64, i32, i32, i32,
+                                  i32, fp, i32, ip, vp, ctypes.c_int, u32, f32, vp, sz, ip, vp]
+    lib.kda_segment_summarize_and_scan.restype = ctypes.c_int
+    lib.kda_segment_summarize_and_scan.argtypes = [vp, vp, ctypes.c_int, fp, fp, fp, fp, i64, i32, i32,
+                                                   i32, i32, ip, i32, fp, fp, fp, fp, fp, fp, u32, f32,
+                                                   vp, sz, ip, vp]
+    lib.kda_workspace_size.restype = sz
+    lib.kda_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32, i32, u32]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_version.restype = i32
+    lib.kda_version.argtypes = []
+    _lib = lib
+    return lib
+
+
+def kda_status_string(code: int) -> str:
+    return load_library().kda_status_string(int(code)).decode()
+
+
+def kda_workspace_size(total_tokens, batch, num_k_heads, num_v_heads, dk, dv, num_segments=0, flags=0) -> int:
+    return int(load_library().kda_workspace_size(total_tokens, batch, num_k_heads, num_v_heads, dk, dv,
+                                                 num_segments, flags))
+
+
+def _flags(gate_mode, beta_mode, state_layout, use_computebound=False, force_simt=False, scan_only=False):
+    if gate_mode not in ("original", "safe"):
+        raise ValueError(f"gate_mode must be 'original' or 'safe', got {gate_mode!r}")
+    if beta_mode not in ("logits", "probability"):
+        raise ValueError(f"beta_mode must be 'logits' or 'probability', got {beta_mode!r}")
+    if state_layout not in ("K_FIRST", "V_FIRST"):
+        raise ValueError(f"state_layout must be 'K_FIRST' or 'V_FIRST', got {state_layout!r}")
+    f = 0
+    f |= GATE_SAFE if gate_mode == "safe" else 0
+    f |= BETA_PROB if beta_mode == "probability" else 0
+    f |= STATE_V_FIRST if state_layout == "V_FIRST" else 0
+    f |= FUSED if use_computebound else 0
+    f |= FORCE_SIMT if force_simt else 0
+    f |= SEG_SCAN_ONLY if scan_only else 0
+    return f
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None, device=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device}); there is no CPU path")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _shape(t, name, shape):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, state_pool, state_indices,
+                  out=None, *, output_dtype=None, use_computebound=False, gate_mode="original",
+                  beta_mode="logits", state_layout="K_FIRST", gate_lower_bound=-5.0, force_simt=False,
+                  device_status=None, stream=None):
+    """Chunk-parallel KDA prefill (``max.nn.state_space.kda_chunk`` semantics).
+
+    Shapes: q,k [T,Hk,dk]; v [T,Hv,dv]; raw_gate [T,Hv,dk] f32; beta_logits [T,Hv] f32;
+    a_log [Hv] f32; dt_bias [Hv,dk] f32; cu_seqlens [B+1] i32; state_pool [slots,Hv,dk,dv]
+    (K_FIRST) or [slots,Hv,dv,dk] (V_FIRST) f32, mutated in place; state_indices [B] i32.
+    Returns out [T,Hv,dv] in ``output_dtype`` (default: the dtype of v).
+    """
+    lib = load_library()
+    dev = q.device
+    _dev(q, "q", device=dev)
+    if q.dtype not in _DTYPES:
+        raise ValueError("q/k/v must be float32 or bfloat16")
+    T, Hk, dk = q.shape
+    _dev(k, "k", q.dtype, dev)
+    _shape(k, "k", (T, Hk, dk))
+    _dev(v, "v", q.dtype, dev)
+    if v.dim() != 3 or v.shape[0] != T:
+        raise ValueError(f"v has shape {tuple(v.shape)}, expected [{T}, Hv, dv]")
+    Hv, dv = v.shape[1], v.shape[2]
+    _shape(_dev(raw_gate, "raw_gate", torch.float32, dev), "raw_gate", (T, Hv, dk))
+    _shape(_dev(beta_logits, "beta_logits", torch.float32, dev), "beta_logits", (T, Hv))
+    _shape(_dev(a_log, "a_log", torch.float32, dev), "a_log", (Hv,))
+    _shape(_dev(dt_bias, "dt_bias", torch.float32, dev), "dt_bias", (Hv, dk))
+    _dev(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    B = cu_seqlens.numel() - 1
+    _shape(_dev(state_indices, "state_indices", torch.int32, dev), "state_indices", (B,))
+    _dev(state_pool, "state_pool", torch.float32, dev)
+    blk = (Hv, dk, dv) if state_layout == "K_FIRST" else (Hv, dv, dk)
+    if state_pool.dim() != 4 or tuple(state_pool.shape[1:]) != blk:
+        raise ValueError(f"state_pool has shape {tuple(state_pool.shape)}, expected [slots, {blk}]")
+    if output_dtype is None:
+        output_dtype = v.dtype if out is None else out.dtype
+    if output_dtype not in _DTYPES:
+        raise ValueError("output_dtype must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty((T, Hv, dv), dtype=output_dtype, device=dev)
+    _shape(_dev(out, "out", output_dtype, dev), "out", (T, Hv, dv))
+    if device_status is not None:
+        _shape(_dev(device_status, "device_status", torch.int32, dev), "device_status", (1,))
+    flags = _flags(gate_mode, beta_mode, state_layout, use_computebound, force_simt)
+    rc = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], _ptr(raw_gate), _ptr(beta_logits),
+                           _ptr(a_log), _ptr(dt_bias), _ptr(cu_seqlens), B, T, Hk, Hv, dk, dv,
+                           _ptr(state_pool), state_pool.shape[0], _ptr(state_indices), _ptr(out),
+                           _DTYPES[output_dtype], flags, float(gate_lower_bound), None, 0,
+                           _ptr(device_status), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_chunk_fwd")
+    return out
+
+
+def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, seg_offsets, initial_state,
+                                   *, M=None, U=None, incoming=None, outgoing=None, final_state=None,
+                                   scan_only=False, gate_mode="original", beta_mode="logits",
+                                   state_layout="K_FIRST", gate_lower_bound=-5.0, device_status=None,
+                                   stream=None):
+    """Segment summaries (M_i, U_i) of one sequence and the exclusive scan over them.
+
+    Returns dict(incoming_states, outgoing_states, final_state, transition_matrices,
+    local_contributions); the segment axis leads every stack.  With ``scan_only`` the given
+    M and U are inputs and are not written.
+    """
+    lib = load_library()
+    dev = initial_state.device
+    _dev(initial_state, "initial_state", torch.float32, dev)
+    Hv = initial_state.shape[0]
+    N = seg_offsets.numel() - 1
+    if scan_only:
+        if M is None or U is None:
+            raise ValueError("scan_only needs M and U")
+        dk = M.shape[-1]
+        dv = U.shape[-1] if state_layout == "K_FIRST" else U.shape[-2]
+        kv_dtype, T, Hk = _F32, 0, Hv
+    else:
+        _dev(k, "k", None, dev)
+        if k.dtype not in _DTYPES:
+            raise ValueError("k/v must be float32 or bfloat16")
+        T, Hk, dk = k.shape
+        _dev(v, "v", k.dtype, dev)
+        dv = v.shape[2]
+        _shape(v, "v", (T, Hv, dv))
+        _shape(_dev(raw_gate, "raw_gate", torch.float32, dev), "raw_gate", (T, Hv, dk))
+        _shape(_dev(beta_logits, "beta_logits", torch.float32, dev), "beta_logits", (T, Hv))
+        _shape(_dev(a_log, "a_log", torch.float32, dev), "a_log", (Hv,))
+        _shape(_dev(dt_bias, "dt_bias", torch.float32, dev), "dt_bias", (Hv, dk))
+        kv_dtype = _DTYPES[k.dtype]
+    _dev(seg_offsets, "seg_offsets", torch.int32, dev) if not scan_only else None
+    st = (dk, dv) if state_layout == "K_FIRST" else (dv, dk)
+    _shape(initial_state, "initial_state", (Hv, *st))
+
+    def buf(t, name, shape):
+        if t is None:
+            return torch.empty(shape, dtype=torch.float32, device=dev)
+        _shape(_dev(t, name, torch.float32, dev), name, shape)
+        return t
+
+    M = buf(M, "M", (N, Hv, dk, dk))
+    U = buf(U, "U", (N, Hv, *st))
+    incoming = buf(incoming, "incoming", (N, Hv, *st))
+    outgoing = buf(outgoing, "outgoing", (N, Hv, *st))
+    final_state = buf(final_state, "final_state", (Hv, *st))
+    flags = _flags(gate_mode, beta_mode, state_layout, scan_only=scan_only)
+    rc = lib.kda_segment_summarize_and_scan(
+        _ptr(k) if not scan_only else None, _ptr(v) if not scan_only else None, kv_dtype,
+        _ptr(raw_gate) if not scan_only else None, _ptr(beta_logits) if not scan_only else None,
+        _ptr(a_log) if not scan_only else None, _ptr(dt_bias) if not scan_only else None, T, Hk, Hv, dk, dv,
+        _ptr(seg_offsets) if not scan_only else None, N, _ptr(initial_state), _ptr(M), _ptr(U),
+        _ptr(incoming), _ptr(outgoing), _ptr(final_state), flags, float(gate_lower_bound), None, 0,
+        _ptr(device_status), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_segment_summarize_and_scan")
+    return {"incoming_states": incoming, "outgoing_states": outgoing, "final_state": final_state,
+            "transition_matrices": M, "local_contributions": U}
+
+
+def kda_context_parallel(transition_matrices, local_contributions, initial_state, *, state_layout="K_FIRST",
+                         stream=None):
+    """The exclusive affine scan alone ("KDA Context Parallelism", Requirements).
+
+    transition_matrices (N, dk, dk), local_contributions (N, dk, dv), initial_state (dk, dv),
+    fp32 CUDA tensors (a leading head axis after N is also accepted).  Returns a dict with
+    exactly incoming_states, outgoing_states and final_state; no input is written.
+    """
+    M, U, S0 = transition_matrices, local_contributions, initial_state
+    if M.dtype != torch.float32:
+        raise ValueError("the scan kernel computes in float32; pass float32 tensors")
+    if M.dim() < 3:
+        raise ValueError("at least one segment is required: transition_matrices is (N, dk, dk)")
+    squeeze = M.dim() == 3
+    if squeeze:
+        M, U, S0 = M.unsqueeze(1), U.unsqueeze(1), S0.unsqueeze(0)
+    if M.shape[0] < 1:
+        raise ValueError("at least one segment is required")
+    res = kda_segment_summarize_and_scan(None, None, None, None, None, None,
+                                         torch.zeros(M.shape[0] + 1, dtype=torch.int32), S0.contiguous(),
+                                         M=M.contiguous(), U=U.contiguous(), scan_only=True,
+                                         state_layout=state_layout, stream=stream)
+    out = {k: res[k] for k in ("incoming_states", "outgoing_states", "final_state")}
+    if squeeze:
+        out = {"incoming_states": out["incoming_states"][:, 0], "outgoing_states": out["outgoing_states"][:, 0],
+               "final_state": out["final_state"][0]}
+    return out

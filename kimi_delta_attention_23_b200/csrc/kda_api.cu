@@ -1,0 +1,209 @@
+// kda_api.cu -- the C ABI (include/kda.h): host-side validation and kernel dispatch.
+//
+// Shapes, flags and the state pool follow "max.nn.state_space.kda_chunk" (Parameters, Returns,
+// Raises): a dtype grouping that binds no kernel, or ranks/extents that disagree, is an error.
+// Unlike that op, whose shape guards are debug-only, every check here is always on.
+#include <cuda_runtime.h>
+
+#include "../../include/kda.h"
+#include "kda_internal.h"
+
+namespace kda {
+cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream);
+bool fused_available();
+}  // namespace kda
+
+namespace {
+
+constexpr uint32_t kKnownFlags = KDA_GATE_SAFE | KDA_BETA_PROB | KDA_STATE_V_FIRST | KDA_FUSED |
+                                 KDA_SEG_SCAN_ONLY | KDA_FORCE_SIMT;
+
+bool dtype_ok(kda_dtype_t t) { return t == KDA_F32 || t == KDA_BF16; }
+
+}  // namespace
+
+extern "C" kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,
+                                      const float* raw_gate, const float* beta_logits, const float* a_log,
+                                      const float* dt_bias, const int32_t* cu_seqlens, int32_t batch,
+                                      int64_t total_tokens, int32_t num_k_heads, int32_t num_v_heads,
+                                      int32_t dk, int32_t dv, float* state_pool, int32_t max_slots,
+                                      const int32_t* state_indices, void* out, kda_dtype_t out_dtype,
+                                      uint32_t flags, float gate_lower_bound, void* workspace,
+                                      size_t workspace_bytes, int32_t* device_status, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (batch < 0 || total_tokens < 0 || num_k_heads <= 0 || num_v_heads <= 0 || dk <= 0 || dv <= 0 ||
+      max_slots <= 0)
+    return KDA_ERR_INVALID_ARG;
+  if (num_v_heads % num_k_heads != 0) return KDA_ERR_INVALID_ARG;
+  if ((flags & ~kKnownFlags) != 0 || (flags & KDA_SEG_SCAN_ONLY)) return KDA_ERR_INVALID_ARG;
+  if (!cu_seqlens || !state_pool || !state_indices) return KDA_ERR_INVALID_ARG;
+  if (total_tokens > 0 && (!q || !k || !v || !raw_gate || !beta_logits || !out)) return KDA_ERR_INVALID_ARG;
+  if (!a_log || !dt_bias) return KDA_ERR_INVALID_ARG;
+  if (!dtype_ok(qkv_dtype) || !dtype_ok(out_dtype)) return KDA_ERR_UNSUPPORTED;
+  if (batch == 0) return KDA_OK;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf16 = qkv_dtype == KDA_BF16;
+  const bool use_fused = bf16 && !(flags & KDA_FORCE_SIMT) && dk == 128 && dv == 128 && kda::fused_available();
+  if (!use_fused) {
+    if (dk > 128 || dv > 128) return KDA_ERR_UNSUPPORTED;
+    if (!bf16 && out_dtype != KDA_F32) return KDA_ERR_UNSUPPORTED;
+    if (bf16 && !(flags & KDA_FORCE_SIMT) && (dk != 128 || dv != 128)) return KDA_ERR_UNSUPPORTED;
+    kda::SimtArgs a{};
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.in_bf16 = bf16;
+    a.raw_gate = raw_gate;
+    a.beta = beta_logits;
+    a.a_log = a_log;
+    a.dt_bias = dt_bias;
+    a.cu = cu_seqlens;
+    a.batch = batch;
+    a.total_tokens = total_tokens;
+    a.Hk = num_k_heads;
+    a.Hv = num_v_heads;
+    a.dk = dk;
+    a.w = dv;
+    a.dv_in = dv;
+    a.state_in = state_pool;
+    a.state_out = state_pool;
+    a.max_slots = max_slots;
+    a.slots = state_indices;
+    a.v_first = (flags & KDA_STATE_V_FIRST) ? 1 : 0;
+    a.init_mode = 0;
+    a.values_zero = 0;
+    a.out = out;
+    a.out_bf16 = out_dtype == KDA_BF16;
+    a.flags = flags;
+    a.lb = gate_lower_bound;
+    a.status = device_status;
+    return kda::launch_simt_chunk(a, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  }
+  kda::FusedArgs f{};
+  f.q = q;
+  f.k = k;
+  f.v = v;
+  f.raw_gate = raw_gate;
+  f.beta = beta_logits;
+  f.a_log = a_log;
+  f.dt_bias = dt_bias;
+  f.cu = cu_seqlens;
+  f.batch = batch;
+  f.total_tokens = total_tokens;
+  f.Hk = num_k_heads;
+  f.Hv = num_v_heads;
+  f.state = state_pool;
+  f.max_slots = max_slots;
+  f.slots = state_indices;
+  f.v_first = (flags & KDA_STATE_V_FIRST) ? 1 : 0;
+  f.out = out;
+  f.out_bf16 = out_dtype == KDA_BF16;
+  f.flags = flags;
+  f.lb = gate_lower_bound;
+  f.status = device_status;
+  return kda::launch_fused_chunk(f, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" kda_status_t kda_segment_summarize_and_scan(
+    const void* k, const void* v, kda_dtype_t kv_dtype, const float* raw_gate, const float* beta_logits,
+    const float* a_log, const float* dt_bias, int64_t T, int32_t num_k_heads, int32_t num_v_heads,
+    int32_t dk, int32_t dv, const int32_t* seg_offsets, int32_t num_segments, const float* initial_state,
+    float* M, float* U, float* incoming, float* outgoing, float* final_state, uint32_t flags,
+    float gate_lower_bound, void* workspace, size_t workspace_bytes, int32_t* device_status,
+    void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (num_segments < 1 || num_v_heads <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+  if ((flags & ~kKnownFlags) != 0) return KDA_ERR_INVALID_ARG;
+  if (!initial_state || !M || !U || !incoming || !outgoing || !final_state) return KDA_ERR_INVALID_ARG;
+  if (dk > 128 || dv > 128) return KDA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int v_first = (flags & KDA_STATE_V_FIRST) ? 1 : 0;
+  if (!(flags & KDA_SEG_SCAN_ONLY)) {
+    if (T < 0 || num_k_heads <= 0 || num_v_heads % num_k_heads != 0) return KDA_ERR_INVALID_ARG;
+    if (!seg_offsets || !a_log || !dt_bias) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && (!k || !v || !raw_gate || !beta_logits)) return KDA_ERR_INVALID_ARG;
+    if (!dtype_ok(kv_dtype)) return KDA_ERR_UNSUPPORTED;
+    kda::SimtArgs a{};
+    a.q = nullptr;
+    a.k = k;
+    a.v = v;
+    a.in_bf16 = kv_dtype == KDA_BF16;
+    a.raw_gate = raw_gate;
+    a.beta = beta_logits;
+    a.a_log = a_log;
+    a.dt_bias = dt_bias;
+    a.cu = seg_offsets;
+    a.batch = num_segments;
+    a.total_tokens = T;
+    a.Hk = num_k_heads;
+    a.Hv = num_v_heads;
+    a.dk = dk;
+    a.dv_in = dv;
+    a.max_slots = num_segments;
+    a.slots = nullptr;
+    a.out = nullptr;
+    a.flags = flags;
+    a.lb = gate_lower_bound;
+    a.status = device_status;
+    // transition M_i: state started at I (width dk), zero values, stored row-major
+    a.w = dk;
+    a.state_in = nullptr;
+    a.state_out = M;
+    a.v_first = 0;
+    a.init_mode = 2;
+    a.values_zero = 1;
+    if (kda::launch_simt_chunk(a, s) != cudaSuccess) return KDA_ERR_CUDA;
+    // local contribution U_i: state started at 0, real values, stored in the state layout
+    a.w = dv;
+    a.state_out = U;
+    a.v_first = v_first;
+    a.init_mode = 1;
+    a.values_zero = 0;
+    if (kda::launch_simt_chunk(a, s) != cudaSuccess) return KDA_ERR_CUDA;
+  }
+  kda::ScanArgs sa{};
+  sa.M = M;
+  sa.U = U;
+  sa.initial = initial_state;
+  sa.N = num_segments;
+  sa.H = num_v_heads;
+  sa.dk = dk;
+  sa.dv = dv;
+  sa.v_first = v_first;
+  sa.incoming = incoming;
+  sa.outgoing = outgoing;
+  sa.final_state = final_state;
+  return kda::launch_affine_scan(sa, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" size_t kda_workspace_size(int64_t total_tokens, int32_t batch, int32_t num_k_heads,
+                                     int32_t num_v_heads, int32_t dk, int32_t dv, int32_t num_segments,
+                                     uint32_t flags) {
+  (void)total_tokens;
+  (void)batch;
+  (void)num_k_heads;
+  (void)num_v_heads;
+  (void)dk;
+  (void)dv;
+  (void)num_segments;
+  (void)flags;
+  return 0;
+}
+
+extern "C" const char* kda_status_string(kda_status_t status) {
+  switch (status) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: null pointer, bad extent or bad flags";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: dtype grouping or head dims bind no kernel";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA runtime call failed";
+    case KDA_ERR_DEVICE_CHECK: return "KDA_ERR_DEVICE_CHECK: bad state slot or decreasing offsets";
+    case KDA_ERR_DEVICE_TIMEOUT: return "KDA_ERR_DEVICE_TIMEOUT: a bounded device wait gave up";
+  }
+  return "KDA_ERR_UNKNOWN";
+}
+
+extern "C" int32_t kda_version(void) { return 100; }

@@ -1,0 +1,78 @@
+// kda_internal.h -- launch arguments and launchers shared between the C-ABI layer and kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kda {
+
+// fp32 CUDA-core chunk kernel.  One block per (sequence, value head).
+struct SimtArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int32_t in_bf16;
+  const float* raw_gate;
+  const float* beta;
+  const float* a_log;
+  const float* dt_bias;
+  const int32_t* cu;        // [batch+1]
+  int32_t batch;
+  int64_t total_tokens;
+  int32_t Hk, Hv, dk;
+  int32_t w;                // state width (value columns carried by the state)
+  int32_t dv_in;            // row length of v
+  const float* state_in;    // read when init_mode == 0
+  float* state_out;         // final state destination (may equal state_in)
+  int32_t max_slots;
+  const int32_t* slots;     // [batch] or NULL (slot = sequence index)
+  int32_t v_first;          // state blocks stored transposed ([w][dk])
+  int32_t init_mode;        // 0: state_in slot, 1: zero, 2: identity
+  int32_t values_zero;      // 1: all values are zero (transition build)
+  void* out;                // [T,Hv,w] or NULL
+  int32_t out_bf16;
+  uint32_t flags;
+  float lb;
+  int32_t* status;
+};
+
+struct ScanArgs {
+  const float* M;
+  const float* U;
+  const float* initial;
+  int32_t N, H, dk, dv, v_first;
+  float* incoming;
+  float* outgoing;
+  float* final_state;
+};
+
+// Fused tensor-core chunk kernel (bf16 q/k/v, dk = dv = 128).
+struct FusedArgs {
+  const void* q;            // bf16 [T,Hk,128]
+  const void* k;            // bf16 [T,Hk,128]
+  const void* v;            // bf16 [T,Hv,128]
+  const float* raw_gate;
+  const float* beta;
+  const float* a_log;
+  const float* dt_bias;
+  const int32_t* cu;
+  int32_t batch;
+  int64_t total_tokens;
+  int32_t Hk, Hv;
+  float* state;             // pool base (read + written in place)
+  int32_t max_slots;
+  const int32_t* slots;
+  int32_t v_first;
+  void* out;
+  int32_t out_bf16;
+  uint32_t flags;
+  float lb;
+  int32_t* status;
+};
+
+size_t simt_smem_bytes(int dk, int w);
+cudaError_t launch_simt_chunk(const SimtArgs& a, cudaStream_t stream);
+cudaError_t launch_affine_scan(const ScanArgs& a, cudaStream_t stream);
+
+}  // namespace kda

@@ -1,0 +1,106 @@
+"""The C-ABI library loads here (no GPU) and exports every symbol include/kda.h declares; host-side
+argument checks return their error codes before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kimi_delta_attention_23_b200 as kda
+from kimi_delta_attention_23_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda.load_library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"KDA_API\s+[\w\s\*]+?\b(kda_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_symbols())
+    assert {"kda_chunk_fwd", "kda_segment_summarize_and_scan", "kda_workspace_size", "kda_status_string",
+            "kda_version"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {kda.LIB_PATH}").read()
+    exported = set(re.findall(r"\bT (kda_\w+)", out))
+    assert set(declared_symbols()) <= exported
+
+
+def test_status_strings_and_version(lib):
+    for code in range(7):
+        s = kda.kda_status_string(code)
+        assert s.startswith("KDA_")
+    assert kda.kda_status_string(99) == "KDA_ERR_UNKNOWN"
+    assert lib.kda_version() >= 100
+    assert kda.kda_workspace_size(1000, 2, 4, 4, 128, 128) == 0
+
+
+def _chunk(lib, **over):
+    args = dict(q=1, k=1, v=1, qkv=1, raw=1, beta=1, a_log=1, dt_bias=1, cu=1, batch=1, T=16, Hk=2, Hv=4,
+                dk=128, dv=128, pool=1, slots=4, idx=1, out=1, out_dtype=1, flags=0)
+    args.update(over)
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731  (never dereferenced: checks fail first)
+    return lib.kda_chunk_fwd(p(args["q"]), p(args["k"]), p(args["v"]), args["qkv"], p(args["raw"]),
+                             p(args["beta"]), p(args["a_log"]), p(args["dt_bias"]), p(args["cu"]), args["batch"],
+                             args["T"], args["Hk"], args["Hv"], args["dk"], args["dv"], p(args["pool"]),
+                             args["slots"], p(args["idx"]), p(args["out"]), args["out_dtype"], args["flags"],
+                             -5.0, None, 0, None, None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(batch=-1), 1), (dict(T=-3), 1), (dict(Hk=0), 1), (dict(Hv=5), 1), (dict(dk=0), 1),
+    (dict(slots=0), 1), (dict(flags=1 << 12), 1), (dict(flags=kda.SEG_SCAN_ONLY), 1), (dict(q=0), 1),
+    (dict(pool=0), 1), (dict(idx=0), 1), (dict(cu=0), 1), (dict(out=0), 1), (dict(a_log=0), 1),
+    (dict(qkv=7), 2), (dict(out_dtype=9), 2),
+    (dict(qkv=0, out_dtype=1, Hv=2, Hk=2, dk=16, dv=16), 2),       # fp32 inputs need fp32 output
+    (dict(qkv=0, out_dtype=0, dk=256, dv=16, Hv=2, Hk=2), 2),      # head dims beyond the kernels
+    (dict(dk=64, dv=128), 2),                                       # bf16 fast path is dk = dv = 128
+])
+def test_chunk_fwd_host_checks(lib, over, code):
+    assert _chunk(lib, **over) == code
+
+
+def test_empty_batch_is_a_no_op(lib):
+    assert _chunk(lib, batch=0, T=0) == 0
+
+
+def _seg(lib, **over):
+    args = dict(k=1, v=1, kv=1, raw=1, beta=1, a_log=1, dt_bias=1, T=64, Hk=2, Hv=2, dk=128, dv=128, offs=1,
+                N=4, init=1, M=1, U=1, inc=1, outg=1, fin=1, flags=0)
+    args.update(over)
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
+    return lib.kda_segment_summarize_and_scan(
+        p(args["k"]), p(args["v"]), args["kv"], p(args["raw"]), p(args["beta"]), p(args["a_log"]),
+        p(args["dt_bias"]), args["T"], args["Hk"], args["Hv"], args["dk"], args["dv"], p(args["offs"]),
+        args["N"], p(args["init"]), p(args["M"]), p(args["U"]), p(args["inc"]), p(args["outg"]),
+        p(args["fin"]), args["flags"], -5.0, None, 0, None, None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(N=0), 1), (dict(Hv=0), 1), (dict(init=0), 1), (dict(M=0), 1), (dict(U=0), 1), (dict(inc=0), 1),
+    (dict(outg=0), 1), (dict(fin=0), 1), (dict(flags=1 << 20), 1), (dict(offs=0), 1), (dict(k=0), 1),
+    (dict(Hk=3), 1), (dict(dk=129), 2), (dict(kv=5), 2),
+])
+def test_segment_host_checks(lib, over, code):
+    assert _seg(lib, **over) == code
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    w = torch.zeros(4, 1, 16)
+    with pytest.raises(ValueError, match="CUDA"):
+        kda.kda_chunk_fwd(w, w, w, torch.zeros(4, 1, 16), torch.zeros(4, 1), torch.zeros(1), torch.zeros(1, 16),
+                          torch.zeros(2, dtype=torch.int32), torch.zeros(1, 1, 16, 16),
+                          torch.zeros(1, dtype=torch.int32))
