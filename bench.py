@@ -118,13 +118,21 @@ class ClockSampler:
         self.path = os.path.join("/tmp", f"kda_clocks_{os.getpid()}.csv")
         sel = []
         try:
-            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
-            sel = ["-i", bus] if bus else []
+            pr = torch.cuda.get_device_properties(device_index)
+            sel = ["-i", "%08X:%02X:%02X.0" % (int(pr.pci_domain_id), int(pr.pci_bus_id), int(pr.pci_device_id))]
         except Exception:
             sel = []
         self.cmd = ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
 
     def __enter__(self):
+        if len(self.cmd) > 2 and self.cmd[1] == "-i":
+            try:
+                r = subprocess.run(["nvidia-smi", "-i", self.cmd[2], "--query-gpu=index", "--format=csv,noheader"],
+                                   capture_output=True, text=True, timeout=20)
+                if r.returncode != 0 or not r.stdout.strip():
+                    self.cmd = [self.cmd[0]] + self.cmd[3:]
+            except Exception:
+                self.cmd = [self.cmd[0]] + self.cmd[3:]
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(self.cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
