@@ -20,6 +20,8 @@ constexpr uint32_t kKnownFlags = KDA_GATE_SAFE | KDA_BETA_PROB | KDA_STATE_V_FIR
 
 bool dtype_ok(kda_dtype_t t) { return t == KDA_F32 || t == KDA_BF16; }
 
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 }  // namespace
 
 extern "C" kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,
@@ -81,6 +83,9 @@ extern "C" kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* 
     a.status = device_status;
     return kda::launch_simt_chunk(a, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
   }
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(raw_gate) || !aligned16(dt_bias) ||
+      !aligned16(state_pool) || !aligned16(out))
+    return KDA_ERR_INVALID_ARG;
   kda::FusedArgs f{};
   f.q = q;
   f.k = k;
@@ -94,10 +99,13 @@ extern "C" kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* 
   f.total_tokens = total_tokens;
   f.Hk = num_k_heads;
   f.Hv = num_v_heads;
-  f.state = state_pool;
+  f.state_in = state_pool;
+  f.state_out = state_pool;
   f.max_slots = max_slots;
   f.slots = state_indices;
   f.v_first = (flags & KDA_STATE_V_FIRST) ? 1 : 0;
+  f.init_mode = 0;
+  f.values_zero = 0;
   f.out = out;
   f.out_bf16 = out_dtype == KDA_BF16;
   f.flags = flags;
@@ -126,43 +134,85 @@ extern "C" kda_status_t kda_segment_summarize_and_scan(
     if (!seg_offsets || !a_log || !dt_bias) return KDA_ERR_INVALID_ARG;
     if (T > 0 && (!k || !v || !raw_gate || !beta_logits)) return KDA_ERR_INVALID_ARG;
     if (!dtype_ok(kv_dtype)) return KDA_ERR_UNSUPPORTED;
-    kda::SimtArgs a{};
-    a.q = nullptr;
-    a.k = k;
-    a.v = v;
-    a.in_bf16 = kv_dtype == KDA_BF16;
-    a.raw_gate = raw_gate;
-    a.beta = beta_logits;
-    a.a_log = a_log;
-    a.dt_bias = dt_bias;
-    a.cu = seg_offsets;
-    a.batch = num_segments;
-    a.total_tokens = T;
-    a.Hk = num_k_heads;
-    a.Hv = num_v_heads;
-    a.dk = dk;
-    a.dv_in = dv;
-    a.max_slots = num_segments;
-    a.slots = nullptr;
-    a.out = nullptr;
-    a.flags = flags;
-    a.lb = gate_lower_bound;
-    a.status = device_status;
-    // transition M_i: state started at I (width dk), zero values, stored row-major
-    a.w = dk;
-    a.state_in = nullptr;
-    a.state_out = M;
-    a.v_first = 0;
-    a.init_mode = 2;
-    a.values_zero = 1;
-    if (kda::launch_simt_chunk(a, s) != cudaSuccess) return KDA_ERR_CUDA;
-    // local contribution U_i: state started at 0, real values, stored in the state layout
-    a.w = dv;
-    a.state_out = U;
-    a.v_first = v_first;
-    a.init_mode = 1;
-    a.values_zero = 0;
-    if (kda::launch_simt_chunk(a, s) != cudaSuccess) return KDA_ERR_CUDA;
+    const bool use_fused = kv_dtype == KDA_BF16 && !(flags & KDA_FORCE_SIMT) && dk == 128 && dv == 128 &&
+                           kda::fused_available();
+    if (use_fused) {
+      if (!aligned16(k) || !aligned16(v) || !aligned16(raw_gate) || !aligned16(dt_bias) || !aligned16(M) ||
+          !aligned16(U))
+        return KDA_ERR_INVALID_ARG;
+      kda::FusedArgs f{};
+      f.q = nullptr;
+      f.k = k;
+      f.v = v;
+      f.raw_gate = raw_gate;
+      f.beta = beta_logits;
+      f.a_log = a_log;
+      f.dt_bias = dt_bias;
+      f.cu = seg_offsets;
+      f.batch = num_segments;
+      f.total_tokens = T;
+      f.Hk = num_k_heads;
+      f.Hv = num_v_heads;
+      f.max_slots = num_segments;
+      f.slots = nullptr;
+      f.out = nullptr;
+      f.out_bf16 = 0;
+      f.flags = flags;
+      f.lb = gate_lower_bound;
+      f.status = device_status;
+      f.state_in = nullptr;
+      // transition M_i: from I with zero values, stored row-major
+      f.state_out = M;
+      f.v_first = 0;
+      f.init_mode = 2;
+      f.values_zero = 1;
+      if (kda::launch_fused_chunk(f, s) != cudaSuccess) return KDA_ERR_CUDA;
+      // contribution U_i: from 0 with the real values, stored in the state layout
+      f.state_out = U;
+      f.v_first = v_first;
+      f.init_mode = 1;
+      f.values_zero = 0;
+      if (kda::launch_fused_chunk(f, s) != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    if (!use_fused) {
+      kda::SimtArgs a{};
+      a.q = nullptr;
+      a.k = k;
+      a.v = v;
+      a.in_bf16 = kv_dtype == KDA_BF16;
+      a.raw_gate = raw_gate;
+      a.beta = beta_logits;
+      a.a_log = a_log;
+      a.dt_bias = dt_bias;
+      a.cu = seg_offsets;
+      a.batch = num_segments;
+      a.total_tokens = T;
+      a.Hk = num_k_heads;
+      a.Hv = num_v_heads;
+      a.dk = dk;
+      a.dv_in = dv;
+      a.max_slots = num_segments;
+      a.slots = nullptr;
+      a.out = nullptr;
+      a.flags = flags;
+      a.lb = gate_lower_bound;
+      a.status = device_status;
+      // transition M_i: state started at I (width dk), zero values, stored row-major
+      a.w = dk;
+      a.state_in = nullptr;
+      a.state_out = M;
+      a.v_first = 0;
+      a.init_mode = 2;
+      a.values_zero = 1;
+      if (kda::launch_simt_chunk(a, s) != cudaSuccess) return KDA_ERR_CUDA;
+      // local contribution U_i: state started at 0, real values, stored in the state layout
+      a.w = dv;
+      a.state_out = U;
+      a.v_first = v_first;
+      a.init_mode = 1;
+      a.values_zero = 0;
+      if (kda::launch_simt_chunk(a, s) != cudaSuccess) return KDA_ERR_CUDA;
+    }
   }
   kda::ScanArgs sa{};
   sa.M = M;

@@ -60,11 +60,14 @@ struct FusedArgs {
   int32_t batch;
   int64_t total_tokens;
   int32_t Hk, Hv;
-  float* state;             // pool base (read + written in place)
+  const float* state_in;    // read when init_mode == 0 (pool base)
+  float* state_out;         // final state destination (pool base; may equal state_in)
   int32_t max_slots;
-  const int32_t* slots;
-  int32_t v_first;
-  void* out;
+  const int32_t* slots;     // [batch] or NULL (slot = sequence index)
+  int32_t v_first;          // state blocks stored transposed ([dv][dk])
+  int32_t init_mode;        // 0: state_in slot, 1: zero, 2: identity
+  int32_t values_zero;      // 1: all values are zero (transition build)
+  void* out;                // [T,Hv,128] or NULL (no readout)
   int32_t out_bf16;
   uint32_t flags;
   float lb;

@@ -1,0 +1,130 @@
+"""GPU parity of the segment summaries, the exclusive scan and the context-parallel prefill.
+
+Against the fp64 oracle: M_i (recurrence from I with zero values), U_i (recurrence from 0),
+the scan's incoming / outgoing / final states, and the second pass (every segment as its own
+sequence, starting from its incoming state) against the straight token-by-token recurrence.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import kda_workloads as W
+import kimi_delta_attention_23_b200 as kda
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rel_l2(x, ref):
+    x = x.double().cpu().numpy() if isinstance(x, torch.Tensor) else np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    n = np.linalg.norm(ref)
+    return float(np.linalg.norm(x - ref) / (n if n > 0 else 1.0))
+
+
+def test_scalar_three_segment_example_on_gpu():
+    with open(os.path.join(GOLD, "scalar_three_segments.json")) as f:
+        g = json.load(f)
+    M = torch.tensor([[[m]] for m, _ in g["maps"]], dtype=torch.float32, device="cuda")
+    U = torch.tensor([[[u]] for _, u in g["maps"]], dtype=torch.float32, device="cuda")
+    S0 = torch.tensor([[g["initial_state"]]], dtype=torch.float32, device="cuda")
+    copies = [t.clone() for t in (M, U, S0)]
+    res = kda.kda_context_parallel(M, U, S0)
+    torch.cuda.synchronize()
+    assert set(res) == {"incoming_states", "outgoing_states", "final_state"}
+    assert res["incoming_states"].flatten().tolist() == g["incoming_states"]
+    assert res["outgoing_states"].flatten().tolist() == g["outgoing_states"]
+    assert res["final_state"].item() == g["final_state"]
+    assert res["final_state"].dtype == torch.float32 and res["final_state"].device.type == "cuda"
+    for t, c in zip((M, U, S0), copies):
+        assert torch.equal(t, c)
+
+
+def test_scan_only_matches_oracle_scan():
+    rng = np.random.default_rng(0)
+    N, H, dk, dv = 5, 3, 128, 128
+    M = rng.normal(size=(N, H, dk, dk)) / np.sqrt(dk)
+    U = rng.normal(size=(N, H, dk, dv))
+    S0 = rng.normal(size=(H, dk, dv))
+    ref = oracle.kda_affine_scan(M, U, S0)
+    cu = lambda x: torch.tensor(x, dtype=torch.float32, device="cuda")  # noqa: E731
+    res = kda.kda_context_parallel(cu(M), cu(U), cu(S0))
+    for key in ref:
+        assert rel_l2(res[key], ref[key]) < 1e-5, key
+
+
+CASES = [
+    (torch.float32, 16, "K_FIRST", 1e-4),
+    (torch.float32, 32, "V_FIRST", 1e-4),
+    (torch.bfloat16, 128, "K_FIRST", 1e-2),
+    (torch.bfloat16, 128, "V_FIRST", 1e-2),
+]
+
+
+@pytest.mark.parametrize("dtype,d,layout,tol", CASES)
+def test_segment_summaries_and_scan(dtype, d, layout, tol):
+    T = 300
+    w = W.random_inputs([T], 2, 2, d, d, seed=d, qkv_dtype=dtype, state_std=0.2, state_layout=layout,
+                        output_dtype=dtype)
+    offs = torch.tensor([0, 37, 100, 164, 300], dtype=torch.int32)
+    wd = w.to("cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    res = kda.kda_segment_summarize_and_scan(wd.k, wd.v, wd.raw_gate, wd.beta_logits, wd.a_log, wd.dt_bias,
+                                             offs.cuda(), wd.state_pool[0].contiguous(), state_layout=layout,
+                                             device_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    M, U = oracle.kda_segment_summary(w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, offs,
+                                      state_layout=layout)
+    ref = oracle.kda_affine_scan(M, U, w.state_pool[0], state_layout=layout)
+    assert rel_l2(res["transition_matrices"], M) < tol
+    assert rel_l2(res["local_contributions"], U) < tol
+    assert rel_l2(res["incoming_states"], ref["incoming_states"]) < tol
+    assert rel_l2(res["outgoing_states"], ref["outgoing_states"]) < tol
+    assert rel_l2(res["final_state"], ref["final_state"]) < tol
+
+
+def _cp_prefill(wd, offs, init, layout="K_FIRST", gate_mode="original", lb=-5.0):
+    N = offs.numel() - 1
+    res = kda.kda_segment_summarize_and_scan(wd.k, wd.v, wd.raw_gate, wd.beta_logits, wd.a_log, wd.dt_bias, offs,
+                                             init, state_layout=layout, gate_mode=gate_mode, gate_lower_bound=lb)
+    pool = res["incoming_states"].clone()
+    out = kda.kda_chunk_fwd(wd.q, wd.k, wd.v, wd.raw_gate, wd.beta_logits, wd.a_log, wd.dt_bias, offs, pool,
+                            torch.arange(N, dtype=torch.int32, device=wd.q.device), state_layout=layout,
+                            gate_mode=gate_mode, gate_lower_bound=lb)
+    torch.cuda.synchronize()
+    return out, pool, res
+
+
+@pytest.mark.parametrize("layout", ["K_FIRST", "V_FIRST"])
+def test_context_parallel_prefill_matches_straight_recurrence(layout):
+    w = W.random_inputs([1000], 2, 2, 128, 128, seed=3, state_std=0.1, state_layout=layout)
+    wd = w.to("cuda")
+    offs = torch.tensor([0, 250, 500, 777, 1000], dtype=torch.int32, device="cuda")
+    out, pool, res = _cp_prefill(wd, offs, wd.state_pool[0].contiguous(), layout)
+    o_ref, p_ref = oracle.kda_forward(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens,
+                                      w.state_pool, w.state_indices, state_layout=layout)
+    assert rel_l2(out, o_ref) < 1e-2
+    assert rel_l2(res["final_state"], p_ref[0]) < 1e-2
+    assert rel_l2(pool[-1], p_ref[0]) < 1e-2
+    # the second pass ends every segment in the scan's outgoing state
+    assert rel_l2(pool, res["outgoing_states"].double().cpu().numpy()) < 1e-2
+
+
+def test_full_size_context_parallel_sampled_heads():
+    """The benchmark's launch configuration: 131072 tokens, 32 heads, 16 segments of 8192."""
+    w = W.make("long_T131072_H32_cp16", device="cuda")
+    out, pool, res = _cp_prefill(w, w.seg_offsets, w.state_pool[0])
+    heads = [2, 21]
+    cpu = lambda t: t.detach().cpu()  # noqa: E731
+    o_ref, p_ref = oracle.kda_forward(cpu(w.q)[:, heads], cpu(w.k)[:, heads], cpu(w.v)[:, heads],
+                                      cpu(w.raw_gate)[:, heads], cpu(w.beta_logits)[:, heads], cpu(w.a_log)[heads],
+                                      cpu(w.dt_bias)[heads], cpu(w.cu_seqlens), cpu(w.state_pool)[:, heads],
+                                      cpu(w.state_indices))
+    assert rel_l2(out[:, heads], o_ref) < 1e-2
+    assert rel_l2(res["final_state"][heads], p_ref[0]) < 1e-2
