@@ -28,6 +28,9 @@
 //     D1o += Delta^T P^T, S^T += Delta^T K'.  S^T stays in TMEM in fp32 across chunks; a bf16
 //     copy in shared memory is the A operand of the next chunk's first product.  Warps 0-3
 //     (one per TMEM lane quadrant) run the epilogues; thread 128 issues the MMAs.
+#include <cuda.h>
+#include <string.h>
+
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_sm100.cuh"
@@ -41,6 +44,7 @@ constexpr int C = 64;          // chunk length
 constexpr int D = 128;         // dk = dv
 constexpr int kThreads = 256;
 constexpr int kMmaThread = 128;
+constexpr int kPfThread = 160;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far beyond any legitimate wait
 
@@ -68,7 +72,12 @@ constexpr int OFF_BAR = OFF_GC + 512;       // 4 mbarriers, TMEM base, abort fla
 constexpr int kSmemBytes = OFF_BAR + 64;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for aligning the base to 1024
 constexpr int OFF_XI = OFF_KPI;             // fp32 [64][68] inverse (after the scores are done)
-constexpr int OFF_Y = OFF_KPI8;             // fp32 [3][16][16] inverse temporaries
+constexpr int OFF_Y = OFF_KPI8;             // fp32 inverse temporaries: [2][16][16] then [32][32]
+// inputs of the next chunk land here (bulk async copies issued during the state phase, when the
+// score scratch above is dead): raw gate fp32 [64][128], then k, q, v bf16 [64][128]
+constexpr int OFF_PF = OFF_KPI;
+constexpr int PF_RAW = OFF_PF, PF_K = OFF_PF + 32768, PF_Q = OFF_PF + 49152, PF_V = OFF_PF + 65536;
+static_assert(PF_V + 16384 <= OFF_TAU, "prefetch region overlaps live data");
 constexpr int kLdA = 68;                    // row stride of the fp32 [64][*] arrays
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
@@ -91,6 +100,13 @@ __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t x, float s0, float s1)
   return pack_bf16(f.x * s0, f.y * s1);
 }
 
+// slot -> (row, column) of the 8x8 diagonal-block scores: slots 0..27 are A (row > column),
+// slots 28..63 are P (row >= column); entry = row * 8 + column
+__constant__ unsigned char kDiagPair[64] = {
+    8,  16, 17, 24, 25, 26, 32, 33, 34, 35, 40, 41, 42, 43, 44, 48, 49, 50, 51, 52, 53, 56,
+    57, 58, 59, 60, 61, 62, 0,  8,  9,  16, 17, 18, 24, 25, 26, 27, 32, 33, 34, 35, 36, 40,
+    41, 42, 43, 44, 45, 48, 49, 50, 51, 52, 53, 54, 56, 57, 58, 59, 60, 61, 62, 63};
+
 // the six (row block, column block) pairs of 16-blocks below the diagonal
 __device__ __forceinline__ void pair_of(int p, int& a, int& b) {
   const int pa[6] = {1, 2, 2, 3, 3, 3};
@@ -101,7 +117,13 @@ __device__ __forceinline__ void pair_of(int p, int& a, int& b) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
+// Tensor maps of the four token-major inputs, each viewed as [tokens][heads][128] with a box of
+// 64 tokens x 1 head x 128 channels: one copy per tensor moves a whole chunk of one head.
+struct InputMaps {
+  CUtensorMap raw, k, q, v;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArgs a, const __grid_constant__ InputMaps tm) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -117,9 +139,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
   }
 
   const uint32_t sbase = smem_addr(sm);
-  const uint32_t bar0 = sbase + OFF_BAR, bar1 = bar0 + 8, bar2 = bar0 + 16, bar3 = bar0 + 24;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 32);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + OFF_BAR + 36);
+  const uint32_t bar0 = sbase + OFF_BAR, bar1 = bar0 + 8, bar2 = bar0 + 16, bar3 = bar0 + 24, bar_pf = bar0 + 32;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 40);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + OFF_BAR + 44);
   float* sA = reinterpret_cast<float*>(sm + OFF_A);
   float* sTau = reinterpret_cast<float*>(sm + OFF_TAU);
   float* sMp = reinterpret_cast<float*>(sm + OFF_MP);
@@ -131,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
     mbar_init(bar1, 1);
     mbar_init(bar2, 1);
     mbar_init(bar3, 1);
+    mbar_init(bar_pf, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -144,6 +167,24 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
   const uint32_t tmem = *s_tmem;
   const uint32_t tmD1 = tmem, tmS = tmem + 128;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+  const bool qb = a.q != nullptr;
+  // one thread copies the inputs of the chunk starting at token c0n into the prefetch region
+  // with four tensor copies (rows past the end of the tensor arrive as zeros; rows past the
+  // end of the sequence are never read); completion is counted in bytes on bar_pf
+  const uint32_t pf_bytes = 32768u + 16384u * (1u + (qb ? 1u : 0u) + (a.values_zero ? 0u : 1u));
+  auto issue_prefetch = [&](int64_t c0n) {
+    mbar_arrive_expect_tx(bar_pf, pf_bytes);
+    tma_load_3d(sbase + PF_RAW, &tm.raw, 0, h, (int)c0n, bar_pf);
+    tma_load_3d(sbase + PF_K, &tm.k, 0, kh, (int)c0n, bar_pf);
+    if (qb) tma_load_3d(sbase + PF_Q, &tm.q, 0, kh, (int)c0n, bar_pf);
+    if (!a.values_zero) tma_load_3d(sbase + PF_V, &tm.v, 0, h, (int)c0n, bar_pf);
+  };
+  bool pf_pending = false;  // a prefetch was issued and its completion not yet observed
+  uint32_t pf_parity = 0;   // parity of the next prefetch completion on bar_pf
+  if (t1 > t0) {
+    if (tid == kPfThread) issue_prefetch(t0);
+    pf_pending = true;
+  }
   const size_t blk_off = ((size_t)slot * a.Hv + h) * (size_t)(D * D);
   const float* in_blk = a.state_in ? a.state_in + blk_off : nullptr;
   float* out_blk = a.state_out + blk_off;
@@ -190,9 +231,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
   const float cexp = expf(a.a_log[h]);
   const float alpha_floor = safe ? expf(a.lb) : 0.f;
   const int b16 = warp >> 1, upper = warp & 1;
-  const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(a.q);
-  const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(a.k);
-  const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(a.v);
 
   uint32_t phase = 0;
   bool aborted = false;
@@ -200,18 +238,24 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
   for (int64_t c0 = t0; c0 < t1; c0 += C, phase ^= 1u) {
     const int L = (int)((t1 - c0) < C ? (t1 - c0) : C);
 
-    // =============================== k-side, part 1: loads, gates, in-block products
+    // =============================== k-side, part 1: gates and in-block products
+    if (mbar_wait_bounded(bar_pf, pf_parity, kWaitLimitNs)) {
+      pf_pending = false;
+      pf_parity ^= 1u;
+    } else {
+      *s_abort = 1;
+      report(a.status, KDA_ERR_DEVICE_TIMEOUT);
+    }
     float al[8][4];
     uint2 k2[8], q2[8], v2[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int row = warp * 8 + r;
       if (row < L) {
-        const size_t t = (size_t)(c0 + row);
-        const float4 raw = __ldg(reinterpret_cast<const float4*>(a.raw_gate + (t * a.Hv + h) * D + ch));
-        k2[r] = __ldg(reinterpret_cast<const uint2*>(kb + (t * a.Hk + kh) * D + ch));
-        q2[r] = qb ? __ldg(reinterpret_cast<const uint2*>(qb + (t * a.Hk + kh) * D + ch)) : make_uint2(0u, 0u);
-        v2[r] = a.values_zero ? make_uint2(0u, 0u) : __ldg(reinterpret_cast<const uint2*>(vb + (t * a.Hv + h) * D + ch));
+        const float4 raw = *reinterpret_cast<const float4*>(sm + PF_RAW + row * 512 + ch * 4);
+        k2[r] = *reinterpret_cast<const uint2*>(sm + PF_K + row * 256 + ch * 2);
+        q2[r] = qb ? *reinterpret_cast<const uint2*>(sm + PF_Q + row * 256 + ch * 2) : make_uint2(0u, 0u);
+        v2[r] = a.values_zero ? make_uint2(0u, 0u) : *reinterpret_cast<const uint2*>(sm + PF_V + row * 256 + ch * 2);
         const float xs[4] = {raw.x + dtb.x, raw.y + dtb.y, raw.z + dtb.z, raw.w + dtb.w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -233,8 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
       const int row = warp * 8 + lane;
       sBeta[row] = row < L ? beta_f32(a.beta[(size_t)(c0 + row) * a.Hv + h], prob) : 0.f;
     }
-    // zero the score buffers (their upper triangles must read as 0)
-    for (int e = tid; e < C * kLdA / 4; e += kThreads) reinterpret_cast<float4*>(sA)[e] = make_float4(0, 0, 0, 0);
+    // P's upper triangle must read as zero (A's upper triangle is never read)
     for (int e = tid; e < 8192 / 16; e += kThreads) reinterpret_cast<uint4*>(sm + OFF_P)[e] = make_uint4(0, 0, 0, 0);
     // in-block products: p8 inclusive prefix from the block start, s8 exclusive suffix
     float p8[8][4], s8[8][4];
@@ -254,7 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
       }
     }
     *reinterpret_cast<float4*>(sTau + warp * D + ch) = make_float4(p8[7][0], p8[7][1], p8[7][2], p8[7][3]);
-    __syncthreads();  // (1) block products visible; previous chunk's output flush finished
+    __syncthreads();  // (1) block products visible; prefetched inputs consumed; output flushed
+    if (*s_abort) {
+      aborted = true;
+      break;
+    }
 
     // V rows (plain row-major) for the first epilogue
 #pragma unroll
@@ -341,10 +388,18 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
         }
       }
     }
+    // the four stores rotate over the channels by lane so that each store instruction spreads
+    // its 32 rows over all eight 16-byte bank groups
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
-      *reinterpret_cast<uint4*>(sm + OFF_KPT + sw_off(ch + c, warp * 8, 128)) =
-          make_uint4(kpt[c][0], kpt[c][1], kpt[c][2], kpt[c][3]);
+    for (int cs = 0; cs < 4; ++cs) {
+      const int c = (cs + (lane >> 1)) & 3;
+      uint4 val;
+      val.x = c == 0 ? kpt[0][0] : c == 1 ? kpt[1][0] : c == 2 ? kpt[2][0] : kpt[3][0];
+      val.y = c == 0 ? kpt[0][1] : c == 1 ? kpt[1][1] : c == 2 ? kpt[2][1] : kpt[3][1];
+      val.z = c == 0 ? kpt[0][2] : c == 1 ? kpt[1][2] : c == 2 ? kpt[2][2] : kpt[3][2];
+      val.w = c == 0 ? kpt[0][3] : c == 1 ? kpt[1][3] : c == 2 ? kpt[2][3] : kpt[3][3];
+      *reinterpret_cast<uint4*>(sm + OFF_KPT + sw_off(ch + c, warp * 8, 128)) = val;
+    }
 
     // diagonal 8x8 blocks on CUDA cores: partial sums over my 4 channels of
     //   A_rs (r > s, slots 0..27) and P_rs (r >= s, slots 28..63), then a butterfly
@@ -391,18 +446,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int idx = 2 * lane + u;
-        int r, s;
+        const int rs = kDiagPair[idx], r = rs >> 3, sc = rs & 7;
         if (idx < 28) {
-          r = 1;
-          while ((r + 1) * r / 2 <= idx) ++r;
-          s = idx - r * (r - 1) / 2;
-          sA[(warp * 8 + r) * kLdA + warp * 8 + s] = acc[u];
+          sA[(warp * 8 + r) * kLdA + warp * 8 + sc] = acc[u];
         } else {
-          const int e = idx - 28;
-          r = 0;
-          while ((r + 1) * (r + 2) / 2 <= e) ++r;
-          s = e - r * (r + 1) / 2;
-          *reinterpret_cast<__nv_bfloat16*>(sm + OFF_P + sw_off(warp * 8 + r, warp * 8 + s, 64)) =
+          *reinterpret_cast<__nv_bfloat16*>(sm + OFF_P + sw_off(warp * 8 + r, warp * 8 + sc, 64)) =
               __float2bfloat16_rn(acc[u]);
         }
       }
@@ -474,11 +522,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
     __syncthreads();  // (3) A and P complete
 
     // =============================== k-side, part 3: T = (I + diag(beta) A)^{-1} diag(beta)
+    // X = (I + L)^{-1}, L = diag(beta) A strictly lower: diagonal 16-blocks by forward
+    // substitution, then two doubling levels -- X10, X32 from 16-blocks, then the lower-left
+    // 32-block -- each as X_ab = -X_aa (L_ab X_bb) over the blocks just finished.
     {
       float* Xi = reinterpret_cast<float*>(sm + OFF_XI);
-      float* Y = reinterpret_cast<float*>(sm + OFF_Y);
+      float* Y1 = reinterpret_cast<float*>(sm + OFF_Y);  // [2][16][16]
+      float* Y2 = Y1 + 512;                               // [32][32]
       if (tid < 64) {
-        // diagonal 16-blocks by forward substitution, one column per thread
         const int blk = tid >> 4, col = tid & 15, base = 16 * blk;
         float x[16];
 #pragma unroll
@@ -491,27 +542,66 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) Xi[(base + r) * kLdA + base + col] = x[r];
+        if ((blk & 1) == 0) {
+#pragma unroll
+          for (int r = 0; r < 16; ++r) Xi[(base + r) * kLdA + base + 16 + col] = 0.f;
+        }
       }
       __syncthreads();
-#pragma unroll 1
-      for (int ab = 1; ab < 4; ++ab) {
-        for (int idx = tid; idx < ab * 256; idx += kThreads) {
-          const int bb = idx >> 8, r = (idx >> 4) & 15, col = idx & 15;
-          const int R = 16 * ab + r;
-          float acc = 0.f;
-          for (int u = 16 * bb; u < 16 * ab; ++u) acc += sA[R * kLdA + u] * Xi[u * kLdA + 16 * bb + col];
-          Y[idx] = sBeta[R] * acc;
-        }
-        __syncthreads();
-        for (int idx = tid; idx < ab * 256; idx += kThreads) {
-          const int bb = idx >> 8, r = (idx >> 4) & 15, col = idx & 15;
-          float acc = 0.f;
+      {
+        // level 1: p = 0 -> X10, p = 1 -> X32; two columns per thread
+        const int p = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
+        const int ra = p ? 3 : 1, cb = 16 * (ra - 1), R = 16 * ra + r;
+        float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-          for (int u = 0; u < 16; ++u) acc += Xi[(16 * ab + r) * kLdA + 16 * ab + u] * Y[(bb << 8) + u * 16 + col];
-          Xi[(16 * ab + r) * kLdA + 16 * bb + col] = -acc;
+        for (int u = 0; u < 16; ++u) {
+          const float l = sA[R * kLdA + cb + u];
+          y0 += l * Xi[(cb + u) * kLdA + cb + c];
+          y1 += l * Xi[(cb + u) * kLdA + cb + c + 1];
         }
+        Y1[p * 256 + r * 16 + c] = sBeta[R] * y0;
+        Y1[p * 256 + r * 16 + c + 1] = sBeta[R] * y1;
         __syncthreads();
+        float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const float xr = Xi[R * kLdA + 16 * ra + u];
+          x0 += xr * Y1[p * 256 + u * 16 + c];
+          x1 += xr * Y1[p * 256 + u * 16 + c + 1];
+        }
+        Xi[R * kLdA + cb + c] = -x0;
+        Xi[R * kLdA + cb + c + 1] = -x1;
       }
+      __syncthreads();
+      {
+        // level 2: rows 32..63, columns 0..31; four columns per thread
+        const int r = tid >> 3, c = (tid & 7) * 4;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int u = 0; u < 32; ++u) {
+          const float l = sA[(32 + r) * kLdA + u];
+          const float4 xv = *reinterpret_cast<const float4*>(Xi + u * kLdA + c);
+          y[0] += l * xv.x;
+          y[1] += l * xv.y;
+          y[2] += l * xv.z;
+          y[3] += l * xv.w;
+        }
+        const float bR = sBeta[32 + r];
+        *reinterpret_cast<float4*>(Y2 + r * 32 + c) = make_float4(bR * y[0], bR * y[1], bR * y[2], bR * y[3]);
+        __syncthreads();
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int u = 0; u < 32; ++u) {
+          const float xr = Xi[(32 + r) * kLdA + 32 + u];
+          const float4 yv = *reinterpret_cast<const float4*>(Y2 + u * 32 + c);
+          x[0] += xr * yv.x;
+          x[1] += xr * yv.y;
+          x[2] += xr * yv.z;
+          x[3] += xr * yv.w;
+        }
+        *reinterpret_cast<float4*>(Xi + (32 + r) * kLdA + c) = make_float4(-x[0], -x[1], -x[2], -x[3]);
+      }
+      __syncthreads();
       // T[r][s] = X[r][s] beta_s for s <= r, else 0; bf16 tile [r][s]
       for (int idx = tid; idx < 64 * 8; idx += kThreads) {
         const int r = idx >> 3, sc = idx & 7;
@@ -528,6 +618,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
     }
     fence_async_smem();
     __syncthreads();  // (4) every operand of this chunk is in shared memory
+    if (c0 + C < t1) {
+      if (tid == kPfThread) issue_prefetch(c0 + C);
+      pf_pending = true;
+    }
 
     // =============================== state side
     // D1 = S^T [K o Gamma ; Q o Gamma]^T   (M = 128, N = 128, K = 128)
@@ -549,19 +643,18 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
       } else {
         tc_fence_after();
         // X^T[j][r] = V[r][j] - D1[j][r]
-#pragma unroll 1
-        for (int r0 = 0; r0 < C; r0 += 16) {
-          float d[16];
-          tmem_ld16(tmD1 + lane_base + r0, d);
-          tmem_wait_ld();
-          float x[16];
+        float d[64];
+        tmem_ld16n<4>(tmD1 + lane_base, d);
+        tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 16; ++u)
-            x[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_V + ((r0 + u) * D + j) * 2)) - d[u];
+        for (int r0 = 0; r0 < C; r0 += 8) {
+          float x[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            x[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_V + ((r0 + u) * D + j) * 2)) -
+                   d[r0 + u];
           *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(j, r0, 128)) =
               make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-          *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(j, r0 + 8, 128)) = make_uint4(
-              pack_bf16(x[8], x[9]), pack_bf16(x[10], x[11]), pack_bf16(x[12], x[13]), pack_bf16(x[14], x[15]));
         }
       }
       fence_async_smem();
@@ -589,25 +682,27 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
         report(a.status, KDA_ERR_DEVICE_TIMEOUT);
       } else {
         tc_fence_after();
-#pragma unroll 1
-        for (int r0 = 0; r0 < C; r0 += 16) {
-          float d[16];
-          tmem_ld16(tmD1 + lane_base + r0, d);
+        {
+          float d[64];
+          tmem_ld16n<4>(tmD1 + lane_base, d);
           tmem_wait_ld();
-          *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(j, r0, 128)) =
-              make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]), pack_bf16(d[4], d[5]), pack_bf16(d[6], d[7]));
-          *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(j, r0 + 8, 128)) = make_uint4(
-              pack_bf16(d[8], d[9]), pack_bf16(d[10], d[11]), pack_bf16(d[12], d[13]), pack_bf16(d[14], d[15]));
+#pragma unroll
+          for (int r0 = 0; r0 < C; r0 += 8)
+            *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(j, r0, 128)) =
+                make_uint4(pack_bf16(d[r0], d[r0 + 1]), pack_bf16(d[r0 + 2], d[r0 + 3]),
+                           pack_bf16(d[r0 + 4], d[r0 + 5]), pack_bf16(d[r0 + 6], d[r0 + 7]));
         }
         // decay the state columns: S^T[j][i] *= Gamma_63[i]
 #pragma unroll 1
-        for (int i0 = 0; i0 < D; i0 += 16) {
-          float sv[16];
-          tmem_ld16(tmS + lane_base + i0, sv);
+        for (int i0 = 0; i0 < D; i0 += 64) {
+          float sv[64];
+          tmem_ld16n<4>(tmS + lane_base + i0, sv);
           tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 16; ++u) sv[u] *= sGC[i0 + u];
-          tmem_st16(tmS + lane_base + i0, sv);
+          for (int u = 0; u < 64; ++u) sv[u] *= sGC[i0 + u];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            tmem_st16(tmS + lane_base + i0 + 16 * q, *reinterpret_cast<const float(*)[16]>(sv + 16 * q));
         }
         tmem_wait_st();
       }
@@ -641,31 +736,30 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
       } else {
         tc_fence_after();
         // outputs O[r][j] staged row-major (bf16 in the V region, fp32 across X..V)
-#pragma unroll 1
-        for (int r0 = 0; r0 < (a.out ? C : 0); r0 += 16) {
-          float d[16];
-          tmem_ld16(tmD1 + lane_base + 64 + r0, d);
+        if (a.out) {
+          float d[64];
+          tmem_ld16n<4>(tmD1 + lane_base + 64, d);
           tmem_wait_ld();
           if (a.out_bf16) {
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
-              *reinterpret_cast<__nv_bfloat16*>(sm + OFF_V + ((r0 + u) * D + j) * 2) = __float2bfloat16_rn(d[u]);
+            for (int u = 0; u < C; ++u)
+              *reinterpret_cast<__nv_bfloat16*>(sm + OFF_V + (u * D + j) * 2) = __float2bfloat16_rn(d[u]);
           } else {
 #pragma unroll
-            for (int u = 0; u < 16; ++u) reinterpret_cast<float*>(sm + OFF_X)[(r0 + u) * D + j] = d[u];
+            for (int u = 0; u < C; ++u) reinterpret_cast<float*>(sm + OFF_X)[u * D + j] = d[u];
           }
         }
         // bf16 copy of the new state for the next chunk
 #pragma unroll 1
-        for (int i0 = 0; i0 < D; i0 += 16) {
-          float sv[16];
-          tmem_ld16(tmS + lane_base + i0, sv);
+        for (int i0 = 0; i0 < D; i0 += 64) {
+          float sv[64];
+          tmem_ld16n<4>(tmS + lane_base + i0, sv);
           tmem_wait_ld();
-          *reinterpret_cast<uint4*>(sm + OFF_S + sw_off(j, i0, 128)) = make_uint4(
-              pack_bf16(sv[0], sv[1]), pack_bf16(sv[2], sv[3]), pack_bf16(sv[4], sv[5]), pack_bf16(sv[6], sv[7]));
-          *reinterpret_cast<uint4*>(sm + OFF_S + sw_off(j, i0 + 8, 128)) =
-              make_uint4(pack_bf16(sv[8], sv[9]), pack_bf16(sv[10], sv[11]), pack_bf16(sv[12], sv[13]),
-                         pack_bf16(sv[14], sv[15]));
+#pragma unroll
+          for (int u = 0; u < 64; u += 8)
+            *reinterpret_cast<uint4*>(sm + OFF_S + sw_off(j, i0 + u, 128)) =
+                make_uint4(pack_bf16(sv[u], sv[u + 1]), pack_bf16(sv[u + 2], sv[u + 3]),
+                           pack_bf16(sv[u + 4], sv[u + 5]), pack_bf16(sv[u + 6], sv[u + 7]));
         }
       }
       fence_async_smem();
@@ -714,6 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
       }
     }
   }
+  if (pf_pending) mbar_wait_bounded(bar_pf, pf_parity, kWaitLimitNs);  // copies still in flight
   if (aborted && tid == kMmaThread) {
     // let any MMA still in flight finish before the tensor memory is released
     mma_commit(bar3);
@@ -726,12 +821,55 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(FusedArgs a) {
 
 bool fused_available() { return true; }
 
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [tokens][heads][128] row-major, box = 128 channels x 1 head x 64 tokens, no swizzle
+bool encode_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t esize, int64_t tokens,
+                 int heads) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)tokens};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * esize, (cuuint64_t)heads * D * esize};
+  const cuuint32_t box[3] = {(cuuint32_t)D, 1u, (cuuint32_t)C};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream) {
   cudaError_t err = cudaFuncSetAttribute(fused_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   if (err != cudaSuccess) return err;
   if (a.batch == 0) return cudaSuccess;
+  InputMaps tm;
+  memset(&tm, 0, sizeof(tm));
+  // with no tokens at all the maps are never used (every sequence is empty)
+  const int64_t rows = a.total_tokens;
+  const bool ok = rows == 0 || encode_rows(&tm.raw, a.raw_gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, a.Hv) &&
+                  encode_rows(&tm.k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hk) &&
+                  encode_rows(&tm.q, a.q ? a.q : a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hk) &&
+                  encode_rows(&tm.v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv);
+  if (!ok) return cudaErrorInvalidValue;
   dim3 grid(a.Hv, a.batch);
-  fused_chunk_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(a);
+  fused_chunk_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(a, tm);
   return cudaGetLastError();
 }
 

@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_chunk_kernel(SimtArgs a) {
     }
     __syncthreads();
     for (int e = tid; e < C * dk; e += kSimtThreads) {
-      const int r = e / dk, i = e % dk;
+      const int i = e % dk;
       const float Gr = G[e], GC = G[(C - 1) * dk + i];
       const float gam = expf(Gr);
       qg[e] = qq[e] * gam;
