@@ -434,6 +434,22 @@ def cpu_baseline(w, args):
             "seconds": dt}
 
 
+def profile_launches(args):
+    """Plain launches of the prefill kernel on one workload, nothing else (a target for ncu)."""
+    import kimi_delta_attention_23_b200 as kda
+    from kimi_delta_attention_23_b200 import build as kbuild
+    kbuild.build()
+    w = W.make(args.workload, device="cuda")
+    for _ in range(args.profile_launches):
+        pool = w.state_pool.clone()
+        kda.kda_chunk_fwd(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens, pool,
+                          w.state_indices, output_dtype=w.output_dtype, gate_mode=w.gate_mode, beta_mode=w.beta_mode,
+                          state_layout=w.state_layout, gate_lower_bound=w.gate_lower_bound)
+    torch.cuda.synchronize()
+    print("launched", args.profile_launches)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -445,7 +461,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    ap.add_argument("--profile-launches", type=int, default=0,
+                    help="only run this many kda_chunk_fwd launches on the workload (for ncu), no timing")
     args = ap.parse_args()
+    if args.profile_launches:
+        return profile_launches(args)
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":

@@ -146,6 +146,7 @@ WORKLOADS = (
     "varlen8_H32_vfirst",
     "long_T131072_H32_cp16",
     "batch64_T2048_H16_safe",
+    "batch4_T2048_H32",  # one wave of 128 chains, inputs 404 MB (> L2): the profiling case
 )
 
 
@@ -172,6 +173,8 @@ def make(name: str, device="cpu", seed: Optional[int] = None) -> Workload:
         w = random_inputs([2048] * 64, 16, 16, 128, 128, seed=s, raw_std=2.0, beta_mean=2.0,
                           beta_std=1.0, state_std=0.1, gate_mode="safe", gate_lower_bound=-5.0,
                           device=device, name=name)
+    elif name == "batch4_T2048_H32":
+        w = random_inputs([2048] * 4, 32, 32, 128, 128, seed=s, state_std=0.1, device=device, name=name)
     else:  # pragma: no cover
         raise KeyError(name)
     return w

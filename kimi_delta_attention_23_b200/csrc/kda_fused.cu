@@ -54,7 +54,8 @@ constexpr int OFF_S = 0;                    // S^T        128 rows x 128 K
 constexpr int OFF_KQ = OFF_S + 32768;       // [K o Gamma ; Q o Gamma]   128 rows x 128 K
 constexpr int OFF_KPT = OFF_KQ + 32768;     // K'^T       128 rows x 64 K
 constexpr int OFF_X = OFF_KPT + 16384;      // X^T, then Delta^T   128 rows x 64 K
-constexpr int OFF_V = OFF_X + 16384;        // V row-major [64][128] bf16 (plain); O staging spans X..V
+constexpr int OFF_V = OFF_X + 16384;        // V as the MN-major A operand V^T (two 64-column halves, 8 KB
+                                            // apart, 128B-swizzled by the tensor copy)
 constexpr int OFF_T = OFF_V + 16384;        // T          64 rows x 64 K
 constexpr int OFF_P = OFF_T + 8192;         // P          64 rows x 64 K
 constexpr int OFF_KPI = OFF_P + 8192;       // K o pi     64 x 128 (rows scaled from their 16-block start)
@@ -76,8 +77,8 @@ constexpr int OFF_Y = OFF_KPI8;             // fp32 inverse temporaries: [2][16]
 // inputs of the next chunk land here (bulk async copies issued during the state phase, when the
 // score scratch above is dead): raw gate fp32 [64][128], then k, q, v bf16 [64][128]
 constexpr int OFF_PF = OFF_KPI;
-constexpr int PF_RAW = OFF_PF, PF_K = OFF_PF + 32768, PF_Q = OFF_PF + 49152, PF_V = OFF_PF + 65536;
-static_assert(PF_V + 16384 <= OFF_TAU, "prefetch region overlaps live data");
+constexpr int PF_RAW = OFF_PF, PF_K = OFF_PF + 32768, PF_Q = OFF_PF + 49152;
+static_assert(PF_Q + 16384 <= OFF_TAU, "prefetch region overlaps live data");
 constexpr int kLdA = 68;                    // row stride of the fp32 [64][*] arrays
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
@@ -106,14 +107,6 @@ __constant__ unsigned char kDiagPair[64] = {
     8,  16, 17, 24, 25, 26, 32, 33, 34, 35, 40, 41, 42, 43, 44, 48, 49, 50, 51, 52, 53, 56,
     57, 58, 59, 60, 61, 62, 0,  8,  9,  16, 17, 18, 24, 25, 26, 27, 32, 33, 34, 35, 36, 40,
     41, 42, 43, 44, 45, 48, 49, 50, 51, 52, 53, 54, 56, 57, 58, 59, 60, 61, 62, 63};
-
-// the six (row block, column block) pairs of 16-blocks below the diagonal
-__device__ __forceinline__ void pair_of(int p, int& a, int& b) {
-  const int pa[6] = {1, 2, 2, 3, 3, 3};
-  const int pb[6] = {0, 0, 1, 0, 1, 2};
-  a = pa[p];
-  b = pb[p];
-}
 
 }  // namespace
 
@@ -172,17 +165,27 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   // with four tensor copies (rows past the end of the tensor arrive as zeros; rows past the
   // end of the sequence are never read); completion is counted in bytes on bar_pf
   const uint32_t pf_bytes = 32768u + 16384u * (1u + (qb ? 1u : 0u) + (a.values_zero ? 0u : 1u));
-  auto issue_prefetch = [&](int64_t c0n) {
+  // gate, k and q land in the score scratch (free once the chunk's operands are built); V
+  // lands in its operand tile (free once the chunk's second product completed)
+  auto issue_prefetch_gkq = [&](int64_t c0n) {
     mbar_arrive_expect_tx(bar_pf, pf_bytes);
     tma_load_3d(sbase + PF_RAW, &tm.raw, 0, h, (int)c0n, bar_pf);
     tma_load_3d(sbase + PF_K, &tm.k, 0, kh, (int)c0n, bar_pf);
     if (qb) tma_load_3d(sbase + PF_Q, &tm.q, 0, kh, (int)c0n, bar_pf);
-    if (!a.values_zero) tma_load_3d(sbase + PF_V, &tm.v, 0, h, (int)c0n, bar_pf);
+  };
+  auto issue_prefetch_v = [&](int64_t c0n) {
+    if (!a.values_zero) {
+      tma_load_3d(sbase + OFF_V, &tm.v, 0, h, (int)c0n, bar_pf);
+      tma_load_3d(sbase + OFF_V + 8192, &tm.v, 64, h, (int)c0n, bar_pf);
+    }
   };
   bool pf_pending = false;  // a prefetch was issued and its completion not yet observed
   uint32_t pf_parity = 0;   // parity of the next prefetch completion on bar_pf
   if (t1 > t0) {
-    if (tid == kPfThread) issue_prefetch(t0);
+    if (tid == kPfThread) {
+      issue_prefetch_gkq(t0);
+      issue_prefetch_v(t0);
+    }
     pf_pending = true;
   }
   const size_t blk_off = ((size_t)slot * a.Hv + h) * (size_t)(D * D);
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       report(a.status, KDA_ERR_DEVICE_TIMEOUT);
     }
     float al[8][4];
-    uint2 k2[8], q2[8], v2[8];
+    uint2 k2[8], q2[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int row = warp * 8 + r;
@@ -255,7 +258,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         const float4 raw = *reinterpret_cast<const float4*>(sm + PF_RAW + row * 512 + ch * 4);
         k2[r] = *reinterpret_cast<const uint2*>(sm + PF_K + row * 256 + ch * 2);
         q2[r] = qb ? *reinterpret_cast<const uint2*>(sm + PF_Q + row * 256 + ch * 2) : make_uint2(0u, 0u);
-        v2[r] = a.values_zero ? make_uint2(0u, 0u) : *reinterpret_cast<const uint2*>(sm + PF_V + row * 256 + ch * 2);
         const float xs[4] = {raw.x + dtb.x, raw.y + dtb.y, raw.z + dtb.z, raw.w + dtb.w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -268,7 +270,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       } else {
         k2[r] = make_uint2(0u, 0u);
         q2[r] = make_uint2(0u, 0u);
-        v2[r] = make_uint2(0u, 0u);
 #pragma unroll
         for (int c = 0; c < 4; ++c) al[r][c] = 1.f;
       }
@@ -303,9 +304,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       break;
     }
 
-    // V rows (plain row-major) for the first epilogue
-#pragma unroll
-    for (int r = 0; r < 8; ++r) *reinterpret_cast<uint2*>(sm + OFF_V + ((warp * 8 + r) * D + ch) * 2) = v2[r];
 
     // chunk-level and 16-block-level factors
     float pre[4], suf[4], prevb[4], nextb[4];
@@ -332,14 +330,24 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       *reinterpret_cast<float4*>(sGC + ch) =
           make_float4(p8[7][0] * suf[0], p8[7][1] * suf[1], p8[7][2] * suf[2], p8[7][3] * suf[3]);
     }
-    // decay between the two 16-blocks of each pair (excluding both blocks)
-    for (int e = tid; e < 6 * D; e += kThreads) {
-      int pa, pb;
-      pair_of(e / D, pa, pb);
-      const int i = e % D;
-      float m = 1.f;
-      for (int cb = pb + 1; cb < pa; ++cb) m *= sTau[(2 * cb) * D + i] * sTau[(2 * cb + 1) * D + i];
-      sMp[e] = m;
+    // decay between the two 16-blocks of each pair (both blocks excluded); pairs in the order
+    // (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
+    if (warp == 0) {
+      float t16a[4], t16b[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float* tv = sTau + ch + c;
+        t16a[c] = tv[2 * D] * tv[3 * D];  // 16-block 1
+        t16b[c] = tv[4 * D] * tv[5 * D];  // 16-block 2
+      }
+      const float4 one = make_float4(1.f, 1.f, 1.f, 1.f);
+      *reinterpret_cast<float4*>(sMp + 0 * D + ch) = one;
+      *reinterpret_cast<float4*>(sMp + 1 * D + ch) = make_float4(t16a[0], t16a[1], t16a[2], t16a[3]);
+      *reinterpret_cast<float4*>(sMp + 2 * D + ch) = one;
+      *reinterpret_cast<float4*>(sMp + 3 * D + ch) =
+          make_float4(t16a[0] * t16b[0], t16a[1] * t16b[1], t16a[2] * t16b[2], t16a[3] * t16b[3]);
+      *reinterpret_cast<float4*>(sMp + 4 * D + ch) = make_float4(t16b[0], t16b[1], t16b[2], t16b[3]);
+      *reinterpret_cast<float4*>(sMp + 5 * D + ch) = one;
     }
     // operand tiles
     uint32_t kpt[4][4];  // K'^T chunk for each of my 4 channels (8 consecutive tokens)
@@ -461,8 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     {
       const int g = lane >> 2, t = lane & 3, m = lane >> 3;
       if (warp < 6) {
-        int pa, pb;
-        pair_of(warp, pa, pb);
+        // pairs (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
+        const int pa = warp < 1 ? 1 : (warp < 3 ? 2 : 3), pb = warp - pa * (pa - 1) / 2;
         float accA[2][4] = {}, accP[2][4] = {};
         const float* mp = sMp + warp * D;
 #pragma unroll
@@ -473,12 +481,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           ldsm_x4(sbase + OFF_QPI + sw_off(ar, akc * 8, 64), aq0, aq1, aq2, aq3);
           const int br = 16 * pb + (m >> 1) * 8 + (lane & 7), bkc = 2 * kk + (m & 1);
           ldsm_x4(sbase + OFF_KC + sw_off(br, bkc * 8, 64), b00, b01, b10, b11);
-          const int k0 = 16 * kk + 2 * t;
-          const float m0 = mp[k0], m1 = mp[k0 + 1], m2 = mp[k0 + 8], m3 = mp[k0 + 9];
-          b00 = scale_bf16x2(b00, m0, m1);
-          b10 = scale_bf16x2(b10, m0, m1);
-          b01 = scale_bf16x2(b01, m2, m3);
-          b11 = scale_bf16x2(b11, m2, m3);
+          if (pa - pb > 1) {  // adjacent 16-blocks have nothing between them
+            const int k0 = 16 * kk + 2 * t;
+            const float m0 = mp[k0], m1 = mp[k0 + 1], m2 = mp[k0 + 8], m3 = mp[k0 + 9];
+            b00 = scale_bf16x2(b00, m0, m1);
+            b10 = scale_bf16x2(b10, m0, m1);
+            b01 = scale_bf16x2(b01, m2, m3);
+            b11 = scale_bf16x2(b11, m2, m3);
+          }
           mma16816(accA[0], ak0, ak1, ak2, ak3, b00, b01);
           mma16816(accA[1], ak0, ak1, ak2, ak3, b10, b11);
           mma16816(accP[0], aq0, aq1, aq2, aq3, b00, b01);
@@ -522,84 +532,107 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     __syncthreads();  // (3) A and P complete
 
     // =============================== k-side, part 3: T = (I + diag(beta) A)^{-1} diag(beta)
-    // X = (I + L)^{-1}, L = diag(beta) A strictly lower: diagonal 16-blocks by forward
-    // substitution, then two doubling levels -- X10, X32 from 16-blocks, then the lower-left
-    // 32-block -- each as X_ab = -X_aa (L_ab X_bb) over the blocks just finished.
+    // X = (I + L)^{-1}, L = diag(beta) A strictly lower.  Diagonal 16-blocks by forward
+    // substitution (four threads per column); then two doubling levels on tf32 mma.sync --
+    // X10 and X32 from the 16-blocks, then the lower-left 32-block from the 32-blocks -- each as
+    // X_ab = -X_aa (L_ab X_bb).  T is rounded to bf16 afterwards, so tf32 products suffice.
     {
       float* Xi = reinterpret_cast<float*>(sm + OFF_XI);
-      float* Y1 = reinterpret_cast<float*>(sm + OFF_Y);  // [2][16][16]
-      float* Y2 = Y1 + 512;                               // [32][32]
-      if (tid < 64) {
-        const int blk = tid >> 4, col = tid & 15, base = 16 * blk;
-        float x[16];
+      float* Yb = reinterpret_cast<float*>(sm + OFF_Y);  // per-warp 16x8 tiles, then [32][32]
+      {
+        const int col = (tid >> 2) & 15, q = tid & 3, base = 16 * (tid >> 6);
+        float lrow[16][4];  // L[base + r][base + 4j + q]
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-          float acc = 0.f;
+          const float br = sBeta[base + r];
 #pragma unroll
-          for (int u = 0; u < 15; ++u)
-            if (u < r) acc += sA[(base + r) * kLdA + base + u] * x[u];
-          x[r] = (r == col) ? 1.f : (r < col ? 0.f : -sBeta[base + r] * acc);
+          for (int jj = 0; jj < 4; ++jj) lrow[r][jj] = br * sA[(base + r) * kLdA + base + 4 * jj + q];
+        }
+        float xq[4] = {0.f, 0.f, 0.f, 0.f};  // x[4 jj + q]: the entries this thread sums over
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          float part = 0.f;
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
+            if (4 * jj + q < r) part += lrow[r][jj] * xq[jj];
+          part += __shfl_xor_sync(0xffffffffu, part, 1);
+          part += __shfl_xor_sync(0xffffffffu, part, 2);
+          const float xr = (r == col) ? 1.f : (r < col ? 0.f : -part);
+          if ((r & 3) == q) xq[r >> 2] = xr;
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Xi[(base + r) * kLdA + base + col] = x[r];
-        if ((blk & 1) == 0) {
+        for (int jj = 0; jj < 4; ++jj) Xi[(base + 4 * jj + q) * kLdA + base + col] = xq[jj];
+      }
+      __syncthreads();
+      const int g = lane >> 2, t = lane & 3;
+      auto lval = [&](int r, int c) { return sBeta[r] * sA[r * kLdA + c]; };
+      if (warp < 4) {
+        // level 1: warp -> (problem, 8-column tile); problem 0 = X10, problem 1 = X32
+        const int ra = (warp >> 1) ? 3 : 1, cb = 16 * (ra - 1), R0 = 16 * ra, n0 = 8 * (warp & 1);
+        float* yt = Yb + warp * 128;  // 16 x 8 tile of Y, row-major
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int r = 0; r < 16; ++r) Xi[(base + r) * kLdA + base + 16 + col] = 0.f;
+        for (int ks = 0; ks < 2; ++ks) {
+          const int k0 = 8 * ks;
+          mma1688_tf32(acc, to_tf32(lval(R0 + g, cb + k0 + t)), to_tf32(lval(R0 + g + 8, cb + k0 + t)),
+                       to_tf32(lval(R0 + g, cb + k0 + t + 4)), to_tf32(lval(R0 + g + 8, cb + k0 + t + 4)),
+                       to_tf32(Xi[(cb + k0 + t) * kLdA + cb + n0 + g]),
+                       to_tf32(Xi[(cb + k0 + t + 4) * kLdA + cb + n0 + g]));
         }
+        yt[g * 8 + 2 * t] = acc[0];
+        yt[g * 8 + 2 * t + 1] = acc[1];
+        yt[(g + 8) * 8 + 2 * t] = acc[2];
+        yt[(g + 8) * 8 + 2 * t + 1] = acc[3];
+        __syncwarp();
+        float xo[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          const int k0 = 8 * ks;
+          mma1688_tf32(xo, to_tf32(Xi[(R0 + g) * kLdA + R0 + k0 + t]), to_tf32(Xi[(R0 + g + 8) * kLdA + R0 + k0 + t]),
+                       to_tf32(Xi[(R0 + g) * kLdA + R0 + k0 + t + 4]),
+                       to_tf32(Xi[(R0 + g + 8) * kLdA + R0 + k0 + t + 4]), to_tf32(yt[(k0 + t) * 8 + g]),
+                       to_tf32(yt[(k0 + t + 4) * 8 + g]));
+        }
+        Xi[(R0 + g) * kLdA + cb + n0 + 2 * t] = -xo[0];
+        Xi[(R0 + g) * kLdA + cb + n0 + 2 * t + 1] = -xo[1];
+        Xi[(R0 + g + 8) * kLdA + cb + n0 + 2 * t] = -xo[2];
+        Xi[(R0 + g + 8) * kLdA + cb + n0 + 2 * t + 1] = -xo[3];
       }
       __syncthreads();
       {
-        // level 1: p = 0 -> X10, p = 1 -> X32; two columns per thread
-        const int p = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
-        const int ra = p ? 3 : 1, cb = 16 * (ra - 1), R = 16 * ra + r;
-        float y0 = 0.f, y1 = 0.f;
+        // level 2: Y = L[32:64, 0:32] X[0:32, 0:32]; X[32:64, 0:32] = -X[32:64, 32:64] Y
+        // warp -> (16-row tile mt, 8-column tile nt); X[0:16, 16:32] and X[32:48, 48:64] are zero
+        float* Y2 = Yb + 512;
+        const int mt = warp >> 2, nt = warp & 3, R0 = 32 + 16 * mt, n0 = 8 * nt;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const float l = sA[R * kLdA + cb + u];
-          y0 += l * Xi[(cb + u) * kLdA + cb + c];
-          y1 += l * Xi[(cb + u) * kLdA + cb + c + 1];
+        for (int ks = 0; ks < 4; ++ks) {
+          const int k0 = 8 * ks;
+          if (nt >= 2 && ks < 2) continue;
+          mma1688_tf32(acc, to_tf32(lval(R0 + g, k0 + t)), to_tf32(lval(R0 + g + 8, k0 + t)),
+                       to_tf32(lval(R0 + g, k0 + t + 4)), to_tf32(lval(R0 + g + 8, k0 + t + 4)),
+                       to_tf32(Xi[(k0 + t) * kLdA + n0 + g]), to_tf32(Xi[(k0 + t + 4) * kLdA + n0 + g]));
         }
-        Y1[p * 256 + r * 16 + c] = sBeta[R] * y0;
-        Y1[p * 256 + r * 16 + c + 1] = sBeta[R] * y1;
+        const int yr = 16 * mt;
+        Y2[(yr + g) * 32 + n0 + 2 * t] = acc[0];
+        Y2[(yr + g) * 32 + n0 + 2 * t + 1] = acc[1];
+        Y2[(yr + g + 8) * 32 + n0 + 2 * t] = acc[2];
+        Y2[(yr + g + 8) * 32 + n0 + 2 * t + 1] = acc[3];
         __syncthreads();
-        float x0 = 0.f, x1 = 0.f;
+        float xo[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const float xr = Xi[R * kLdA + 16 * ra + u];
-          x0 += xr * Y1[p * 256 + u * 16 + c];
-          x1 += xr * Y1[p * 256 + u * 16 + c + 1];
+        for (int ks = 0; ks < 4; ++ks) {
+          const int k0 = 8 * ks;
+          if (mt == 0 && ks >= 2) continue;
+          mma1688_tf32(xo, to_tf32(Xi[(R0 + g) * kLdA + 32 + k0 + t]), to_tf32(Xi[(R0 + g + 8) * kLdA + 32 + k0 + t]),
+                       to_tf32(Xi[(R0 + g) * kLdA + 32 + k0 + t + 4]),
+                       to_tf32(Xi[(R0 + g + 8) * kLdA + 32 + k0 + t + 4]), to_tf32(Y2[(k0 + t) * 32 + n0 + g]),
+                       to_tf32(Y2[(k0 + t + 4) * 32 + n0 + g]));
         }
-        Xi[R * kLdA + cb + c] = -x0;
-        Xi[R * kLdA + cb + c + 1] = -x1;
-      }
-      __syncthreads();
-      {
-        // level 2: rows 32..63, columns 0..31; four columns per thread
-        const int r = tid >> 3, c = (tid & 7) * 4;
-        float y[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-        for (int u = 0; u < 32; ++u) {
-          const float l = sA[(32 + r) * kLdA + u];
-          const float4 xv = *reinterpret_cast<const float4*>(Xi + u * kLdA + c);
-          y[0] += l * xv.x;
-          y[1] += l * xv.y;
-          y[2] += l * xv.z;
-          y[3] += l * xv.w;
-        }
-        const float bR = sBeta[32 + r];
-        *reinterpret_cast<float4*>(Y2 + r * 32 + c) = make_float4(bR * y[0], bR * y[1], bR * y[2], bR * y[3]);
-        __syncthreads();
-        float x[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-        for (int u = 0; u < 32; ++u) {
-          const float xr = Xi[(32 + r) * kLdA + 32 + u];
-          const float4 yv = *reinterpret_cast<const float4*>(Y2 + u * 32 + c);
-          x[0] += xr * yv.x;
-          x[1] += xr * yv.y;
-          x[2] += xr * yv.z;
-          x[3] += xr * yv.w;
-        }
-        *reinterpret_cast<float4*>(Xi + (32 + r) * kLdA + c) = make_float4(-x[0], -x[1], -x[2], -x[3]);
+        Xi[(R0 + g) * kLdA + n0 + 2 * t] = -xo[0];
+        Xi[(R0 + g) * kLdA + n0 + 2 * t + 1] = -xo[1];
+        Xi[(R0 + g + 8) * kLdA + n0 + 2 * t] = -xo[2];
+        Xi[(R0 + g + 8) * kLdA + n0 + 2 * t + 1] = -xo[3];
       }
       __syncthreads();
       // T[r][s] = X[r][s] beta_s for s <= r, else 0; bf16 tile [r][s]
@@ -619,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     fence_async_smem();
     __syncthreads();  // (4) every operand of this chunk is in shared memory
     if (c0 + C < t1) {
-      if (tid == kPfThread) issue_prefetch(c0 + C);
+      if (tid == kPfThread) issue_prefetch_gkq(c0 + C);
       pf_pending = true;
     }
 
@@ -642,20 +675,15 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         report(a.status, KDA_ERR_DEVICE_TIMEOUT);
       } else {
         tc_fence_after();
-        // X^T[j][r] = V[r][j] - D1[j][r]
+        // Y^T[j][r] = -D1[j][r] = -((K o Gamma) S0)^T; V enters in the next product
         float d[64];
         tmem_ld16n<4>(tmD1 + lane_base, d);
         tmem_wait_ld();
 #pragma unroll
-        for (int r0 = 0; r0 < C; r0 += 8) {
-          float x[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            x[u] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sm + OFF_V + ((r0 + u) * D + j) * 2)) -
-                   d[r0 + u];
+        for (int r0 = 0; r0 < C; r0 += 8)
           *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(j, r0, 128)) =
-              make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
-        }
+              make_uint4(pack_bf16(-d[r0], -d[r0 + 1]), pack_bf16(-d[r0 + 2], -d[r0 + 3]),
+                         pack_bf16(-d[r0 + 4], -d[r0 + 5]), pack_bf16(-d[r0 + 6], -d[r0 + 7]));
       }
       fence_async_smem();
       tc_fence_before();
@@ -666,13 +694,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       break;
     }
 
-    // D1[:, 0:64] = X^T T^T = Delta^T   (N = 64, K = 64)
+    // D1[:, 0:64] = V^T T^T + Y^T T^T = (V - (K o Gamma) S0)^T T^T = Delta^T   (N = 64, K = 64)
     if (tid == kMmaThread) {
       tc_fence_after();
+      if (!a.values_zero) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmD1, desc_sw128_mn(sbase + OFF_V + kk * 2048, 8192), desc_sw128(sbase + OFF_T + kk * 32),
+                   idesc_bf16_f32(64, true), kk > 0);
+      }
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmD1, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128(sbase + OFF_T + kk * 32), idesc_bf16_f32(64),
-                 kk > 0);
+                 (kk > 0) || !a.values_zero);
       mma_commit(bar1);
     }
     if (warp < 4) {
@@ -699,7 +733,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           tmem_ld16n<4>(tmS + lane_base + i0, sv);
           tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 64; ++u) sv[u] *= sGC[i0 + u];
+          for (int u = 0; u < 64; u += 4) {
+            const float4 gv = *reinterpret_cast<const float4*>(sGC + i0 + u);
+            sv[u] *= gv.x;
+            sv[u + 1] *= gv.y;
+            sv[u + 2] *= gv.z;
+            sv[u + 3] *= gv.w;
+          }
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             tmem_st16(tmS + lane_base + i0 + 16 * q, *reinterpret_cast<const float(*)[16]>(sv + 16 * q));
@@ -714,6 +754,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       aborted = true;
       break;
     }
+    // the V tile is free now that the second product completed
+    if (c0 + C < t1 && tid == kPfThread) issue_prefetch_v(c0 + C);
 
     // D1[:, 64:128] += Delta^T P^T ;  S^T += Delta^T K'   (accumulate)
     if (tid == kMmaThread) {
@@ -735,7 +777,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         report(a.status, KDA_ERR_DEVICE_TIMEOUT);
       } else {
         tc_fence_after();
-        // outputs O[r][j] staged row-major (bf16 in the V region, fp32 across X..V)
+        // outputs O[r][j] staged row-major (bf16 in the X tile, fp32 in the K/Q tile: both are
+        // free once the last products completed; the V tile already receives the next chunk)
         if (a.out) {
           float d[64];
           tmem_ld16n<4>(tmD1 + lane_base + 64, d);
@@ -743,10 +786,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           if (a.out_bf16) {
 #pragma unroll
             for (int u = 0; u < C; ++u)
-              *reinterpret_cast<__nv_bfloat16*>(sm + OFF_V + (u * D + j) * 2) = __float2bfloat16_rn(d[u]);
+              *reinterpret_cast<__nv_bfloat16*>(sm + OFF_X + (u * D + j) * 2) = __float2bfloat16_rn(d[u]);
           } else {
 #pragma unroll
-            for (int u = 0; u < C; ++u) reinterpret_cast<float*>(sm + OFF_X)[u * D + j] = d[u];
+            for (int u = 0; u < C; ++u) reinterpret_cast<float*>(sm + OFF_KQ)[u * D + j] = d[u];
           }
         }
         // bf16 copy of the new state for the next chunk
@@ -777,14 +820,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         const int row = e >> 4, cc = e & 15;
         if (row < L)
           *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)(c0 + row) * a.Hv + h) * D +
-                                    cc * 8) = *reinterpret_cast<const uint4*>(sm + OFF_V + row * 256 + cc * 16);
+                                    cc * 8) = *reinterpret_cast<const uint4*>(sm + OFF_X + row * 256 + cc * 16);
       }
     } else {
       for (int e = tid; e < C * 32; e += kThreads) {
         const int row = e >> 5, cc = e & 31;
         if (row < L)
           *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + ((size_t)(c0 + row) * a.Hv + h) * D + cc * 4) =
-              *reinterpret_cast<const float4*>(sm + OFF_X + row * 512 + cc * 16);
+              *reinterpret_cast<const float4*>(sm + OFF_KQ + row * 512 + cc * 16);
       }
     }
   }
@@ -839,18 +882,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [tokens][heads][128] row-major, box = 128 channels x 1 head x 64 tokens, no swizzle
+// [tokens][heads][128] row-major; box = box_x channels x 1 head x 64 tokens
 bool encode_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t esize, int64_t tokens,
-                 int heads) {
+                 int heads, uint32_t box_x = D, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)tokens};
   const cuuint64_t strides[2] = {(cuuint64_t)D * esize, (cuuint64_t)heads * D * esize};
-  const cuuint32_t box[3] = {(cuuint32_t)D, 1u, (cuuint32_t)C};
+  const cuuint32_t box[3] = {box_x, 1u, (cuuint32_t)C};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
-  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -866,7 +908,8 @@ cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream) {
   const bool ok = rows == 0 || encode_rows(&tm.raw, a.raw_gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, a.Hv) &&
                   encode_rows(&tm.k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hk) &&
                   encode_rows(&tm.q, a.q ? a.q : a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hk) &&
-                  encode_rows(&tm.v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv);
+                  encode_rows(&tm.v, a.v ? a.v : a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv, 64,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
   dim3 grid(a.Hv, a.batch);
   fused_chunk_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(a, tm);

@@ -189,34 +189,65 @@ cudaError_t launch_simt_chunk(const SimtArgs& a, cudaStream_t stream) {
 //   in_0 = S_initial;  out_i = M_i in_i + U_i;  in_{i+1} = out_i;  final = out_{N-1}.
 // One block per (head, 32-column tile of the state); the segment loop is serial.
 // ------------------------------------------------------------------------------------------
-constexpr int kScanCols = 32;
+constexpr int kScanCols = 16;
 constexpr int kScanThreads = 256;
 
+// One block per (head, 16-column tile of the state).  Each step stages M_i (dk x dk) in shared
+// memory with coalesced float4 loads; thread t then owns row t / 2 and eight of the sixteen
+// columns, so every M element read from shared memory feeds eight independent accumulators.
 __global__ void __launch_bounds__(kScanThreads) affine_scan_kernel(ScanArgs a) {
   extern __shared__ float sm[];
   const int h = blockIdx.x, j0 = blockIdx.y * kScanCols, tid = threadIdx.x;
   const int dk = a.dk, dv = a.dv, H = a.H;
   const int nc = min(kScanCols, dv - j0);
-  float* cur = sm;                   // [dk][kScanCols]
-  float* nxt = sm + dk * kScanCols;  // [dk][kScanCols]
+  float* Ms = sm;                           // [dk][dk + 1]
+  float* cur = Ms + dk * (dk + 1);          // [dk][kScanCols]
+  float* nxt = cur + dk * kScanCols;        // [dk][kScanCols]
   const size_t st = (size_t)dk * dv;
   for (int e = tid; e < dk * kScanCols; e += kScanThreads) {
     const int i = e / kScanCols, jj = e % kScanCols;
     cur[e] = jj < nc ? a.initial[(size_t)h * st + state_off(i, j0 + jj, dk, dv, a.v_first)] : 0.f;
   }
-  __syncthreads();
+  const int row = tid >> 1, c0 = (tid & 1) * 8;
   for (int s = 0; s < a.N; ++s) {
     const size_t base = ((size_t)s * H + h) * st;
-    const float* Ms = a.M + ((size_t)s * H + h) * (size_t)dk * dk;
-    for (int e = tid; e < dk * kScanCols; e += kScanThreads) {
-      const int i = e / kScanCols, jj = e % kScanCols;
-      if (jj >= nc) continue;
-      const size_t o = base + state_off(i, j0 + jj, dk, dv, a.v_first);
-      if (a.incoming) a.incoming[o] = cur[e];
-      float acc = a.U[o];
-      for (int l = 0; l < dk; ++l) acc = fmaf(Ms[(size_t)i * dk + l], cur[l * kScanCols + jj], acc);
-      nxt[e] = acc;
-      if (a.outgoing) a.outgoing[o] = acc;
+    const float* Mg = a.M + ((size_t)s * H + h) * (size_t)dk * dk;
+    __syncthreads();  // previous step's reads of Ms are done
+    if ((dk & 3) == 0) {
+      for (int e = tid; e < dk * dk / 4; e += kScanThreads) {
+        const float4 m4 = reinterpret_cast<const float4*>(Mg)[e];
+        const int i = (4 * e) / dk, l = (4 * e) % dk;
+        float* d = Ms + i * (dk + 1) + l;
+        d[0] = m4.x;
+        d[1] = m4.y;
+        d[2] = m4.z;
+        d[3] = m4.w;
+      }
+    } else {
+      for (int e = tid; e < dk * dk; e += kScanThreads) Ms[(e / dk) * (dk + 1) + e % dk] = Mg[e];
+    }
+    __syncthreads();
+    for (int r = row; r < dk; r += kScanThreads / 2) {
+      float acc[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+      const float* mrow = Ms + r * (dk + 1);
+      for (int l = 0; l < dk; ++l) {
+        const float m = mrow[l];
+        const float* cr = cur + l * kScanCols + c0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[u] = fmaf(m, cr[u], acc[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int jj = c0 + u;
+        if (jj >= nc) continue;
+        const size_t o = base + state_off(r, j0 + jj, dk, dv, a.v_first);
+        if (a.incoming) a.incoming[o] = cur[r * kScanCols + jj];
+        const float v = acc[u] + a.U[o];
+        nxt[r * kScanCols + jj] = v;
+        if (a.outgoing) a.outgoing[o] = v;
+      }
     }
     __syncthreads();
     float* t = cur;
@@ -224,6 +255,7 @@ __global__ void __launch_bounds__(kScanThreads) affine_scan_kernel(ScanArgs a) {
     nxt = t;
   }
   if (a.final_state) {
+    __syncthreads();
     for (int e = tid; e < dk * kScanCols; e += kScanThreads) {
       const int i = e / kScanCols, jj = e % kScanCols;
       if (jj < nc) a.final_state[(size_t)h * st + state_off(i, j0 + jj, dk, dv, a.v_first)] = cur[e];
@@ -232,7 +264,7 @@ __global__ void __launch_bounds__(kScanThreads) affine_scan_kernel(ScanArgs a) {
 }
 
 cudaError_t launch_affine_scan(const ScanArgs& a, cudaStream_t stream) {
-  const size_t smem = 2 * (size_t)a.dk * kScanCols * sizeof(float);
+  const size_t smem = ((size_t)a.dk * (a.dk + 1) + 2 * (size_t)a.dk * kScanCols) * sizeof(float);
   cudaError_t err = cudaFuncSetAttribute(affine_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return err;
