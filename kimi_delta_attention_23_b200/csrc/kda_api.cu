@@ -161,17 +161,12 @@ extern "C" kda_status_t kda_segment_summarize_and_scan(
       f.lb = gate_lower_bound;
       f.status = device_status;
       f.state_in = nullptr;
-      // transition M_i: from I with zero values, stored row-major
+      // one launch carries both: transition M_i (from I, zero values, row-major) and the local
+      // contribution U_i (from 0, the real values, in the state layout)
+      f.build = 1;
       f.state_out = M;
-      f.v_first = 0;
-      f.init_mode = 2;
-      f.values_zero = 1;
-      if (kda::launch_fused_chunk(f, s) != cudaSuccess) return KDA_ERR_CUDA;
-      // contribution U_i: from 0 with the real values, stored in the state layout
-      f.state_out = U;
+      f.state_out2 = U;
       f.v_first = v_first;
-      f.init_mode = 1;
-      f.values_zero = 0;
       if (kda::launch_fused_chunk(f, s) != cudaSuccess) return KDA_ERR_CUDA;
     }
     if (!use_fused) {

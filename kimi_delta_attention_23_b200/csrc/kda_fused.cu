@@ -26,8 +26,8 @@
 //   * state side: the four products that touch S run on tcgen05 with the state transposed
 //     (dv = 128 rows = the 128 TMEM lanes): D1 = S^T [K o Gamma; Q o Gamma]^T, D2 = X^T T^T,
 //     D1o += Delta^T P^T, S^T += Delta^T K'.  S^T stays in TMEM in fp32 across chunks; a bf16
-//     copy in shared memory is the A operand of the next chunk's first product.  Warps 0-3
-//     (one per TMEM lane quadrant) run the epilogues; thread 128 issues the MMAs.
+//     copy, also in TMEM, is the A operand of the next chunk's first product.  All eight warps
+//     run the epilogues (two per TMEM lane quadrant); thread 128 issues the MMAs.
 #include <cuda.h>
 #include <string.h>
 
@@ -45,12 +45,12 @@ constexpr int D = 128;         // dk = dv
 constexpr int kThreads = 256;
 constexpr int kMmaThread = 128;
 constexpr int kPfThread = 160;
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;  // D1 [0,128), S fp32 [128,256), S bf16 A operand [256,320)
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far beyond any legitimate wait
 
 // shared-memory map (bytes from a 1024-aligned base); bf16 operand tiles use the K-major
 // 128-byte swizzle layout (see sw_off)
-constexpr int OFF_S = 0;                    // S^T        128 rows x 128 K
+constexpr int OFF_S = 0;                    // free in prefill (the bf16 state lives in TMEM)
 constexpr int OFF_KQ = OFF_S + 32768;       // [K o Gamma ; Q o Gamma]   128 rows x 128 K
 constexpr int OFF_KPT = OFF_KQ + 32768;     // K'^T       128 rows x 64 K
 constexpr int OFF_X = OFF_KPT + 16384;      // X^T, then Delta^T   128 rows x 64 K
@@ -72,6 +72,7 @@ constexpr int OFF_GC = OFF_BETA + 256;      // fp32 [128] Gamma of the last row
 constexpr int OFF_BAR = OFF_GC + 512;       // 4 mbarriers, TMEM base, abort flag
 constexpr int kSmemBytes = OFF_BAR + 64;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for aligning the base to 1024
+constexpr int OFF_XM = OFF_S;               // build: X^T / Delta^T of the transition state
 constexpr int OFF_XI = OFF_KPI;             // fp32 [64][68] inverse (after the scores are done)
 constexpr int OFF_Y = OFF_KPI8;             // fp32 inverse temporaries: [2][16][16] then [32][32]
 // inputs of the next chunk land here (bulk async copies issued during the state phase, when the
@@ -116,6 +117,10 @@ struct InputMaps {
   CUtensorMap raw, k, q, v;
 };
 
+// kBuild = false: prefill (state from the pool, readout, state back to the pool).
+// kBuild = true: segment build -- two states share every k-side product: the transition M
+// (started at I, zero values) and the contribution U (started at 0, real values); no readout.
+template <bool kBuild>
 __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArgs a, const __grid_constant__ InputMaps tm) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -158,13 +163,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  const uint32_t tmD1 = tmem, tmS = tmem + 128;
+  // TMEM columns.  prefill: D1 [0,128) (X/Delta part, then O part), S fp32 [128,256), S bf16
+  // [256,320).  build: D1 of M [0,64) and of U [64,128), S_M [128,256), S_U [256,384), bf16
+  // copies [384,448) and [448,512).
+  const uint32_t tmD1 = tmem, tmS = tmem + 128, tmSb = kBuild ? tmem + 384 : tmem + 256;
+  const uint32_t tmD1u = tmem + 64, tmSu = tmem + 256, tmSbu = tmem + 448;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  const bool qb = a.q != nullptr;
+  const int ej = (warp & 3) * 32 + lane, ehalf = warp >> 2;  // epilogue row and column half
+  const bool qb = !kBuild && a.q != nullptr;
   // one thread copies the inputs of the chunk starting at token c0n into the prefetch region
   // with four tensor copies (rows past the end of the tensor arrive as zeros; rows past the
   // end of the sequence are never read); completion is counted in bytes on bar_pf
-  const uint32_t pf_bytes = 32768u + 16384u * (1u + (qb ? 1u : 0u) + (a.values_zero ? 0u : 1u));
+  const bool has_v = kBuild || !a.values_zero;
+  const uint32_t pf_bytes = 32768u + 16384u * (1u + (qb ? 1u : 0u) + (has_v ? 1u : 0u));
   // gate, k and q land in the score scratch (free once the chunk's operands are built); V
   // lands in its operand tile (free once the chunk's second product completed)
   auto issue_prefetch_gkq = [&](int64_t c0n) {
@@ -174,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     if (qb) tma_load_3d(sbase + PF_Q, &tm.q, 0, kh, (int)c0n, bar_pf);
   };
   auto issue_prefetch_v = [&](int64_t c0n) {
-    if (!a.values_zero) {
+    if (has_v) {
       tma_load_3d(sbase + OFF_V, &tm.v, 0, h, (int)c0n, bar_pf);
       tma_load_3d(sbase + OFF_V + 8192, &tm.v, 64, h, (int)c0n, bar_pf);
     }
@@ -192,15 +203,16 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   const float* in_blk = a.state_in ? a.state_in + blk_off : nullptr;
   float* out_blk = a.state_out + blk_off;
 
-  // ---- load the incoming state: S^T into TMEM (fp32) and a bf16 copy into shared memory
-  if (warp < 4) {
-    const int j = tid;
+  // ---- load the incoming state: S^T into TMEM (fp32) and a bf16 copy into shared memory;
+  // thread -> state row ej (its TMEM lane), columns split between the two warps of a quadrant
+  {
+    const int j = ej;
 #pragma unroll 1
-    for (int i0 = 0; i0 < D; i0 += 16) {
+    for (int i0 = 64 * ehalf; i0 < 64 * ehalf + 64; i0 += 16) {
       float v[16];
-      if (a.init_mode != 0) {
+      if (kBuild || a.init_mode != 0) {
 #pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] = (a.init_mode == 2 && i0 + u == j) ? 1.f : 0.f;
+        for (int u = 0; u < 16; ++u) v[u] = ((kBuild || a.init_mode == 2) && i0 + u == j) ? 1.f : 0.f;
       } else if (a.v_first) {
         const float4* p = reinterpret_cast<const float4*>(in_blk + (size_t)j * D + i0);
 #pragma unroll
@@ -216,11 +228,18 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         for (int u = 0; u < 16; ++u) v[u] = in_blk[(size_t)(i0 + u) * D + j];
       }
       tmem_st16(tmS + lane_base + i0, v);
-      uint4 c0 = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-      uint4 c1 = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]), pack_bf16(v[12], v[13]),
-                            pack_bf16(v[14], v[15]));
-      *reinterpret_cast<uint4*>(sm + OFF_S + sw_off(j, i0, 128)) = c0;
-      *reinterpret_cast<uint4*>(sm + OFF_S + sw_off(j, i0 + 8, 128)) = c1;
+      uint32_t pk[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) pk[q] = pack_bf16(v[2 * q], v[2 * q + 1]);
+      tmem_st8u(tmSb + lane_base + i0 / 2, pk);
+      if constexpr (kBuild) {  // the contribution starts at zero
+        float z[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) z[u] = 0.f;
+        const uint32_t zp[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        tmem_st16(tmSu + lane_base + i0, z);
+        tmem_st8u(tmSbu + lane_base + i0 / 2, zp);
+      }
     }
     tmem_wait_st();
   }
@@ -235,6 +254,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   const float alpha_floor = safe ? expf(a.lb) : 0.f;
   const int b16 = warp >> 1, upper = warp & 1;
 
+  // beta of the next chunk is read one chunk ahead (lanes 0..7 of each warp, one row each)
+  float beta_raw = 0.f;
+  auto load_beta = [&](int64_t c0n) {
+    const int64_t t = c0n + warp * 8 + lane;
+    if (lane < 8 && t < t1) beta_raw = __ldg(a.beta + (size_t)t * a.Hv + h);
+  };
+  load_beta(t0);
   uint32_t phase = 0;
   bool aborted = false;
 #pragma unroll 1
@@ -276,10 +302,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     }
     if (lane < 8) {
       const int row = warp * 8 + lane;
-      sBeta[row] = row < L ? beta_f32(a.beta[(size_t)(c0 + row) * a.Hv + h], prob) : 0.f;
+      sBeta[row] = row < L ? beta_f32(beta_raw, prob) : 0.f;
     }
     // P's upper triangle must read as zero (A's upper triangle is never read)
-    for (int e = tid; e < 8192 / 16; e += kThreads) reinterpret_cast<uint4*>(sm + OFF_P)[e] = make_uint4(0, 0, 0, 0);
+    if constexpr (!kBuild)
+      for (int e = tid; e < 8192 / 16; e += kThreads) reinterpret_cast<uint4*>(sm + OFF_P)[e] = make_uint4(0, 0, 0, 0);
     // in-block products: p8 inclusive prefix from the block start, s8 exclusive suffix
     float p8[8][4], s8[8][4];
 #pragma unroll
@@ -350,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       *reinterpret_cast<float4*>(sMp + 5 * D + ch) = one;
     }
     // operand tiles
-    uint32_t kpt[4][4];  // K'^T chunk for each of my 4 channels (8 consecutive tokens)
+    float kpv[8][4];  // K' values of my 8 rows x 4 channels (packed pairwise below)
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int row = warp * 8 + r;
@@ -368,34 +395,36 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       }
       *reinterpret_cast<uint2*>(sm + OFF_KQ + sw_off(row, ch, 128)) =
           pack4(kf[0] * g[0], kf[1] * g[1], kf[2] * g[2], kf[3] * g[3]);
-      *reinterpret_cast<uint2*>(sm + OFF_KQ + sw_off(64 + row, ch, 128)) =
-          pack4(qf[0] * g[0], qf[1] * g[1], qf[2] * g[2], qf[3] * g[3]);
+      if constexpr (!kBuild)
+        *reinterpret_cast<uint2*>(sm + OFF_KQ + sw_off(64 + row, ch, 128)) =
+            pack4(qf[0] * g[0], qf[1] * g[1], qf[2] * g[2], qf[3] * g[3]);
       *reinterpret_cast<uint2*>(sm + OFF_KPI + sw_off(row, ch, 64)) =
           pack4(kf[0] * pi[0], kf[1] * pi[1], kf[2] * pi[2], kf[3] * pi[3]);
-      *reinterpret_cast<uint2*>(sm + OFF_QPI + sw_off(row, ch, 64)) =
-          pack4(qf[0] * pi[0], qf[1] * pi[1], qf[2] * pi[2], qf[3] * pi[3]);
+      if constexpr (!kBuild)
+        *reinterpret_cast<uint2*>(sm + OFF_QPI + sw_off(row, ch, 64)) =
+            pack4(qf[0] * pi[0], qf[1] * pi[1], qf[2] * pi[2], qf[3] * pi[3]);
       *reinterpret_cast<uint2*>(sm + OFF_KC + sw_off(row, ch, 64)) =
           pack4(kf[0] * ka[0], kf[1] * ka[1], kf[2] * ka[2], kf[3] * ka[3]);
       const int r32 = b16 * 8 + r;
       if (upper) {
         *reinterpret_cast<uint2*>(sm + OFF_KPI8 + sw_off(r32, ch, 32)) =
             pack4(kf[0] * p8[r][0], kf[1] * p8[r][1], kf[2] * p8[r][2], kf[3] * p8[r][3]);
-        *reinterpret_cast<uint2*>(sm + OFF_QPI8 + sw_off(r32, ch, 32)) =
-            pack4(qf[0] * p8[r][0], qf[1] * p8[r][1], qf[2] * p8[r][2], qf[3] * p8[r][3]);
+        if constexpr (!kBuild)
+          *reinterpret_cast<uint2*>(sm + OFF_QPI8 + sw_off(r32, ch, 32)) =
+              pack4(qf[0] * p8[r][0], qf[1] * p8[r][1], qf[2] * p8[r][2], qf[3] * p8[r][3]);
       } else {
         *reinterpret_cast<uint2*>(sm + OFF_KK8 + sw_off(r32, ch, 32)) =
             pack4(kf[0] * s8[r][0], kf[1] * s8[r][1], kf[2] * s8[r][2], kf[3] * s8[r][3]);
       }
-      // K'^T: channel rows, token columns; pairs of consecutive tokens pack into one word
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (r & 1) {
-          kpt[c][r >> 1] |= (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(kp[c])) << 16;
-        } else {
-          kpt[c][r >> 1] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(kp[c]));
-        }
-      }
+      for (int c = 0; c < 4; ++c) kpv[r][c] = kp[c];
     }
+    // K'^T: channel rows, token columns; pairs of consecutive tokens pack into one word
+    uint32_t kpt[4][4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) kpt[c][m] = pack_bf16(kpv[2 * m][c], kpv[2 * m + 1][c]);
     // the four stores rotate over the channels by lane so that each store instruction spreads
     // its 32 rows over all eight 16-byte bank groups
 #pragma unroll
@@ -412,7 +441,45 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     // diagonal 8x8 blocks on CUDA cores: partial sums over my 4 channels of
     //   A_rs (r > s, slots 0..27) and P_rs (r >= s, slots 28..63), then a butterfly
     //   reduce-scatter over the 32 lanes leaves slots 2*lane and 2*lane+1 in this lane
-    {
+    //   (build: A only, 32 slots, slot lane in this lane)
+    if constexpr (kBuild) {
+      float acc[32];
+      float kf[8][4];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const float2 k01 = unpack_bf16(k2[r].x), k23 = unpack_bf16(k2[r].y);
+        kf[r][0] = k01.x;
+        kf[r][1] = k01.y;
+        kf[r][2] = k23.x;
+        kf[r][3] = k23.y;
+      }
+#pragma unroll
+      for (int i = 28; i < 32; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        float w[4] = {kf[s][0], kf[s][1], kf[s][2], kf[s][3]};
+#pragma unroll
+        for (int r = s + 1; r < 8; ++r) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) w[c] *= al[r][c];
+          acc[r * (r - 1) / 2 + s] = kf[r][0] * w[0] + kf[r][1] * w[1] + kf[r][2] * w[2] + kf[r][3] * w[3];
+        }
+      }
+#pragma unroll
+      for (int half = 16; half >= 1; half >>= 1) {
+        const bool hi = (lane & half) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const float send = hi ? acc[i] : acc[i + half];
+          const float keep = hi ? acc[i + half] : acc[i];
+          acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+        }
+      }
+      if (lane < 28) {
+        const int rs = kDiagPair[lane], r = rs >> 3, sc = rs & 7;
+        sA[(warp * 8 + r) * kLdA + warp * 8 + sc] = acc[0];
+      }
+    } else {
       float acc[64];
       float kf[8][4], qf[8][4];
 #pragma unroll
@@ -478,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           uint32_t ak0, ak1, ak2, ak3, aq0, aq1, aq2, aq3, b00, b01, b10, b11;
           const int ar = 16 * pa + (m & 1) * 8 + (lane & 7), akc = 2 * kk + (m >> 1);
           ldsm_x4(sbase + OFF_KPI + sw_off(ar, akc * 8, 64), ak0, ak1, ak2, ak3);
-          ldsm_x4(sbase + OFF_QPI + sw_off(ar, akc * 8, 64), aq0, aq1, aq2, aq3);
+          if constexpr (!kBuild) ldsm_x4(sbase + OFF_QPI + sw_off(ar, akc * 8, 64), aq0, aq1, aq2, aq3);
           const int br = 16 * pb + (m >> 1) * 8 + (lane & 7), bkc = 2 * kk + (m & 1);
           ldsm_x4(sbase + OFF_KC + sw_off(br, bkc * 8, 64), b00, b01, b10, b11);
           if (pa - pb > 1) {  // adjacent 16-blocks have nothing between them
@@ -491,8 +558,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           }
           mma16816(accA[0], ak0, ak1, ak2, ak3, b00, b01);
           mma16816(accA[1], ak0, ak1, ak2, ak3, b10, b11);
-          mma16816(accP[0], aq0, aq1, aq2, aq3, b00, b01);
-          mma16816(accP[1], aq0, aq1, aq2, aq3, b10, b11);
+          if constexpr (!kBuild) {
+            mma16816(accP[0], aq0, aq1, aq2, aq3, b00, b01);
+            mma16816(accP[1], aq0, aq1, aq2, aq3, b10, b11);
+          }
         }
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -501,8 +570,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
             const int r = 16 * pa + g + 8 * hlf, s = 16 * pb + 8 * nt + 2 * t;
             sA[r * kLdA + s] = accA[nt][2 * hlf];
             sA[r * kLdA + s + 1] = accA[nt][2 * hlf + 1];
-            *reinterpret_cast<uint32_t*>(sm + OFF_P + sw_off(r, s, 64)) =
-                pack_bf16(accP[nt][2 * hlf], accP[nt][2 * hlf + 1]);
+            if constexpr (!kBuild)
+              *reinterpret_cast<uint32_t*>(sm + OFF_P + sw_off(r, s, 64)) =
+                  pack_bf16(accP[nt][2 * hlf], accP[nt][2 * hlf + 1]);
           }
         }
       } else {
@@ -516,16 +586,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
             uint32_t ak0, ak1, ak2, ak3, aq0, aq1, aq2, aq3, b0, b1;
             const int ar = 8 * bb + (lane & 7), akc = 2 * kk + (m >> 1);
             ldsm_x4(sbase + OFF_KPI8 + sw_off(ar, akc * 8, 32), ak0, ak1, ak2, ak3);
-            ldsm_x4(sbase + OFF_QPI8 + sw_off(ar, akc * 8, 32), aq0, aq1, aq2, aq3);
+            if constexpr (!kBuild) ldsm_x4(sbase + OFF_QPI8 + sw_off(ar, akc * 8, 32), aq0, aq1, aq2, aq3);
             const int br = 8 * bb + (lane & 7), bkc = 2 * kk + ((lane >> 3) & 1);
             ldsm_x2(sbase + OFF_KK8 + sw_off(br, bkc * 8, 32), b0, b1);
             mma16816(accA, ak0, ak1, ak2, ak3, b0, b1);
-            mma16816(accP, aq0, aq1, aq2, aq3, b0, b1);
+            if constexpr (!kBuild) mma16816(accP, aq0, aq1, aq2, aq3, b0, b1);
           }
           const int r = 16 * bb + 8 + g, s = 16 * bb + 2 * t;
           sA[r * kLdA + s] = accA[2];
           sA[r * kLdA + s + 1] = accA[3];
-          *reinterpret_cast<uint32_t*>(sm + OFF_P + sw_off(r, s, 64)) = pack_bf16(accP[2], accP[3]);
+          if constexpr (!kBuild)
+            *reinterpret_cast<uint32_t*>(sm + OFF_P + sw_off(r, s, 64)) = pack_bf16(accP[2], accP[3]);
         }
       }
     }
@@ -654,8 +725,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     if (c0 + C < t1) {
       if (tid == kPfThread) issue_prefetch_gkq(c0 + C);
       pf_pending = true;
+      load_beta(c0 + C);
     }
 
+    if constexpr (!kBuild) {
     // =============================== state side
     // D1 = S^T [K o Gamma ; Q o Gamma]^T   (M = 128, N = 128, K = 128)
     if (tid == kMmaThread) {
@@ -663,25 +736,25 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_bf16(tmD1, desc_sw128(sbase + OFF_S + koff), desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(128),
-                 kk > 0);
+        mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(128), kk > 0);
       }
       mma_commit(bar0);
     }
-    if (warp < 4) {
-      const int j = tid;
+    {
+      // epilogues run on all eight warps: warps w and w + 4 share TMEM lane quadrant w % 4
+      // (state row j) and split the columns
       if (!mbar_wait_bounded(bar0, phase, kWaitLimitNs)) {
         *s_abort = 1;
         report(a.status, KDA_ERR_DEVICE_TIMEOUT);
       } else {
         tc_fence_after();
         // Y^T[j][r] = -D1[j][r] = -((K o Gamma) S0)^T; V enters in the next product
-        float d[64];
-        tmem_ld16n<4>(tmD1 + lane_base, d);
+        float d[32];
+        tmem_ld16n<2>(tmD1 + lane_base + 32 * ehalf, d);
         tmem_wait_ld();
 #pragma unroll
-        for (int r0 = 0; r0 < C; r0 += 8)
-          *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(j, r0, 128)) =
+        for (int r0 = 0; r0 < 32; r0 += 8)
+          *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(ej, 32 * ehalf + r0, 128)) =
               make_uint4(pack_bf16(-d[r0], -d[r0 + 1]), pack_bf16(-d[r0 + 2], -d[r0 + 3]),
                          pack_bf16(-d[r0 + 4], -d[r0 + 5]), pack_bf16(-d[r0 + 6], -d[r0 + 7]));
       }
@@ -709,26 +782,25 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
                  (kk > 0) || !a.values_zero);
       mma_commit(bar1);
     }
-    if (warp < 4) {
-      const int j = tid;
+    {
       if (!mbar_wait_bounded(bar1, phase, kWaitLimitNs)) {
         *s_abort = 1;
         report(a.status, KDA_ERR_DEVICE_TIMEOUT);
       } else {
         tc_fence_after();
         {
-          float d[64];
-          tmem_ld16n<4>(tmD1 + lane_base, d);
+          float d[32];
+          tmem_ld16n<2>(tmD1 + lane_base + 32 * ehalf, d);
           tmem_wait_ld();
 #pragma unroll
-          for (int r0 = 0; r0 < C; r0 += 8)
-            *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(j, r0, 128)) =
+          for (int r0 = 0; r0 < 32; r0 += 8)
+            *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(ej, 32 * ehalf + r0, 128)) =
                 make_uint4(pack_bf16(d[r0], d[r0 + 1]), pack_bf16(d[r0 + 2], d[r0 + 3]),
                            pack_bf16(d[r0 + 4], d[r0 + 5]), pack_bf16(d[r0 + 6], d[r0 + 7]));
         }
         // decay the state columns: S^T[j][i] *= Gamma_63[i]
-#pragma unroll 1
-        for (int i0 = 0; i0 < D; i0 += 64) {
+        {
+          const int i0 = 64 * ehalf;
           float sv[64];
           tmem_ld16n<4>(tmS + lane_base + i0, sv);
           tmem_wait_ld();
@@ -770,8 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
                  idesc_bf16_f32(128), 1);
       mma_commit(bar2);
     }
-    if (warp < 4) {
-      const int j = tid;
+    {
       if (!mbar_wait_bounded(bar2, phase, kWaitLimitNs)) {
         *s_abort = 1;
         report(a.status, KDA_ERR_DEVICE_TIMEOUT);
@@ -780,29 +851,33 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         // outputs O[r][j] staged row-major (bf16 in the X tile, fp32 in the K/Q tile: both are
         // free once the last products completed; the V tile already receives the next chunk)
         if (a.out) {
-          float d[64];
-          tmem_ld16n<4>(tmD1 + lane_base + 64, d);
+          float d[32];
+          tmem_ld16n<2>(tmD1 + lane_base + 64 + 32 * ehalf, d);
           tmem_wait_ld();
           if (a.out_bf16) {
 #pragma unroll
-            for (int u = 0; u < C; ++u)
-              *reinterpret_cast<__nv_bfloat16*>(sm + OFF_X + (u * D + j) * 2) = __float2bfloat16_rn(d[u]);
+            for (int u = 0; u < 32; ++u)
+              *reinterpret_cast<__nv_bfloat16*>(sm + OFF_X + ((32 * ehalf + u) * D + ej) * 2) =
+                  __float2bfloat16_rn(d[u]);
           } else {
 #pragma unroll
-            for (int u = 0; u < C; ++u) reinterpret_cast<float*>(sm + OFF_KQ)[u * D + j] = d[u];
+            for (int u = 0; u < 32; ++u) reinterpret_cast<float*>(sm + OFF_KQ)[(32 * ehalf + u) * D + ej] = d[u];
           }
         }
-        // bf16 copy of the new state for the next chunk
-#pragma unroll 1
-        for (int i0 = 0; i0 < D; i0 += 64) {
+        // bf16 copy of the new state for the next chunk, into the TMEM A operand
+        {
+          const int i0 = 64 * ehalf;
           float sv[64];
           tmem_ld16n<4>(tmS + lane_base + i0, sv);
           tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 64; u += 8)
-            *reinterpret_cast<uint4*>(sm + OFF_S + sw_off(j, i0 + u, 128)) =
-                make_uint4(pack_bf16(sv[u], sv[u + 1]), pack_bf16(sv[u + 2], sv[u + 3]),
-                           pack_bf16(sv[u + 4], sv[u + 5]), pack_bf16(sv[u + 6], sv[u + 7]));
+          for (int q = 0; q < 4; ++q) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) pk[u] = pack_bf16(sv[16 * q + 2 * u], sv[16 * q + 2 * u + 1]);
+            tmem_st8u(tmSb + lane_base + i0 / 2 + 8 * q, pk);
+          }
+          tmem_wait_st();
         }
       }
       fence_async_smem();
@@ -830,24 +905,182 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
               *reinterpret_cast<const float4*>(sm + OFF_KQ + row * 512 + cc * 16);
       }
     }
+    } else {
+    // =============================== state side (segment build: both states, no readout)
+    {
+      // D1_M = S_M^T (K o Gamma)^T and D1_U = S_U^T (K o Gamma)^T   (N = 64 each, K = 128)
+      if (tid == kMmaThread) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
+          mma_bf16_ts(tmD1u, tmSbu + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
+        }
+        mma_commit(bar0);
+      }
+      if (!mbar_wait_bounded(bar0, phase, kWaitLimitNs)) {
+        *s_abort = 1;
+        report(a.status, KDA_ERR_DEVICE_TIMEOUT);
+      } else {
+        tc_fence_after();
+        float d[32], e[32];
+        tmem_ld16n<2>(tmD1 + lane_base + 32 * ehalf, d);
+        tmem_ld16n<2>(tmD1u + lane_base + 32 * ehalf, e);
+        tmem_wait_ld();
+#pragma unroll
+        for (int r0 = 0; r0 < 32; r0 += 8) {
+          *reinterpret_cast<uint4*>(sm + OFF_XM + sw_off(ej, 32 * ehalf + r0, 128)) =
+              make_uint4(pack_bf16(-d[r0], -d[r0 + 1]), pack_bf16(-d[r0 + 2], -d[r0 + 3]),
+                         pack_bf16(-d[r0 + 4], -d[r0 + 5]), pack_bf16(-d[r0 + 6], -d[r0 + 7]));
+          *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(ej, 32 * ehalf + r0, 128)) =
+              make_uint4(pack_bf16(-e[r0], -e[r0 + 1]), pack_bf16(-e[r0 + 2], -e[r0 + 3]),
+                         pack_bf16(-e[r0 + 4], -e[r0 + 5]), pack_bf16(-e[r0 + 6], -e[r0 + 7]));
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (*s_abort) {
+        aborted = true;
+        break;
+      }
+
+      // Delta_M^T = Y_M^T T^T ;  Delta_U^T = V^T T^T + Y_U^T T^T
+      if (tid == kMmaThread) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmD1, desc_sw128(sbase + OFF_XM + kk * 32), desc_sw128(sbase + OFF_T + kk * 32),
+                   idesc_bf16_f32(64), kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmD1u, desc_sw128_mn(sbase + OFF_V + kk * 2048, 8192), desc_sw128(sbase + OFF_T + kk * 32),
+                   idesc_bf16_f32(64, true), kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmD1u, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128(sbase + OFF_T + kk * 32),
+                   idesc_bf16_f32(64), 1);
+        mma_commit(bar1);
+      }
+      if (!mbar_wait_bounded(bar1, phase, kWaitLimitNs)) {
+        *s_abort = 1;
+        report(a.status, KDA_ERR_DEVICE_TIMEOUT);
+      } else {
+        tc_fence_after();
+        {
+          float d[32], e[32];
+          tmem_ld16n<2>(tmD1 + lane_base + 32 * ehalf, d);
+          tmem_ld16n<2>(tmD1u + lane_base + 32 * ehalf, e);
+          tmem_wait_ld();
+#pragma unroll
+          for (int r0 = 0; r0 < 32; r0 += 8) {
+            *reinterpret_cast<uint4*>(sm + OFF_XM + sw_off(ej, 32 * ehalf + r0, 128)) =
+                make_uint4(pack_bf16(d[r0], d[r0 + 1]), pack_bf16(d[r0 + 2], d[r0 + 3]),
+                           pack_bf16(d[r0 + 4], d[r0 + 5]), pack_bf16(d[r0 + 6], d[r0 + 7]));
+            *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(ej, 32 * ehalf + r0, 128)) =
+                make_uint4(pack_bf16(e[r0], e[r0 + 1]), pack_bf16(e[r0 + 2], e[r0 + 3]),
+                           pack_bf16(e[r0 + 4], e[r0 + 5]), pack_bf16(e[r0 + 6], e[r0 + 7]));
+          }
+        }
+        // decay both states: S^T[j][i] *= Gamma_63[i]
+#pragma unroll 1
+        for (int st = 0; st < 2; ++st) {
+          const uint32_t tcol = (st ? tmSu : tmS) + lane_base + 64 * ehalf;
+          float sv[64];
+          tmem_ld16n<4>(tcol, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 64; u += 4) {
+            const float4 gv = *reinterpret_cast<const float4*>(sGC + 64 * ehalf + u);
+            sv[u] *= gv.x;
+            sv[u + 1] *= gv.y;
+            sv[u + 2] *= gv.z;
+            sv[u + 3] *= gv.w;
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmem_st16(tcol + 16 * q, *reinterpret_cast<const float(*)[16]>(sv + 16 * q));
+        }
+        tmem_wait_st();
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (*s_abort) {
+        aborted = true;
+        break;
+      }
+      // the V tile is free now that the second products completed
+      if (c0 + C < t1 && tid == kPfThread) issue_prefetch_v(c0 + C);
+
+      // S_M^T += Delta_M^T K' ;  S_U^T += Delta_U^T K'
+      if (tid == kMmaThread) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmS, desc_sw128(sbase + OFF_XM + kk * 32), desc_sw128(sbase + OFF_KPT + kk * 32),
+                   idesc_bf16_f32(128), 1);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(tmSu, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128(sbase + OFF_KPT + kk * 32),
+                   idesc_bf16_f32(128), 1);
+        mma_commit(bar2);
+      }
+      if (!mbar_wait_bounded(bar2, phase, kWaitLimitNs)) {
+        *s_abort = 1;
+        report(a.status, KDA_ERR_DEVICE_TIMEOUT);
+      } else {
+        tc_fence_after();
+        // bf16 copies of both new states for the next chunk's first products
+#pragma unroll 1
+        for (int st = 0; st < 2; ++st) {
+          const int i0 = 64 * ehalf;
+          float sv[64];
+          tmem_ld16n<4>((st ? tmSu : tmS) + lane_base + i0, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) pk[u] = pack_bf16(sv[16 * q + 2 * u], sv[16 * q + 2 * u + 1]);
+            tmem_st8u((st ? tmSbu : tmSb) + lane_base + i0 / 2 + 8 * q, pk);
+          }
+        }
+        tmem_wait_st();
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (*s_abort) {
+        aborted = true;
+        break;
+      }
+    }
+    }
   }
 
-  if (!aborted && warp < 4) {
-    // final state back to the pool slot
+  if (!aborted) {
+    // final state(s): the pool slot (prefill), or M and U of this segment (build); row j, columns
+    // split between the two warps of a quadrant
     tc_fence_after();
-    const int j = tid;
 #pragma unroll 1
-    for (int i0 = 0; i0 < D; i0 += 16) {
-      float sv[16];
-      tmem_ld16(tmS + lane_base + i0, sv);
-      tmem_wait_ld();
-      if (a.v_first) {
-        float4* p = reinterpret_cast<float4*>(out_blk + (size_t)j * D + i0);
+    for (int st = 0; st < (kBuild ? 2 : 1); ++st) {
+      float* dst = st ? a.state_out2 + blk_off : out_blk;
+      const bool vf = (kBuild && st == 0) ? false : (a.v_first != 0);
+      const uint32_t tcol = st ? tmSu : tmS;
+#pragma unroll 1
+      for (int i0 = 64 * ehalf; i0 < 64 * ehalf + 64; i0 += 16) {
+        float sv[16];
+        tmem_ld16(tcol + lane_base + i0, sv);
+        tmem_wait_ld();
+        if (vf) {
+          float4* p = reinterpret_cast<float4*>(dst + (size_t)ej * D + i0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) p[q] = make_float4(sv[4 * q], sv[4 * q + 1], sv[4 * q + 2], sv[4 * q + 3]);
-      } else {
+          for (int q = 0; q < 4; ++q) p[q] = make_float4(sv[4 * q], sv[4 * q + 1], sv[4 * q + 2], sv[4 * q + 3]);
+        } else {
 #pragma unroll
-        for (int u = 0; u < 16; ++u) out_blk[(size_t)(i0 + u) * D + j] = sv[u];
+          for (int u = 0; u < 16; ++u) dst[(size_t)(i0 + u) * D + ej] = sv[u];
+        }
       }
     }
   }
@@ -898,7 +1131,10 @@ bool encode_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint3
 }  // namespace
 
 cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream) {
-  cudaError_t err = cudaFuncSetAttribute(fused_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+  cudaError_t err = cudaFuncSetAttribute(fused_chunk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemAlloc);
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(fused_chunk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   if (err != cudaSuccess) return err;
   if (a.batch == 0) return cudaSuccess;
   InputMaps tm;
@@ -912,7 +1148,10 @@ cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream) {
                               CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
   dim3 grid(a.Hv, a.batch);
-  fused_chunk_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(a, tm);
+  if (a.build)
+    fused_chunk_kernel<true><<<grid, kThreads, kSmemAlloc, stream>>>(a, tm);
+  else
+    fused_chunk_kernel<false><<<grid, kThreads, kSmemAlloc, stream>>>(a, tm);
   return cudaGetLastError();
 }
 

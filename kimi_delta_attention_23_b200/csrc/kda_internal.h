@@ -61,7 +61,11 @@ struct FusedArgs {
   int64_t total_tokens;
   int32_t Hk, Hv;
   const float* state_in;    // read when init_mode == 0 (pool base)
-  float* state_out;         // final state destination (pool base; may equal state_in)
+  float* state_out;         // final state destination (pool base; may equal state_in); with
+                            // build: the transitions M [N][Hv][128][128]
+  float* state_out2;        // build only: the contributions U [N][Hv][128][128] (layout v_first)
+  int32_t build;            // 1: segment build -- transition (from I, zero values) and contribution
+                            // (from 0, real values) carried together, no readout
   int32_t max_slots;
   const int32_t* slots;     // [batch] or NULL (slot = sequence index)
   int32_t v_first;          // state blocks stored transposed ([dv][dk])
