@@ -109,68 +109,90 @@ def recorded_traffic(kernel):
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons sampled during the timed region.
 
-    def __init__(self, device_index=0):
-        self.proc = None
-        self.path = os.path.join("/tmp", f"kda_clocks_{os.getpid()}.csv")
-        sel = []
+    Polls NVML from a background thread every few milliseconds (the timed region can be far
+    shorter than nvidia-smi's sampling interval); falls back to nvidia-smi if NVML is absent."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, device_index=0, period_s=0.005):
+        self.device_index, self.period = device_index, period_s
+        self.samples, self.thread, self.stop_flag, self.nvml = [], None, False, None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        pr = torch.cuda.get_device_properties(self.device_index)
+        bus = "%08X:%02X:%02X.0" % (int(pr.pci_domain_id), int(pr.pci_bus_id), int(pr.pci_device_id))
         try:
-            pr = torch.cuda.get_device_properties(device_index)
-            sel = ["-i", "%08X:%02X:%02X.0" % (int(pr.pci_domain_id), int(pr.pci_bus_id), int(pr.pci_device_id))]
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
         except Exception:
-            sel = []
-        self.cmd = ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.device_index)
+
+    def _run(self):
+        nv, hnd = self.nvml
+        while not self.stop_flag:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(hnd, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(hnd, nv.NVML_CLOCK_SM)
+                get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                rs = get_reasons(hnd)
+                pw = nv.nvmlDeviceGetPowerUsage(hnd) / 1000.0
+                self.samples.append((sm, mx, rs, pw))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def __enter__(self):
-        if len(self.cmd) > 2 and self.cmd[1] == "-i":
-            try:
-                r = subprocess.run(["nvidia-smi", "-i", self.cmd[2], "--query-gpu=index", "--format=csv,noheader"],
-                                   capture_output=True, text=True, timeout=20)
-                if r.returncode != 0 or not r.stdout.strip():
-                    self.cmd = [self.cmd[0]] + self.cmd[3:]
-            except Exception:
-                self.cmd = [self.cmd[0]] + self.cmd[3:]
+        import threading
         try:
-            self.fh = open(self.path, "w")
-            self.proc = subprocess.Popen(self.cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
+            self.nvml = self._handle()
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+            time.sleep(0.02)  # the first samples land before the timed work starts
         except Exception:
-            self.proc = None
+            self.nvml = None
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            self.fh.close()
+        self.stop_flag = True
+        if self.thread is not None:
+            self.thread.join(timeout=2)
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(float(r[2]) for r in rows),
-                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit()),
-                "samples": len(rows), "reasons": reasons}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock samples (NVML unavailable)"]}
+        sm = [s[0] for s in self.samples]
+        reasons = sorted({n for s in self.samples for n, bit in self.REASONS.items() if s[2] & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(s[1] for s in self.samples),
+                "power_w_max": max(s[3] for s in self.samples), "samples": len(self.samples), "reasons": reasons,
+                "source": "nvml"}
 
 
 def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def rank_seed(workload, rank):
+    """Seed of a rank's own replica: rank 0 uses the workload's seed, others a distinct one."""
+    return None if rank == 0 else 1000 * rank + W.WORKLOADS.index(workload)
+
+
+def max_over_ranks(value, pg, device="cpu"):
+    """The slowest rank's time (every rank takes part; the result is the same everywhere)."""
+    if pg is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_throughput(units_per_rank, world, ms_per_step):
+    """Units all ranks processed per second, timed by the slowest rank (weak scaling)."""
+    return units_per_rank * world / (ms_per_step / 1e3)
 
 
 # ------------------------------------------------------------------------------------------
@@ -301,7 +323,7 @@ def run_ours(args):
         pg = dist
     from kimi_delta_attention_23_b200 import build as kbuild
     kbuild.build()
-    w = W.make(args.workload, device=dev, seed=None if rank == 0 else 1000 * rank + W.WORKLOADS.index(args.workload))
+    w = W.make(args.workload, device=dev, seed=rank_seed(args.workload, rank))
     stream = torch.cuda.current_stream(dev)
     step = Step(w, stream)
     for _ in range(args.warmup):
@@ -329,13 +351,10 @@ def run_ours(args):
     ms_total = start.elapsed_time(stop)
     seg_ms = [e[0].elapsed_time(e[1]) for e in step.events]
     pass_ms = [e[1].elapsed_time(e[2]) for e in step.events]
-    if pg is not None:
-        t = torch.tensor([ms_total], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, pg, dev)
     ms_step = ms_total / args.steps
     tokens = w.total_tokens
-    value = tokens * world / (ms_total / args.steps / 1e3)
+    value = whole_job_throughput(tokens, world, ms_step)
 
     e2e = None
     if not args.no_e2e:
@@ -414,13 +433,9 @@ def measure_e2e(w, args, stream, pg):
         one()
     stop.record(stream)
     torch.cuda.synchronize()
-    ms = start.elapsed_time(stop)
-    if pg is not None:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(stop), pg, dev)
     world = pg.get_world_size() if pg is not None else 1
-    return {"value": w.total_tokens * world / (ms / n / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+    return {"value": whole_job_throughput(w.total_tokens, world, ms / n), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n}
 
 
