@@ -4,10 +4,11 @@
 A step is one pass of the whole hot path over one batch of synthetic input.  For the default
 workload (one 131072-token sequence, 32 value heads, dk = dv = 128, bf16 q/k/v, fp32 gates and
 state, cut into 16 segments of 8192) a step is the context-parallel prefill:
-  1. kda_segment_summarize_and_scan: per-segment transition M_i and contribution U_i for every
-     head, then the exclusive affine scan (incoming / outgoing / final states);
-  2. kda_chunk_fwd over the 16 segments as independent sequences, each starting from its
-     incoming state -- every output row of the sequence plus the final state.
+  1. kda_segment_summarize_and_scan with q: every segment in parallel builds its transition M_i,
+     its contribution U_i and each token's two local readouts, then the exclusive affine scan
+     gives incoming / outgoing / final states;
+  2. kda_context_parallel_apply: every output row from its readouts and its segment's incoming
+     state.
 Other workloads (``--workload``) time one kda_chunk_fwd call over the whole batch; their
 state pool carries over from step to step (each step resumes from the previous final states,
 as a split prefill would), so the timed work never includes a pool restore.
@@ -56,13 +57,23 @@ def chunk_fwd_bytes(w, num_seqs, dk=128, dv=128):
     return th * io_bytes_per_token_head(qkv, ob, dk, dv, group) + num_seqs * w.num_v_heads * 2 * dk * dv * 4
 
 
-def segment_bytes(w, N, dk=128, dv=128):
+def segment_build_bytes(w, N, dk=128, dv=128):
+    """Segment build with readouts (q, k, v, gate, beta in; both bf16 readouts, M and U out) plus
+    the scan (M, U, initial in; incoming, outgoing, final out)."""
     th = w.total_tokens * w.num_v_heads
-    qkv = 2 if w.q.dtype == torch.bfloat16 else 4
-    reads = th * (dk * qkv + dv * qkv + dk * 4 + 4)
+    group = w.num_v_heads // w.num_k_heads
+    reads = th * ((2 * dk * 2) / group + dv * 2 + dk * 4 + 4)
+    readouts = th * 2 * dv * 2
     summaries = N * w.num_v_heads * (dk * dk + dk * dv) * 4
-    scan = N * w.num_v_heads * dk * dv * 4 * 2 + summaries  # incoming + outgoing written, M/U re-read
-    return reads + summaries + scan
+    scan = summaries + N * w.num_v_heads * dk * dv * 4 * 2
+    return reads + readouts + summaries + scan
+
+
+def apply_bytes(w, N, dv=128):
+    """Readouts and incoming states in, outputs out."""
+    th = w.total_tokens * w.num_v_heads
+    ob = 2 if w.output_dtype == torch.bfloat16 else 4
+    return th * (2 * dv * 2 + dv * ob) + N * w.num_v_heads * dv * dv * 4
 
 
 def chunk_fwd_flops(w, C=64, dk=128, dv=128):
@@ -276,7 +287,8 @@ class Step:
             self.inc = torch.empty((N, Hv, *st), device=dev)
             self.outg = torch.empty((N, Hv, *st), device=dev)
             self.fin = torch.empty((Hv, *st), device=dev)
-            self.seg_idx = torch.arange(N, dtype=torch.int32, device=dev)
+            self.rm = torch.empty((T, Hv, dv), dtype=torch.bfloat16, device=dev)
+            self.ru = torch.empty((T, Hv, dv), dtype=torch.bfloat16, device=dev)
         self.pool = None if self.cp else w.state_pool.clone()
         self.events = []
 
@@ -286,7 +298,7 @@ class Step:
                     gate_lower_bound=w.gate_lower_bound, device_status=self.status, stream=self.stream)
 
     def launches(self):
-        return 4 if self.cp else 1  # transition build, contribution build, scan, chunk pass
+        return 3 if self.cp else 1  # segment build with readouts, scan, apply
 
     def __call__(self, record=False):
         w, kda = self.w, self.kda
@@ -296,11 +308,13 @@ class Step:
         if self.cp:
             kda.kda_segment_summarize_and_scan(w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias,
                                                w.seg_offsets, self.init, M=self.M, U=self.U, incoming=self.inc,
-                                               outgoing=self.outg, final_state=self.fin, **self.kw())
+                                               outgoing=self.outg, final_state=self.fin, q=w.q, readout_m=self.rm,
+                                               readout_u=self.ru, **self.kw())
             if ev:
                 ev[1].record(self.stream)
-            kda.kda_chunk_fwd(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.seg_offsets,
-                              self.inc, self.seg_idx, self.out, **self.kw())
+            kda.kda_context_parallel_apply(self.rm, self.ru, self.inc, w.seg_offsets, self.out,
+                                           state_layout=w.state_layout, device_status=self.status,
+                                           stream=self.stream)
         else:
             if ev:
                 ev[1].record(self.stream)
@@ -365,15 +379,20 @@ def run_ours(args):
             pg.destroy_process_group()
         return 0
     pk = peaks()
-    n_seq = (step.N if step.cp else w.batch)
-    bytes_pass = chunk_fwd_bytes(w, n_seq)
     ms_pass = statistics.mean(pass_ms)
     ms_seg = statistics.mean(seg_ms) if step.cp else 0.0
-    achieved = bytes_pass / (ms_pass / 1e3) / 1e9
-    dom = "kda_chunk_fwd"
+    if step.cp:
+        # dominant launch: the segment build with readouts (its call also runs the short scan)
+        dom, bytes_dom, ms_dom = "fused_chunk_kernel<build,readout> + affine_scan_kernel", \
+            segment_build_bytes(w, step.N), ms_seg
+        breakdown = {"segment_build_and_scan": ms_seg, "context_parallel_apply": ms_pass}
+    else:
+        dom, bytes_dom, ms_dom = "fused_chunk_kernel<prefill>", chunk_fwd_bytes(w, w.batch), ms_pass
+        breakdown = {"chunk_fwd": ms_pass}
+    achieved = bytes_dom / (ms_dom / 1e3) / 1e9
     roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / pk["hbm_gbs"], "traffic": recorded_traffic(dom),
-            "algorithmic_bytes_per_launch": bytes_pass, "ms_per_launch": ms_pass,
+            "algorithmic_bytes_per_launch": bytes_dom, "ms_per_launch": ms_dom,
             "peak_source": pk["source"]}
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -382,8 +401,9 @@ def run_ours(args):
                        "num_k_heads": w.num_k_heads, "dk": w.dk, "dv": w.dv, "batch": w.batch,
                        "segments": step.N if step.cp else None, "gate_mode": w.gate_mode,
                        "state_layout": w.state_layout, "parallelism": f"dp{world}" if world > 1 else "single",
-                       "l2": "inputs larger than L2 (%.2f GB read per step), no flush" % (bytes_pass / 1e9)},
-            "breakdown_ms": {"segment_summarize_and_scan": ms_seg, "chunk_fwd": ms_pass},
+                       "l2": "inputs larger than L2 (%.2f GB read per step), no flush" % (
+                           (segment_build_bytes(w, step.N) if step.cp else chunk_fwd_bytes(w, w.batch)) / 1e9)},
+            "breakdown_ms": breakdown,
             "roofline": roof, "gpu_launches": step.launches() * args.steps, "clocks": clocks.summary()}
     if e2e is not None:
         line["e2e"] = e2e

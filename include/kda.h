@@ -137,14 +137,71 @@ KDA_API kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, 
  * values); U_i is its local contribution (the recurrence from S = 0).  Left multiplication:
  * out_i = M_i in_i + U_i.  initial_state, M and U (in SCAN_ONLY mode) are never written.
  * Summaries need dk <= 128 and dv <= 128 (fp32 or bf16 k/v).
+ *
+ *   q, readout_m, readout_u  optional (all three or none; bf16 k/v with dk = dv = 128 only):
+ *   q [T, Hk, 128] bf16; the build then also writes, per token, the readout through the
+ *   transition readout_m[t] = q_t^T M_{<=t} and of the contribution readout_u[t] = q_t^T U_{<=t}
+ *   ([T, Hv, 128] bf16 each), the inputs of kda_context_parallel_apply.
  */
 KDA_API kda_status_t kda_segment_summarize_and_scan(
     const void *k, const void *v, kda_dtype_t kv_dtype, const float *raw_gate,
     const float *beta_logits, const float *a_log, const float *dt_bias, int64_t T,
     int32_t num_k_heads, int32_t num_v_heads, int32_t dk, int32_t dv, const int32_t *seg_offsets,
     int32_t num_segments, const float *initial_state, float *M, float *U, float *incoming,
-    float *outgoing, float *final_state, uint32_t flags, float gate_lower_bound, void *workspace,
-    size_t workspace_bytes, int32_t *device_status, void *stream);
+    float *outgoing, float *final_state, const void *q, void *readout_m, void *readout_u,
+    uint32_t flags, float gate_lower_bound, void *workspace, size_t workspace_bytes,
+    int32_t *device_status, void *stream);
+
+/*
+ * kda_context_parallel_apply -- outputs of every segment from its local readouts and its
+ * incoming state ("KDA Context Parallelism", Theory: a segment applied to any incoming state
+ * without replaying its tokens).  Inside a segment the state after token t is
+ * M_{<=t} S_in + U_{<=t}, so out_t = readout_m[t] . S_in + readout_u[t] with
+ * readout_m[t] = q_t^T M_{<=t} and readout_u[t] = q_t^T U_{<=t}.
+ *
+ *   readout_m, readout_u [T, Hv, 128] bf16 (from kda_segment_summarize_and_scan)
+ *   incoming [N, Hv, <state>] fp32 (flags: KDA_STATE_V_FIRST for the transposed layout)
+ *   out [T, Hv, 128] out_dtype
+ * dv must be 128; bad segment offsets are reported in device_status and that segment skipped.
+ */
+KDA_API kda_status_t kda_context_parallel_apply(const void *readout_m, const void *readout_u,
+                                                const float *incoming, const int32_t *seg_offsets,
+                                                int32_t num_segments, int64_t T, int32_t num_v_heads,
+                                                int32_t dv, void *out, kda_dtype_t out_dtype,
+                                                uint32_t flags, int32_t *device_status, void *stream);
+
+/*
+ * kda_context_parallel_prefill -- the whole prefill of ONE long sequence, context-parallel on
+ * one GPU ("KDA Context Parallelism": segment summaries, ordered composition, exclusive scan;
+ * "max.nn.state_space.kda_chunk" semantics for every token).
+ *
+ * The sequence is cut at seg_offsets [N+1] (device int32, 0 .. T, non-decreasing).  One pass
+ * over all segments in parallel builds each segment's transition M_i, contribution U_i and two
+ * local readouts per token -- through the transition (q_t^T M_{<=t}, dk wide) and of the
+ * contribution (q_t^T U_{<=t}) -- into the workspace; the exclusive scan gives every segment its
+ * incoming state; a last pass forms out_t = (q_t^T M_{<=t}) S_in + q_t^T U_{<=t}, which equals
+ * the token-by-token recurrence started from initial_state.
+ *
+ *   q, k, v, raw_gate, beta_logits, a_log, dt_bias   as kda_chunk_fwd, one sequence of T tokens
+ *   initial_state [Hv, <state>] fp32, read only;  final_state [Hv, <state>] fp32, written
+ *   out [T, Hv, dv] out_dtype (BF16 or F32)
+ *   M [N,Hv,dk,dk], U / incoming / outgoing [N,Hv,<state>] fp32, written (as in
+ *     kda_segment_summarize_and_scan)
+ *   workspace >= kda_context_parallel_workspace_size(T, num_v_heads, dv) bytes, 256-byte aligned
+ *     device memory; its contents on return are unspecified
+ * Supported: bf16 q/k/v with dk = dv = 128; otherwise KDA_ERR_UNSUPPORTED.
+ */
+KDA_API kda_status_t kda_context_parallel_prefill(
+    const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype, const float *raw_gate,
+    const float *beta_logits, const float *a_log, const float *dt_bias, int64_t T,
+    int32_t num_k_heads, int32_t num_v_heads, int32_t dk, int32_t dv, const int32_t *seg_offsets,
+    int32_t num_segments, const float *initial_state, void *out, kda_dtype_t out_dtype,
+    float *final_state, float *M, float *U, float *incoming, float *outgoing, uint32_t flags,
+    float gate_lower_bound, void *workspace, size_t workspace_bytes, int32_t *device_status,
+    void *stream);
+
+/* Workspace bytes kda_context_parallel_prefill needs: the two bf16 readouts, 2 * T * Hv * dv * 2. */
+KDA_API size_t kda_context_parallel_workspace_size(int64_t T, int32_t num_v_heads, int32_t dv);
 
 /* Bytes of workspace kda_chunk_fwd / kda_segment_summarize_and_scan need for these extents
  * (0 for the current kernels). */

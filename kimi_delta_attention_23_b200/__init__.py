@@ -9,6 +9,7 @@ Public calls (same names as the C ABI):
   kda_segment_summarize_and_scan(...)     segment (M_i, U_i) summaries + exclusive scan
   kda_context_parallel(M, U, initial)     the scan alone, returning exactly incoming_states,
                                           outgoing_states and final_state
+  kda_context_parallel_prefill(...)       the context-parallel prefill of one long sequence
 """
 from __future__ import annotations
 
@@ -18,7 +19,8 @@ import os
 import torch
 
 __all__ = ["kda_chunk_fwd", "kda_segment_summarize_and_scan", "kda_context_parallel",
-           "kda_workspace_size", "kda_status_string", "load_library", "KdaError", "LIB_PATH"]
+           "kda_context_parallel_apply", "kda_context_parallel_prefill", "kda_context_parallel_workspace_size", "kda_workspace_size",
+           "kda_status_string", "load_library", "KdaError", "LIB_PATH"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkda.so")
@@ -58,8 +60,16 @@ def load_library():
                                   i32, fp, i32, ip, vp, ctypes.c_int, u32, f32, vp, sz, ip, vp]
     lib.kda_segment_summarize_and_scan.restype = ctypes.c_int
     lib.kda_segment_summarize_and_scan.argtypes = [vp, vp, ctypes.c_int, fp, fp, fp, fp, i64, i32, i32,
-                                                   i32, i32, ip, i32, fp, fp, fp, fp, fp, fp, u32, f32,
-                                                   vp, sz, ip, vp]
+                                                   i32, i32, ip, i32, fp, fp, fp, fp, fp, fp, vp, vp, vp, u32,
+                                                   f32, vp, sz, ip, vp]
+    lib.kda_context_parallel_apply.restype = ctypes.c_int
+    lib.kda_context_parallel_apply.argtypes = [vp, vp, fp, ip, i32, i64, i32, i32, vp, ctypes.c_int, u32, ip, vp]
+    lib.kda_context_parallel_prefill.restype = ctypes.c_int
+    lib.kda_context_parallel_prefill.argtypes = [vp, vp, vp, ctypes.c_int, fp, fp, fp, fp, i64, i32, i32, i32, i32,
+                                                 ip, i32, fp, vp, ctypes.c_int, fp, fp, fp, fp, fp, u32, f32, vp, sz,
+                                                 ip, vp]
+    lib.kda_context_parallel_workspace_size.restype = sz
+    lib.kda_context_parallel_workspace_size.argtypes = [i64, i32, i32]
     lib.kda_workspace_size.restype = sz
     lib.kda_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32, i32, u32]
     lib.kda_status_string.restype = ctypes.c_char_p
@@ -181,14 +191,16 @@ def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, st
 
 def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, seg_offsets, initial_state,
                                    *, M=None, U=None, incoming=None, outgoing=None, final_state=None,
-                                   scan_only=False, gate_mode="original", beta_mode="logits",
-                                   state_layout="K_FIRST", gate_lower_bound=-5.0, device_status=None,
-                                   stream=None):
+                                   q=None, readout_m=None, readout_u=None, scan_only=False, gate_mode="original",
+                                   beta_mode="logits", state_layout="K_FIRST", gate_lower_bound=-5.0,
+                                   device_status=None, stream=None):
     """Segment summaries (M_i, U_i) of one sequence and the exclusive scan over them.
 
     Returns dict(incoming_states, outgoing_states, final_state, transition_matrices,
-    local_contributions); the segment axis leads every stack.  With ``scan_only`` the given
-    M and U are inputs and are not written.
+    local_contributions[, readout_m, readout_u]); the segment axis leads every stack.  With
+    ``scan_only`` the given M and U are inputs and are not written.  With ``q`` (bf16, 128-wide
+    heads) the build also returns each token's readouts through the transition and of the
+    contribution, the inputs of ``kda_context_parallel_apply``.
     """
     lib = load_library()
     dev = initial_state.device
@@ -229,18 +241,52 @@ def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, 
     incoming = buf(incoming, "incoming", (N, Hv, *st))
     outgoing = buf(outgoing, "outgoing", (N, Hv, *st))
     final_state = buf(final_state, "final_state", (Hv, *st))
+    if q is not None:
+        _shape(_dev(q, "q", torch.bfloat16, dev), "q", (T, Hk, dk))
+        if readout_m is None:
+            readout_m = torch.empty((T, Hv, dv), dtype=torch.bfloat16, device=dev)
+        if readout_u is None:
+            readout_u = torch.empty((T, Hv, dv), dtype=torch.bfloat16, device=dev)
+        _shape(_dev(readout_m, "readout_m", torch.bfloat16, dev), "readout_m", (T, Hv, dv))
+        _shape(_dev(readout_u, "readout_u", torch.bfloat16, dev), "readout_u", (T, Hv, dv))
     flags = _flags(gate_mode, beta_mode, state_layout, scan_only=scan_only)
     rc = lib.kda_segment_summarize_and_scan(
         _ptr(k) if not scan_only else None, _ptr(v) if not scan_only else None, kv_dtype,
         _ptr(raw_gate) if not scan_only else None, _ptr(beta_logits) if not scan_only else None,
         _ptr(a_log) if not scan_only else None, _ptr(dt_bias) if not scan_only else None, T, Hk, Hv, dk, dv,
         _ptr(seg_offsets) if not scan_only else None, N, _ptr(initial_state), _ptr(M), _ptr(U),
-        _ptr(incoming), _ptr(outgoing), _ptr(final_state), flags, float(gate_lower_bound), None, 0,
-        _ptr(device_status), _stream(stream, dev))
+        _ptr(incoming), _ptr(outgoing), _ptr(final_state), _ptr(q), _ptr(readout_m), _ptr(readout_u), flags,
+        float(gate_lower_bound), None, 0, _ptr(device_status), _stream(stream, dev))
     if rc != 0:
         raise KdaError(rc, "kda_segment_summarize_and_scan")
-    return {"incoming_states": incoming, "outgoing_states": outgoing, "final_state": final_state,
-            "transition_matrices": M, "local_contributions": U}
+    res = {"incoming_states": incoming, "outgoing_states": outgoing, "final_state": final_state,
+           "transition_matrices": M, "local_contributions": U}
+    if q is not None:
+        res["readout_m"], res["readout_u"] = readout_m, readout_u
+    return res
+
+
+def kda_context_parallel_apply(readout_m, readout_u, incoming, seg_offsets, out=None, *, output_dtype=torch.bfloat16,
+                               state_layout="K_FIRST", device_status=None, stream=None):
+    """out_t = readout_m[t] . S_in(segment of t) + readout_u[t] for every token."""
+    lib = load_library()
+    dev = incoming.device
+    _dev(readout_m, "readout_m", torch.bfloat16, dev)
+    T, Hv, dv = readout_m.shape
+    _shape(_dev(readout_u, "readout_u", torch.bfloat16, dev), "readout_u", (T, Hv, dv))
+    _dev(incoming, "incoming", torch.float32, dev)
+    _dev(seg_offsets, "seg_offsets", torch.int32, dev)
+    N = seg_offsets.numel() - 1
+    if out is None:
+        out = torch.empty((T, Hv, dv), dtype=output_dtype, device=dev)
+    _shape(_dev(out, "out", None, dev), "out", (T, Hv, dv))
+    rc = lib.kda_context_parallel_apply(_ptr(readout_m), _ptr(readout_u), _ptr(incoming), _ptr(seg_offsets), N, T,
+                                        Hv, dv, _ptr(out), _DTYPES[out.dtype], _flags("original", "logits",
+                                                                                      state_layout),
+                                        _ptr(device_status), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_context_parallel_apply")
+    return out
 
 
 def kda_context_parallel(transition_matrices, local_contributions, initial_state, *, state_layout="K_FIRST",
@@ -270,3 +316,67 @@ def kda_context_parallel(transition_matrices, local_contributions, initial_state
         out = {"incoming_states": out["incoming_states"][:, 0], "outgoing_states": out["outgoing_states"][:, 0],
                "final_state": out["final_state"][0]}
     return out
+
+
+def kda_context_parallel_workspace_size(T, num_v_heads, dv=128) -> int:
+    return int(load_library().kda_context_parallel_workspace_size(T, num_v_heads, dv))
+
+
+def kda_context_parallel_prefill(q, k, v, raw_gate, beta_logits, a_log, dt_bias, seg_offsets, initial_state,
+                                 out=None, *, final_state=None, M=None, U=None, incoming=None, outgoing=None,
+                                 workspace=None, output_dtype=None, gate_mode="original", beta_mode="logits",
+                                 state_layout="K_FIRST", gate_lower_bound=-5.0, device_status=None, stream=None):
+    """Context-parallel prefill of one sequence (bf16 q/k/v, dk = dv = 128) cut at seg_offsets.
+
+    Returns dict(out, final_state, incoming_states, outgoing_states, transition_matrices,
+    local_contributions).  ``workspace`` (uint8 CUDA tensor of at least
+    kda_context_parallel_workspace_size bytes) is allocated when not given.
+    """
+    lib = load_library()
+    dev = q.device
+    _dev(q, "q", torch.bfloat16, dev)
+    T, Hk, dk = q.shape
+    _shape(_dev(k, "k", torch.bfloat16, dev), "k", (T, Hk, dk))
+    _dev(v, "v", torch.bfloat16, dev)
+    Hv, dv = v.shape[1], v.shape[2]
+    _shape(v, "v", (T, Hv, dv))
+    _shape(_dev(raw_gate, "raw_gate", torch.float32, dev), "raw_gate", (T, Hv, dk))
+    _shape(_dev(beta_logits, "beta_logits", torch.float32, dev), "beta_logits", (T, Hv))
+    _shape(_dev(a_log, "a_log", torch.float32, dev), "a_log", (Hv,))
+    _shape(_dev(dt_bias, "dt_bias", torch.float32, dev), "dt_bias", (Hv, dk))
+    _dev(seg_offsets, "seg_offsets", torch.int32, dev)
+    N = seg_offsets.numel() - 1
+    st = (dk, dv) if state_layout == "K_FIRST" else (dv, dk)
+    _shape(_dev(initial_state, "initial_state", torch.float32, dev), "initial_state", (Hv, *st))
+    if output_dtype is None:
+        output_dtype = v.dtype if out is None else out.dtype
+    if out is None:
+        out = torch.empty((T, Hv, dv), dtype=output_dtype, device=dev)
+    _shape(_dev(out, "out", output_dtype, dev), "out", (T, Hv, dv))
+
+    def buf(t, name, shape):
+        if t is None:
+            return torch.empty(shape, dtype=torch.float32, device=dev)
+        _shape(_dev(t, name, torch.float32, dev), name, shape)
+        return t
+
+    final_state = buf(final_state, "final_state", (Hv, *st))
+    M = buf(M, "M", (N, Hv, dk, dk))
+    U = buf(U, "U", (N, Hv, *st))
+    incoming = buf(incoming, "incoming", (N, Hv, *st))
+    outgoing = buf(outgoing, "outgoing", (N, Hv, *st))
+    need = kda_context_parallel_workspace_size(T, Hv, dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _dev(workspace, "workspace", torch.uint8, dev)
+    flags = _flags(gate_mode, beta_mode, state_layout)
+    rc = lib.kda_context_parallel_prefill(_ptr(q), _ptr(k), _ptr(v), _BF16, _ptr(raw_gate), _ptr(beta_logits),
+                                          _ptr(a_log), _ptr(dt_bias), T, Hk, Hv, dk, dv, _ptr(seg_offsets), N,
+                                          _ptr(initial_state), _ptr(out), _DTYPES[output_dtype], _ptr(final_state),
+                                          _ptr(M), _ptr(U), _ptr(incoming), _ptr(outgoing), flags,
+                                          float(gate_lower_bound), _ptr(workspace), workspace.numel(),
+                                          _ptr(device_status), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_context_parallel_prefill")
+    return {"out": out, "final_state": final_state, "incoming_states": incoming, "outgoing_states": outgoing,
+            "transition_matrices": M, "local_contributions": U}

@@ -3,6 +3,7 @@
 // Shapes, flags and the state pool follow "max.nn.state_space.kda_chunk" (Parameters, Returns,
 // Raises): a dtype grouping that binds no kernel, or ranks/extents that disagree, is an error.
 // Unlike that op, whose shape guards are debug-only, every check here is always on.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "../../include/kda.h"
@@ -118,12 +119,15 @@ extern "C" kda_status_t kda_segment_summarize_and_scan(
     const void* k, const void* v, kda_dtype_t kv_dtype, const float* raw_gate, const float* beta_logits,
     const float* a_log, const float* dt_bias, int64_t T, int32_t num_k_heads, int32_t num_v_heads,
     int32_t dk, int32_t dv, const int32_t* seg_offsets, int32_t num_segments, const float* initial_state,
-    float* M, float* U, float* incoming, float* outgoing, float* final_state, uint32_t flags,
-    float gate_lower_bound, void* workspace, size_t workspace_bytes, int32_t* device_status,
-    void* stream) {
+    float* M, float* U, float* incoming, float* outgoing, float* final_state, const void* q, void* readout_m,
+    void* readout_u, uint32_t flags, float gate_lower_bound, void* workspace, size_t workspace_bytes,
+    int32_t* device_status, void* stream) {
   (void)workspace;
   (void)workspace_bytes;
   if (num_segments < 1 || num_v_heads <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+  const bool readouts = q || readout_m || readout_u;
+  if (readouts && (!q || !readout_m || !readout_u)) return KDA_ERR_INVALID_ARG;
+  if (readouts && (flags & KDA_SEG_SCAN_ONLY)) return KDA_ERR_INVALID_ARG;
   if ((flags & ~kKnownFlags) != 0) return KDA_ERR_INVALID_ARG;
   if (!initial_state || !M || !U || !incoming || !outgoing || !final_state) return KDA_ERR_INVALID_ARG;
   if (dk > 128 || dv > 128) return KDA_ERR_UNSUPPORTED;
@@ -136,12 +140,14 @@ extern "C" kda_status_t kda_segment_summarize_and_scan(
     if (!dtype_ok(kv_dtype)) return KDA_ERR_UNSUPPORTED;
     const bool use_fused = kv_dtype == KDA_BF16 && !(flags & KDA_FORCE_SIMT) && dk == 128 && dv == 128 &&
                            kda::fused_available();
+    if (readouts && !use_fused) return KDA_ERR_UNSUPPORTED;
+    if (readouts && (!aligned16(q) || !aligned16(readout_m) || !aligned16(readout_u))) return KDA_ERR_INVALID_ARG;
     if (use_fused) {
       if (!aligned16(k) || !aligned16(v) || !aligned16(raw_gate) || !aligned16(dt_bias) || !aligned16(M) ||
           !aligned16(U))
         return KDA_ERR_INVALID_ARG;
       kda::FusedArgs f{};
-      f.q = nullptr;
+      f.q = q;
       f.k = k;
       f.v = v;
       f.raw_gate = raw_gate;
@@ -155,8 +161,9 @@ extern "C" kda_status_t kda_segment_summarize_and_scan(
       f.Hv = num_v_heads;
       f.max_slots = num_segments;
       f.slots = nullptr;
-      f.out = nullptr;
-      f.out_bf16 = 0;
+      f.out = readout_m;
+      f.out2 = readout_u;
+      f.out_bf16 = 1;
       f.flags = flags;
       f.lb = gate_lower_bound;
       f.status = device_status;
@@ -222,6 +229,66 @@ extern "C" kda_status_t kda_segment_summarize_and_scan(
   sa.outgoing = outgoing;
   sa.final_state = final_state;
   return kda::launch_affine_scan(sa, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" size_t kda_context_parallel_workspace_size(int64_t T, int32_t num_v_heads, int32_t dv) {
+  if (T < 0 || num_v_heads <= 0 || dv <= 0) return 0;
+  return (size_t)2 * (size_t)T * (size_t)num_v_heads * (size_t)dv * 2;
+}
+
+extern "C" kda_status_t kda_context_parallel_apply(const void* readout_m, const void* readout_u,
+                                                   const float* incoming, const int32_t* seg_offsets,
+                                                   int32_t num_segments, int64_t T, int32_t num_v_heads, int32_t dv,
+                                                   void* out, kda_dtype_t out_dtype, uint32_t flags,
+                                                   int32_t* device_status, void* stream) {
+  if (num_segments < 1 || T < 0 || num_v_heads <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+  if ((flags & ~kKnownFlags) != 0) return KDA_ERR_INVALID_ARG;
+  if (!readout_m || !readout_u || !incoming || !seg_offsets || !out) return KDA_ERR_INVALID_ARG;
+  if (!dtype_ok(out_dtype)) return KDA_ERR_UNSUPPORTED;
+  if (dv != 128) return KDA_ERR_UNSUPPORTED;
+  if (!aligned16(readout_m) || !aligned16(readout_u) || !aligned16(out)) return KDA_ERR_INVALID_ARG;
+  kda::ApplyArgs ap{};
+  ap.seg_offsets = seg_offsets;
+  ap.num_segments = num_segments;
+  ap.total_tokens = T;
+  ap.Hv = num_v_heads;
+  ap.incoming = incoming;
+  ap.v_first = (flags & KDA_STATE_V_FIRST) ? 1 : 0;
+  ap.o_m = readout_m;
+  ap.o_u = readout_u;
+  ap.out = out;
+  ap.out_bf16 = out_dtype == KDA_BF16;
+  ap.status = device_status;
+  return kda::launch_cp_apply(ap, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" kda_status_t kda_context_parallel_prefill(
+    const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype, const float* raw_gate,
+    const float* beta_logits, const float* a_log, const float* dt_bias, int64_t T, int32_t num_k_heads,
+    int32_t num_v_heads, int32_t dk, int32_t dv, const int32_t* seg_offsets, int32_t num_segments,
+    const float* initial_state, void* out, kda_dtype_t out_dtype, float* final_state, float* M, float* U,
+    float* incoming, float* outgoing, uint32_t flags, float gate_lower_bound, void* workspace,
+    size_t workspace_bytes, int32_t* device_status, void* stream) {
+  if (num_segments < 1 || T < 0 || num_k_heads <= 0 || num_v_heads <= 0 || dk <= 0 || dv <= 0)
+    return KDA_ERR_INVALID_ARG;
+  if ((flags & ~kKnownFlags) != 0 || (flags & (KDA_SEG_SCAN_ONLY | KDA_FORCE_SIMT))) return KDA_ERR_INVALID_ARG;
+  if (!q || !out) return KDA_ERR_INVALID_ARG;
+  if (!dtype_ok(qkv_dtype) || !dtype_ok(out_dtype)) return KDA_ERR_UNSUPPORTED;
+  if (qkv_dtype != KDA_BF16 || dk != 128 || dv != 128 || !kda::fused_available()) return KDA_ERR_UNSUPPORTED;
+  const size_t need = kda_context_parallel_workspace_size(T, num_v_heads, dv);
+  if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+    return KDA_ERR_WORKSPACE;
+  __nv_bfloat16_raw* o_m = reinterpret_cast<__nv_bfloat16_raw*>(workspace);
+  __nv_bfloat16_raw* o_u = o_m + (size_t)T * num_v_heads * dv;
+  // every segment in parallel (M_i, U_i and both readouts), then the exclusive scan
+  kda_status_t st = kda_segment_summarize_and_scan(k, v, qkv_dtype, raw_gate, beta_logits, a_log, dt_bias, T,
+                                                   num_k_heads, num_v_heads, dk, dv, seg_offsets, num_segments,
+                                                   initial_state, M, U, incoming, outgoing, final_state, q, o_m,
+                                                   o_u, flags, gate_lower_bound, nullptr, 0, device_status, stream);
+  if (st != KDA_OK) return st;
+  // the incoming state's share added to the readouts
+  return kda_context_parallel_apply(o_m, o_u, incoming, seg_offsets, num_segments, T, num_v_heads, dv, out,
+                                    out_dtype, flags & KDA_STATE_V_FIRST, device_status, stream);
 }
 
 extern "C" size_t kda_workspace_size(int64_t total_tokens, int32_t batch, int32_t num_k_heads,

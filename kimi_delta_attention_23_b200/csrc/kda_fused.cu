@@ -120,7 +120,9 @@ struct InputMaps {
 // kBuild = false: prefill (state from the pool, readout, state back to the pool).
 // kBuild = true: segment build -- two states share every k-side product: the transition M
 // (started at I, zero values) and the contribution U (started at 0, real values); no readout.
-template <bool kBuild>
+// kRead: the query side is present (scores P, Q o Gamma) and readouts are produced -- always
+// in prefill; in the build, the readouts of both states (local outputs of the segment).
+template <bool kBuild, bool kRead>
 __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArgs a, const __grid_constant__ InputMaps tm) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -170,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   const uint32_t tmD1u = tmem + 64, tmSu = tmem + 256, tmSbu = tmem + 448;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   const int ej = (warp & 3) * 32 + lane, ehalf = warp >> 2;  // epilogue row and column half
-  const bool qb = !kBuild && a.q != nullptr;
+  constexpr bool qb = kRead;
   // one thread copies the inputs of the chunk starting at token c0n into the prefetch region
   // with four tensor copies (rows past the end of the tensor arrive as zeros; rows past the
   // end of the sequence are never read); completion is counted in bytes on bar_pf
@@ -305,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       sBeta[row] = row < L ? beta_f32(beta_raw, prob) : 0.f;
     }
     // P's upper triangle must read as zero (A's upper triangle is never read)
-    if constexpr (!kBuild)
+    if constexpr (kRead)
       for (int e = tid; e < 8192 / 16; e += kThreads) reinterpret_cast<uint4*>(sm + OFF_P)[e] = make_uint4(0, 0, 0, 0);
     // in-block products: p8 inclusive prefix from the block start, s8 exclusive suffix
     float p8[8][4], s8[8][4];
@@ -395,12 +397,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       }
       *reinterpret_cast<uint2*>(sm + OFF_KQ + sw_off(row, ch, 128)) =
           pack4(kf[0] * g[0], kf[1] * g[1], kf[2] * g[2], kf[3] * g[3]);
-      if constexpr (!kBuild)
+      if constexpr (kRead)
         *reinterpret_cast<uint2*>(sm + OFF_KQ + sw_off(64 + row, ch, 128)) =
             pack4(qf[0] * g[0], qf[1] * g[1], qf[2] * g[2], qf[3] * g[3]);
       *reinterpret_cast<uint2*>(sm + OFF_KPI + sw_off(row, ch, 64)) =
           pack4(kf[0] * pi[0], kf[1] * pi[1], kf[2] * pi[2], kf[3] * pi[3]);
-      if constexpr (!kBuild)
+      if constexpr (kRead)
         *reinterpret_cast<uint2*>(sm + OFF_QPI + sw_off(row, ch, 64)) =
             pack4(qf[0] * pi[0], qf[1] * pi[1], qf[2] * pi[2], qf[3] * pi[3]);
       *reinterpret_cast<uint2*>(sm + OFF_KC + sw_off(row, ch, 64)) =
@@ -409,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       if (upper) {
         *reinterpret_cast<uint2*>(sm + OFF_KPI8 + sw_off(r32, ch, 32)) =
             pack4(kf[0] * p8[r][0], kf[1] * p8[r][1], kf[2] * p8[r][2], kf[3] * p8[r][3]);
-        if constexpr (!kBuild)
+        if constexpr (kRead)
           *reinterpret_cast<uint2*>(sm + OFF_QPI8 + sw_off(r32, ch, 32)) =
               pack4(qf[0] * p8[r][0], qf[1] * p8[r][1], qf[2] * p8[r][2], qf[3] * p8[r][3]);
       } else {
@@ -442,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     //   A_rs (r > s, slots 0..27) and P_rs (r >= s, slots 28..63), then a butterfly
     //   reduce-scatter over the 32 lanes leaves slots 2*lane and 2*lane+1 in this lane
     //   (build: A only, 32 slots, slot lane in this lane)
-    if constexpr (kBuild) {
+    if constexpr (!kRead) {
       float acc[32];
       float kf[8][4];
 #pragma unroll
@@ -545,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           uint32_t ak0, ak1, ak2, ak3, aq0, aq1, aq2, aq3, b00, b01, b10, b11;
           const int ar = 16 * pa + (m & 1) * 8 + (lane & 7), akc = 2 * kk + (m >> 1);
           ldsm_x4(sbase + OFF_KPI + sw_off(ar, akc * 8, 64), ak0, ak1, ak2, ak3);
-          if constexpr (!kBuild) ldsm_x4(sbase + OFF_QPI + sw_off(ar, akc * 8, 64), aq0, aq1, aq2, aq3);
+          if constexpr (kRead) ldsm_x4(sbase + OFF_QPI + sw_off(ar, akc * 8, 64), aq0, aq1, aq2, aq3);
           const int br = 16 * pb + (m >> 1) * 8 + (lane & 7), bkc = 2 * kk + (m & 1);
           ldsm_x4(sbase + OFF_KC + sw_off(br, bkc * 8, 64), b00, b01, b10, b11);
           if (pa - pb > 1) {  // adjacent 16-blocks have nothing between them
@@ -558,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           }
           mma16816(accA[0], ak0, ak1, ak2, ak3, b00, b01);
           mma16816(accA[1], ak0, ak1, ak2, ak3, b10, b11);
-          if constexpr (!kBuild) {
+          if constexpr (kRead) {
             mma16816(accP[0], aq0, aq1, aq2, aq3, b00, b01);
             mma16816(accP[1], aq0, aq1, aq2, aq3, b10, b11);
           }
@@ -570,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
             const int r = 16 * pa + g + 8 * hlf, s = 16 * pb + 8 * nt + 2 * t;
             sA[r * kLdA + s] = accA[nt][2 * hlf];
             sA[r * kLdA + s + 1] = accA[nt][2 * hlf + 1];
-            if constexpr (!kBuild)
+            if constexpr (kRead)
               *reinterpret_cast<uint32_t*>(sm + OFF_P + sw_off(r, s, 64)) =
                   pack_bf16(accP[nt][2 * hlf], accP[nt][2 * hlf + 1]);
           }
@@ -586,16 +588,16 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
             uint32_t ak0, ak1, ak2, ak3, aq0, aq1, aq2, aq3, b0, b1;
             const int ar = 8 * bb + (lane & 7), akc = 2 * kk + (m >> 1);
             ldsm_x4(sbase + OFF_KPI8 + sw_off(ar, akc * 8, 32), ak0, ak1, ak2, ak3);
-            if constexpr (!kBuild) ldsm_x4(sbase + OFF_QPI8 + sw_off(ar, akc * 8, 32), aq0, aq1, aq2, aq3);
+            if constexpr (kRead) ldsm_x4(sbase + OFF_QPI8 + sw_off(ar, akc * 8, 32), aq0, aq1, aq2, aq3);
             const int br = 8 * bb + (lane & 7), bkc = 2 * kk + ((lane >> 3) & 1);
             ldsm_x2(sbase + OFF_KK8 + sw_off(br, bkc * 8, 32), b0, b1);
             mma16816(accA, ak0, ak1, ak2, ak3, b0, b1);
-            if constexpr (!kBuild) mma16816(accP, aq0, aq1, aq2, aq3, b0, b1);
+            if constexpr (kRead) mma16816(accP, aq0, aq1, aq2, aq3, b0, b1);
           }
           const int r = 16 * bb + 8 + g, s = 16 * bb + 2 * t;
           sA[r * kLdA + s] = accA[2];
           sA[r * kLdA + s + 1] = accA[3];
-          if constexpr (!kBuild)
+          if constexpr (kRead)
             *reinterpret_cast<uint32_t*>(sm + OFF_P + sw_off(r, s, 64)) = pack_bf16(accP[2], accP[3]);
         }
       }
@@ -1013,9 +1015,26 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       // the V tile is free now that the second products completed
       if (c0 + C < t1 && tid == kPfThread) issue_prefetch_v(c0 + C);
 
-      // S_M^T += Delta_M^T K' ;  S_U^T += Delta_U^T K'
+      // [readouts: D_st = S_st,0^T (Q o Gamma)^T + Delta_st^T P^T -- the bf16 copies still hold the
+      //  chunk's incoming states]   S_M^T += Delta_M^T K' ;  S_U^T += Delta_U^T K'
       if (tid == kMmaThread) {
         tc_fence_after();
+        if constexpr (kRead) {
+#pragma unroll 1
+          for (int st = 0; st < 2; ++st) {
+            const uint32_t dcol = st ? tmD1u : tmD1, acol = st ? tmSbu : tmSb;
+            const uint32_t xoff = st ? OFF_X : OFF_XM;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32 + 8192;  // rows 64..127: Q o Gamma
+              mma_bf16_ts(dcol, acol + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(dcol, desc_sw128(sbase + xoff + kk * 32), desc_sw128(sbase + OFF_P + kk * 32),
+                       idesc_bf16_f32(64), 1);
+          }
+        }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmS, desc_sw128(sbase + OFF_XM + kk * 32), desc_sw128(sbase + OFF_KPT + kk * 32),
@@ -1031,6 +1050,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         report(a.status, KDA_ERR_DEVICE_TIMEOUT);
       } else {
         tc_fence_after();
+        if constexpr (kRead) {
+          // readouts of both states, staged row-major bf16 in their (now free) X tiles
+#pragma unroll 1
+          for (int st = 0; st < 2; ++st) {
+            float d[32];
+            tmem_ld16n<2>((st ? tmD1u : tmD1) + lane_base + 32 * ehalf, d);
+            tmem_wait_ld();
+            uint8_t* stage = sm + (st ? OFF_X : OFF_XM);
+#pragma unroll
+            for (int u = 0; u < 32; ++u)
+              *reinterpret_cast<__nv_bfloat16*>(stage + ((32 * ehalf + u) * D + ej) * 2) = __float2bfloat16_rn(d[u]);
+          }
+        }
         // bf16 copies of both new states for the next chunk's first products
 #pragma unroll 1
         for (int st = 0; st < 2; ++st) {
@@ -1054,6 +1086,15 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       if (*s_abort) {
         aborted = true;
         break;
+      }
+      if constexpr (kRead) {
+        for (int e = tid; e < 2 * C * 16; e += kThreads) {
+          const int st = e >> 10, row = (e >> 4) & 63, cc = e & 15;
+          if (row < L)
+            *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(st ? a.out2 : a.out) +
+                                      ((size_t)(c0 + row) * a.Hv + h) * D + cc * 8) =
+                *reinterpret_cast<const uint4*>(sm + (st ? OFF_X : OFF_XM) + row * 256 + cc * 16);
+        }
       }
     }
     }
@@ -1131,10 +1172,14 @@ bool encode_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint3
 }  // namespace
 
 cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream) {
-  cudaError_t err = cudaFuncSetAttribute(fused_chunk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemAlloc);
+  cudaError_t err = cudaFuncSetAttribute(fused_chunk_kernel<false, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   if (err == cudaSuccess)
-    err = cudaFuncSetAttribute(fused_chunk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    err = cudaFuncSetAttribute(fused_chunk_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kSmemAlloc);
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(fused_chunk_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kSmemAlloc);
   if (err != cudaSuccess) return err;
   if (a.batch == 0) return cudaSuccess;
   InputMaps tm;
@@ -1148,10 +1193,12 @@ cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream) {
                               CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
   dim3 grid(a.Hv, a.batch);
-  if (a.build)
-    fused_chunk_kernel<true><<<grid, kThreads, kSmemAlloc, stream>>>(a, tm);
+  if (a.build && a.out)
+    fused_chunk_kernel<true, true><<<grid, kThreads, kSmemAlloc, stream>>>(a, tm);
+  else if (a.build)
+    fused_chunk_kernel<true, false><<<grid, kThreads, kSmemAlloc, stream>>>(a, tm);
   else
-    fused_chunk_kernel<false><<<grid, kThreads, kSmemAlloc, stream>>>(a, tm);
+    fused_chunk_kernel<false, true><<<grid, kThreads, kSmemAlloc, stream>>>(a, tm);
   return cudaGetLastError();
 }
 

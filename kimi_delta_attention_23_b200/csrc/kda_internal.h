@@ -71,14 +71,31 @@ struct FusedArgs {
   int32_t v_first;          // state blocks stored transposed ([dv][dk])
   int32_t init_mode;        // 0: state_in slot, 1: zero, 2: identity
   int32_t values_zero;      // 1: all values are zero (transition build)
-  void* out;                // [T,Hv,128] or NULL (no readout)
+  void* out;                // [T,Hv,128] or NULL (no readout); with build: readout of the transition
+  void* out2;               // build only: readout of the contribution [T,Hv,128] bf16 (or NULL)
   int32_t out_bf16;
   uint32_t flags;
   float lb;
   int32_t* status;
 };
 
+// Context-parallel prefill, last step: out = O_M . S_in(segment) + O_U.
+struct ApplyArgs {
+  const int32_t* seg_offsets;  // [N+1]
+  int32_t num_segments;
+  int64_t total_tokens;
+  int32_t Hv;
+  const float* incoming;       // [N][Hv][128][128] in the state layout
+  int32_t v_first;
+  const void* o_m;             // bf16 [T][Hv][128] readout through the transition
+  const void* o_u;             // bf16 [T][Hv][128] readout of the contribution
+  void* out;                   // [T][Hv][128]
+  int32_t out_bf16;
+  int32_t* status;
+};
+
 size_t simt_smem_bytes(int dk, int w);
+cudaError_t launch_cp_apply(const ApplyArgs& a, cudaStream_t stream);
 cudaError_t launch_simt_chunk(const SimtArgs& a, cudaStream_t stream);
 cudaError_t launch_affine_scan(const ScanArgs& a, cudaStream_t stream);
 

@@ -78,20 +78,23 @@ def test_empty_batch_is_a_no_op(lib):
 
 def _seg(lib, **over):
     args = dict(k=1, v=1, kv=1, raw=1, beta=1, a_log=1, dt_bias=1, T=64, Hk=2, Hv=2, dk=128, dv=128, offs=1,
-                N=4, init=1, M=1, U=1, inc=1, outg=1, fin=1, flags=0)
+                N=4, init=1, M=1, U=1, inc=1, outg=1, fin=1, q=0, rm=0, ru=0, flags=0)
     args.update(over)
     p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
     return lib.kda_segment_summarize_and_scan(
         p(args["k"]), p(args["v"]), args["kv"], p(args["raw"]), p(args["beta"]), p(args["a_log"]),
         p(args["dt_bias"]), args["T"], args["Hk"], args["Hv"], args["dk"], args["dv"], p(args["offs"]),
         args["N"], p(args["init"]), p(args["M"]), p(args["U"]), p(args["inc"]), p(args["outg"]),
-        p(args["fin"]), args["flags"], -5.0, None, 0, None, None)
+        p(args["fin"]), p(args["q"]), p(args["rm"]), p(args["ru"]), args["flags"], -5.0, None, 0, None, None)
 
 
 @pytest.mark.parametrize("over,code", [
     (dict(N=0), 1), (dict(Hv=0), 1), (dict(init=0), 1), (dict(M=0), 1), (dict(U=0), 1), (dict(inc=0), 1),
     (dict(outg=0), 1), (dict(fin=0), 1), (dict(flags=1 << 20), 1), (dict(offs=0), 1), (dict(k=0), 1),
     (dict(Hk=3), 1), (dict(dk=129), 2), (dict(kv=5), 2),
+    (dict(q=16), 1), (dict(q=16, rm=16), 1),                        # readouts need q and both outputs
+    (dict(q=16, rm=16, ru=16, flags=kda.SEG_SCAN_ONLY), 1),
+    (dict(q=16, rm=16, ru=16, kv=0), 2),                            # readouts only on the bf16 fast path
 ])
 def test_segment_host_checks(lib, over, code):
     assert _seg(lib, **over) == code
@@ -104,3 +107,18 @@ def test_binding_refuses_cpu_tensors():
         kda.kda_chunk_fwd(w, w, w, torch.zeros(4, 1, 16), torch.zeros(4, 1), torch.zeros(1), torch.zeros(1, 16),
                           torch.zeros(2, dtype=torch.int32), torch.zeros(1, 1, 16, 16),
                           torch.zeros(1, dtype=torch.int32))
+
+
+def test_context_parallel_host_checks(lib):
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
+    # apply: null pointers, dv != 128
+    assert lib.kda_context_parallel_apply(None, p(16), p(16), p(16), 2, 64, 2, 128, p(16), 1, 0, None, None) == 1
+    assert lib.kda_context_parallel_apply(p(16), p(16), p(16), p(16), 2, 64, 2, 64, p(16), 1, 0, None, None) == 2
+    assert lib.kda_context_parallel_apply(p(16), p(16), p(16), p(16), 0, 64, 2, 128, p(16), 1, 0, None, None) == 1
+    # prefill: workspace too small, fp32 inputs unsupported
+    args = [p(16)] * 3 + [1] + [p(16)] * 4 + [64, 2, 2, 128, 128, p(16), 2, p(16), p(16), 1] + [p(16)] * 5 + [0, -5.0]
+    assert lib.kda_context_parallel_prefill(*args, p(256), 16, None, None) == 3
+    args_f32 = list(args)
+    args_f32[3] = 0
+    assert lib.kda_context_parallel_prefill(*args_f32, p(256), 1 << 30, None, None) == 2
+    assert kda.kda_context_parallel_workspace_size(100, 4, 128) == 2 * 100 * 4 * 128 * 2

@@ -128,3 +128,41 @@ def test_full_size_context_parallel_sampled_heads():
                                       cpu(w.state_indices))
     assert rel_l2(out[:, heads], o_ref) < 1e-2
     assert rel_l2(res["final_state"][heads], p_ref[0]) < 1e-2
+
+
+@pytest.mark.parametrize("layout,out_dtype", [("K_FIRST", torch.bfloat16), ("V_FIRST", torch.float32)])
+def test_context_parallel_prefill_entry_point(layout, out_dtype):
+    w = W.random_inputs([1000], 2, 2, 128, 128, seed=4, state_std=0.1, state_layout=layout)
+    wd = w.to("cuda")
+    offs = torch.tensor([0, 64, 300, 301, 777, 1000], dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    res = kda.kda_context_parallel_prefill(wd.q, wd.k, wd.v, wd.raw_gate, wd.beta_logits, wd.a_log, wd.dt_bias,
+                                           offs, wd.state_pool[0].contiguous(), output_dtype=out_dtype,
+                                           state_layout=layout, device_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    o_ref, p_ref = oracle.kda_forward(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens,
+                                      w.state_pool, w.state_indices, state_layout=layout)
+    assert res["out"].dtype == out_dtype
+    assert rel_l2(res["out"], o_ref) < 1e-2
+    assert rel_l2(res["final_state"], p_ref[0]) < 1e-2
+    M, U = oracle.kda_segment_summary(w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, offs.cpu(),
+                                      state_layout=layout)
+    assert rel_l2(res["transition_matrices"], M) < 1e-2
+    assert rel_l2(res["local_contributions"], U) < 1e-2
+
+
+def test_full_size_context_parallel_prefill_sampled_heads():
+    """The benchmark's step: 131072 tokens, 32 heads, 16 segments, one entry point."""
+    w = W.make("long_T131072_H32_cp16", device="cuda")
+    res = kda.kda_context_parallel_prefill(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias,
+                                           w.seg_offsets, w.state_pool[0])
+    torch.cuda.synchronize()
+    heads = [9, 30]
+    cpu = lambda t: t.detach().cpu()  # noqa: E731
+    o_ref, p_ref = oracle.kda_forward(cpu(w.q)[:, heads], cpu(w.k)[:, heads], cpu(w.v)[:, heads],
+                                      cpu(w.raw_gate)[:, heads], cpu(w.beta_logits)[:, heads], cpu(w.a_log)[heads],
+                                      cpu(w.dt_bias)[heads], cpu(w.cu_seqlens), cpu(w.state_pool)[:, heads],
+                                      cpu(w.state_indices))
+    assert rel_l2(res["out"][:, heads], o_ref) < 1e-2
+    assert rel_l2(res["final_state"][heads], p_ref[0]) < 1e-2
