@@ -200,6 +200,32 @@ KDA_API kda_status_t kda_context_parallel_prefill(
     float gate_lower_bound, void *workspace, size_t workspace_bytes, int32_t *device_status,
     void *stream);
 
+/*
+ * kda_context_parallel_prefill_static -- kda_context_parallel_prefill for callers that cannot
+ * allocate device memory where they run it (a host whose device memory belongs to another
+ * component's pool, or a serving loop that must not allocate while requests are in flight,
+ * since allocation can synchronise the device).  Same arguments and results, without the
+ * workspace: the scratch is a fixed 32 MiB array in device memory carried by the library, which
+ * every GPU that loads libkda.so holds until the process exits.  No counterpart on the pages:
+ * this is an interface convenience, not part of the method.
+ *
+ * Limit: kda_context_parallel_workspace_size(T, num_v_heads, dv) <= 32 MiB, i.e. at most
+ * 65536 token-heads per call with dv = 128 (for example 2048 tokens x 32 heads); larger calls
+ * return KDA_ERR_WORKSPACE and do nothing.  The call allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.  The first call on a device looks up the array's
+ * device address (once per device, with that device current); make that first call before any
+ * stream capture.  Every call shares the one array and leaves its last contents there (nothing
+ * in it needs to start at zero); calls whose work overlaps on the GPU (other streams, or other
+ * host threads) race on it and must be serialised by the caller.
+ */
+KDA_API kda_status_t kda_context_parallel_prefill_static(
+    const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype, const float *raw_gate,
+    const float *beta_logits, const float *a_log, const float *dt_bias, int64_t T,
+    int32_t num_k_heads, int32_t num_v_heads, int32_t dk, int32_t dv, const int32_t *seg_offsets,
+    int32_t num_segments, const float *initial_state, void *out, kda_dtype_t out_dtype,
+    float *final_state, float *M, float *U, float *incoming, float *outgoing, uint32_t flags,
+    float gate_lower_bound, int32_t *device_status, void *stream);
+
 /* Workspace bytes kda_context_parallel_prefill needs: the two bf16 readouts, 2 * T * Hv * dv * 2. */
 KDA_API size_t kda_context_parallel_workspace_size(int64_t T, int32_t num_v_heads, int32_t dv);
 
