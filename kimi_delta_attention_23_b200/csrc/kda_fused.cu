@@ -50,8 +50,8 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far beyond any legitim
 
 // shared-memory map (bytes from a 1024-aligned base); bf16 operand tiles use the K-major
 // 128-byte swizzle layout (see sw_off)
-constexpr int OFF_S = 0;                    // free in prefill (the bf16 state lives in TMEM)
-constexpr int OFF_KQ = OFF_S + 32768;       // [K o Gamma ; Q o Gamma]   128 rows x 128 K
+constexpr int OFF_S = 0;                    // prefill: bf16 output staging (the bf16 state lives in TMEM)
+constexpr int OFF_KQ = OFF_S + 32768;       // [K o Gamma ; Q o Gamma]   128 rows x 128 K (then output staging)
 constexpr int OFF_KPT = OFF_KQ + 32768;     // K'^T       128 rows x 64 K
 constexpr int OFF_X = OFF_KPT + 16384;      // X^T, then Delta^T   128 rows x 64 K
 constexpr int OFF_V = OFF_X + 16384;        // V as the MN-major A operand V^T (two 64-column halves, 8 KB
@@ -69,7 +69,7 @@ constexpr int OFF_TAU = OFF_A + 17408;      // fp32 [8][128] decay product of ea
 constexpr int OFF_MP = OFF_TAU + 4096;      // fp32 [6][128] decay between 16-blocks of a pair
 constexpr int OFF_BETA = OFF_MP + 3072;     // fp32 [64]
 constexpr int OFF_GC = OFF_BETA + 256;      // fp32 [128] Gamma of the last row
-constexpr int OFF_BAR = OFF_GC + 512;       // 4 mbarriers, TMEM base, abort flag
+constexpr int OFF_BAR = OFF_GC + 512;       // mbarriers (+0..+39, +48, +56), TMEM base (+40), abort flag (+44)
 constexpr int kSmemBytes = OFF_BAR + 64;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for aligning the base to 1024
 constexpr int OFF_XM = OFF_S;               // build: X^T / Delta^T of the transition state
@@ -115,6 +115,7 @@ __constant__ unsigned char kDiagPair[64] = {
 // 64 tokens x 1 head x 128 channels: one copy per tensor moves a whole chunk of one head.
 struct InputMaps {
   CUtensorMap raw, k, q, v;
+  CUtensorMap out, out2;  // bf16 outputs (readouts in the build), written by tensor stores
 };
 
 // kBuild = false: prefill (state from the pool, readout, state back to the pool).
@@ -140,6 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
 
   const uint32_t sbase = smem_addr(sm);
   const uint32_t bar0 = sbase + OFF_BAR, bar1 = bar0 + 8, bar2 = bar0 + 16, bar3 = bar0 + 24, bar_pf = bar0 + 32;
+  const uint32_t bar4 = bar0 + 48, bar_v = bar0 + 56;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 40);
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + OFF_BAR + 44);
   float* sA = reinterpret_cast<float*>(sm + OFF_A);
@@ -154,6 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     mbar_init(bar2, 1);
     mbar_init(bar3, 1);
     mbar_init(bar_pf, 1);
+    mbar_init(bar4, 1);
+    mbar_init(bar_v, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -173,33 +177,35 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   const int ej = (warp & 3) * 32 + lane, ehalf = warp >> 2;  // epilogue row and column half
   constexpr bool qb = kRead;
-  // one thread copies the inputs of the chunk starting at token c0n into the prefetch region
-  // with four tensor copies (rows past the end of the tensor arrive as zeros; rows past the
-  // end of the sequence are never read); completion is counted in bytes on bar_pf
+  // one thread copies the inputs of the chunk starting at token c0n with tensor copies (rows
+  // past the end of the tensor arrive as zeros; rows past the end of the sequence are never
+  // read); completion is counted in bytes, on bar_pf for the gate, k and q and on bar_v for V
   const bool has_v = kBuild || !a.values_zero;
-  const uint32_t pf_bytes = 32768u + 16384u * (1u + (qb ? 1u : 0u) + (has_v ? 1u : 0u));
-  // gate, k and q land in the score scratch (free once the chunk's operands are built); V
-  // lands in its operand tile (free once the chunk's second product completed)
+  const uint32_t gkq_bytes = 32768u + 16384u * (1u + (qb ? 1u : 0u));
+  // gate, k and q land in the score scratch (free once the chunk's inverse is done); V lands
+  // in its operand tile (free once the chunk's second product completed)
   auto issue_prefetch_gkq = [&](int64_t c0n) {
-    mbar_arrive_expect_tx(bar_pf, pf_bytes);
+    mbar_arrive_expect_tx(bar_pf, gkq_bytes);
     tma_load_3d(sbase + PF_RAW, &tm.raw, 0, h, (int)c0n, bar_pf);
     tma_load_3d(sbase + PF_K, &tm.k, 0, kh, (int)c0n, bar_pf);
     if (qb) tma_load_3d(sbase + PF_Q, &tm.q, 0, kh, (int)c0n, bar_pf);
   };
   auto issue_prefetch_v = [&](int64_t c0n) {
     if (has_v) {
-      tma_load_3d(sbase + OFF_V, &tm.v, 0, h, (int)c0n, bar_pf);
-      tma_load_3d(sbase + OFF_V + 8192, &tm.v, 64, h, (int)c0n, bar_pf);
+      mbar_arrive_expect_tx(bar_v, 16384u);
+      tma_load_3d(sbase + OFF_V, &tm.v, 0, h, (int)c0n, bar_v);
+      tma_load_3d(sbase + OFF_V + 8192, &tm.v, 64, h, (int)c0n, bar_v);
     }
   };
-  bool pf_pending = false;  // a prefetch was issued and its completion not yet observed
-  uint32_t pf_parity = 0;   // parity of the next prefetch completion on bar_pf
+  bool pf_pending = false, v_pending = false;  // copies issued whose completion was not yet observed
+  uint32_t pf_parity = 0, v_parity = 0;        // parities of the next completions on bar_pf, bar_v
   if (t1 > t0) {
     if (tid == kPfThread) {
       issue_prefetch_gkq(t0);
       issue_prefetch_v(t0);
     }
     pf_pending = true;
+    v_pending = has_v;
   }
   const size_t blk_off = ((size_t)slot * a.Hv + h) * (size_t)(D * D);
   const float* in_blk = a.state_in ? a.state_in + blk_off : nullptr;
@@ -262,14 +268,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     const int64_t t = c0n + warp * 8 + lane;
     if (lane < 8 && t < t1) beta_raw = __ldg(a.beta + (size_t)t * a.Hv + h);
   };
-  load_beta(t0);
-  uint32_t phase = 0;
-  bool aborted = false;
-#pragma unroll 1
-  for (int64_t c0 = t0; c0 < t1; c0 += C, phase ^= 1u) {
-    const int L = (int)((t1 - c0) < C ? (t1 - c0) : C);
-
-    // =============================== k-side, part 1: gates and in-block products
+  // gates of the chunk whose inputs are in the prefetch region (Ln valid rows): the decay alpha
+  // replaces the raw gate in place (1 past the sequence end) and beta goes to sBeta.  It runs
+  // for the next chunk while the last products of the current one are on the tensor cores.
+  auto gate_phase = [&](int Ln) {
     if (mbar_wait_bounded(bar_pf, pf_parity, kWaitLimitNs)) {
       pf_pending = false;
       pf_parity ^= 1u;
@@ -277,34 +279,58 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       *s_abort = 1;
       report(a.status, KDA_ERR_DEVICE_TIMEOUT);
     }
-    float al[8][4];
-    uint2 k2[8], q2[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int row = warp * 8 + r;
-      if (row < L) {
-        const float4 raw = *reinterpret_cast<const float4*>(sm + PF_RAW + row * 512 + ch * 4);
-        k2[r] = *reinterpret_cast<const uint2*>(sm + PF_K + row * 256 + ch * 2);
-        q2[r] = qb ? *reinterpret_cast<const uint2*>(sm + PF_Q + row * 256 + ch * 2) : make_uint2(0u, 0u);
+      float4* cell = reinterpret_cast<float4*>(sm + PF_RAW + row * 512 + ch * 4);
+      float o[4] = {1.f, 1.f, 1.f, 1.f};
+      if (row < Ln) {
+        const float4 raw = *cell;
         const float xs[4] = {raw.x + dtb.x, raw.y + dtb.y, raw.z + dtb.z, raw.w + dtb.w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const float x = xs[c];
           // softplus(x) in log2 units, then alpha = exp(-exp(a_log) softplus(x)) = 2^(-c sp2)
           const float sp2 = fmaxf(x, 0.f) * kLog2e + fast_lg2(1.f + fast_ex2(-fabsf(x) * kLog2e));
-          float al_c = fast_ex2(-cexp * sp2);
-          al[r][c] = safe ? fmaxf(al_c, alpha_floor) : al_c;
+          const float al_c = fast_ex2(-cexp * sp2);
+          o[c] = safe ? fmaxf(al_c, alpha_floor) : al_c;
         }
-      } else {
-        k2[r] = make_uint2(0u, 0u);
-        q2[r] = make_uint2(0u, 0u);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) al[r][c] = 1.f;
       }
+      *cell = make_float4(o[0], o[1], o[2], o[3]);
     }
     if (lane < 8) {
       const int row = warp * 8 + lane;
-      sBeta[row] = row < L ? beta_f32(beta_raw, prob) : 0.f;
+      sBeta[row] = row < Ln ? beta_f32(beta_raw, prob) : 0.f;
+    }
+  };
+  auto rows_of = [&](int64_t c0n) { return (int)((t1 - c0n) < C ? (t1 - c0n) : C); };
+  load_beta(t0);
+  if (t1 > t0) gate_phase(rows_of(t0));
+  uint32_t phase = 0;
+  bool aborted = false;
+#pragma unroll 1
+  for (int64_t c0 = t0; c0 < t1; c0 += C, phase ^= 1u) {
+    const int L = rows_of(c0);
+
+    // =============================== k-side, part 1: in-block products (the gates were done
+    // while the previous chunk's last products ran)
+    float al[8][4];
+    uint2 k2[8], q2[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int row = warp * 8 + r;
+      const float4 a4 = *reinterpret_cast<const float4*>(sm + PF_RAW + row * 512 + ch * 4);
+      al[r][0] = a4.x;
+      al[r][1] = a4.y;
+      al[r][2] = a4.z;
+      al[r][3] = a4.w;
+      if (row < L) {
+        k2[r] = *reinterpret_cast<const uint2*>(sm + PF_K + row * 256 + ch * 2);
+        q2[r] = qb ? *reinterpret_cast<const uint2*>(sm + PF_Q + row * 256 + ch * 2) : make_uint2(0u, 0u);
+      } else {
+        k2[r] = make_uint2(0u, 0u);
+        q2[r] = make_uint2(0u, 0u);
+      }
     }
     // P's upper triangle must read as zero (A's upper triangle is never read)
     if constexpr (kRead)
@@ -327,6 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       }
     }
     *reinterpret_cast<float4*>(sTau + warp * D + ch) = make_float4(p8[7][0], p8[7][1], p8[7][2], p8[7][3]);
+    if (tid == kPfThread) bulk_wait_read_all();  // the previous chunk's staged outputs were read
     __syncthreads();  // (1) block products visible; prefetched inputs consumed; output flushed
     if (*s_abort) {
       aborted = true;
@@ -532,7 +559,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         }
       }
     }
+    fence_async_smem();  // the operand tiles are read by the tensor cores
     __syncthreads();  // (2) operand tiles, block factors and diagonal scores in place
+
 
     // =============================== k-side, part 2: off-diagonal scores on mma.sync
     {
@@ -639,7 +668,31 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       __syncthreads();
       const int g = lane >> 2, t = lane & 3;
       auto lval = [&](int r, int c) { return sBeta[r] * sA[r * kLdA + c]; };
-      if (warp < 4) {
+      if (warp >= 4) {
+        // warps 4..7 have no part in the first doubling level: one thread issues the first
+        // state-side product, which needs only [K o Gamma ; Q o Gamma] (complete since (2))
+        // and the chunk's incoming state(s); it runs while the inverse is finished
+        if (tid == kMmaThread) {
+          tc_fence_after();
+          if constexpr (!kBuild) {
+            // D1 = S^T [K o Gamma ; Q o Gamma]^T   (M = 128, N = 128, K = 128)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+              mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(128), kk > 0);
+            }
+          } else {
+            // D1_M = S_M^T (K o Gamma)^T and D1_U = S_U^T (K o Gamma)^T   (N = 64 each, K = 128)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+              mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
+              mma_bf16_ts(tmD1u, tmSbu + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
+            }
+          }
+          mma_commit(bar0);
+        }
+      } else {
         // level 1: warp -> (problem, 8-column tile); problem 0 = X10, problem 1 = X32
         const int ra = (warp >> 1) ? 3 : 1, cb = 16 * (ra - 1), R0 = 16 * ra, n0 = 8 * (warp & 1);
         float* yt = Yb + warp * 128;  // 16 x 8 tile of Y, row-major
@@ -731,17 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     }
 
     if constexpr (!kBuild) {
-    // =============================== state side
-    // D1 = S^T [K o Gamma ; Q o Gamma]^T   (M = 128, N = 128, K = 128)
-    if (tid == kMmaThread) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(128), kk > 0);
-      }
-      mma_commit(bar0);
-    }
+    // =============================== state side (the first product was issued in the inverse)
     {
       // epilogues run on all eight warps: warps w and w + 4 share TMEM lane quadrant w % 4
       // (state row j) and split the columns
@@ -772,6 +815,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     // D1[:, 0:64] = V^T T^T + Y^T T^T = (V - (K o Gamma) S0)^T T^T = Delta^T   (N = 64, K = 64)
     if (tid == kMmaThread) {
       tc_fence_after();
+      if (has_v && !mbar_wait_bounded(bar_v, v_parity, kWaitLimitNs)) {  // this chunk's V has landed
+        *s_abort = 1;
+        report(a.status, KDA_ERR_DEVICE_TIMEOUT);
+      }
       if (!a.values_zero) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -785,41 +832,40 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       mma_commit(bar1);
     }
     {
+      // decay the state columns while the second product runs (it reads neither state copy):
+      // S^T[j][i] *= Gamma_63[i]
+      {
+        const int i0 = 64 * ehalf;
+        float sv[64];
+        tmem_ld16n<4>(tmS + lane_base + i0, sv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 64; u += 4) {
+          const float4 gv = *reinterpret_cast<const float4*>(sGC + i0 + u);
+          sv[u] *= gv.x;
+          sv[u + 1] *= gv.y;
+          sv[u + 2] *= gv.z;
+          sv[u + 3] *= gv.w;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          tmem_st16(tmS + lane_base + i0 + 16 * q, *reinterpret_cast<const float(*)[16]>(sv + 16 * q));
+      }
       if (!mbar_wait_bounded(bar1, phase, kWaitLimitNs)) {
         *s_abort = 1;
         report(a.status, KDA_ERR_DEVICE_TIMEOUT);
       } else {
         tc_fence_after();
-        {
-          float d[32];
-          tmem_ld16n<2>(tmD1 + lane_base + 32 * ehalf, d);
-          tmem_wait_ld();
+        float d[32];
+        tmem_ld16n<2>(tmD1 + lane_base + 32 * ehalf, d);
+        tmem_wait_ld();
 #pragma unroll
-          for (int r0 = 0; r0 < 32; r0 += 8)
-            *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(ej, 32 * ehalf + r0, 128)) =
-                make_uint4(pack_bf16(d[r0], d[r0 + 1]), pack_bf16(d[r0 + 2], d[r0 + 3]),
-                           pack_bf16(d[r0 + 4], d[r0 + 5]), pack_bf16(d[r0 + 6], d[r0 + 7]));
-        }
-        // decay the state columns: S^T[j][i] *= Gamma_63[i]
-        {
-          const int i0 = 64 * ehalf;
-          float sv[64];
-          tmem_ld16n<4>(tmS + lane_base + i0, sv);
-          tmem_wait_ld();
-#pragma unroll
-          for (int u = 0; u < 64; u += 4) {
-            const float4 gv = *reinterpret_cast<const float4*>(sGC + i0 + u);
-            sv[u] *= gv.x;
-            sv[u + 1] *= gv.y;
-            sv[u + 2] *= gv.z;
-            sv[u + 3] *= gv.w;
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            tmem_st16(tmS + lane_base + i0 + 16 * q, *reinterpret_cast<const float(*)[16]>(sv + 16 * q));
-        }
-        tmem_wait_st();
+        for (int r0 = 0; r0 < 32; r0 += 8)
+          *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(ej, 32 * ehalf + r0, 128)) =
+              make_uint4(pack_bf16(d[r0], d[r0 + 1]), pack_bf16(d[r0 + 2], d[r0 + 3]),
+                         pack_bf16(d[r0 + 4], d[r0 + 5]), pack_bf16(d[r0 + 6], d[r0 + 7]));
       }
+      tmem_wait_st();
       fence_async_smem();
       tc_fence_before();
     }
@@ -828,8 +874,15 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       aborted = true;
       break;
     }
-    // the V tile is free now that the second product completed
-    if (c0 + C < t1 && tid == kPfThread) issue_prefetch_v(c0 + C);
+    // the V tile is free now that the second product completed (and its copy was observed)
+    if (has_v) {
+      v_pending = false;
+      v_parity ^= 1u;
+    }
+    if (c0 + C < t1) {
+      if (tid == kPfThread) issue_prefetch_v(c0 + C);
+      v_pending = has_v;
+    }
 
     // D1[:, 64:128] += Delta^T P^T ;  S^T += Delta^T K'   (accumulate)
     if (tid == kMmaThread) {
@@ -838,20 +891,22 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmD1 + 64, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128(sbase + OFF_P + kk * 32),
                  idesc_bf16_f32(64), 1);
+      mma_commit(bar2);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmS, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128(sbase + OFF_KPT + kk * 32),
                  idesc_bf16_f32(128), 1);
-      mma_commit(bar2);
+      mma_commit(bar4);
     }
+    // the next chunk's gates run on the CUDA cores while these products are on the tensor cores
+    if (c0 + C < t1) gate_phase(rows_of(c0 + C));
     {
-      if (!mbar_wait_bounded(bar2, phase, kWaitLimitNs)) {
-        *s_abort = 1;
-        report(a.status, KDA_ERR_DEVICE_TIMEOUT);
-      } else {
+      // the output is staged while the state update still runs
+      const bool out_done = mbar_wait_bounded(bar2, phase, kWaitLimitNs);
+      if (out_done) {
         tc_fence_after();
-        // outputs O[r][j] staged row-major (bf16 in the X tile, fp32 in the K/Q tile: both are
-        // free once the last products completed; the V tile already receives the next chunk)
+        // outputs O[r][j] staged row-major: bf16 in the spare state tile, fp32 in the K/Q tile
+        // (read by no product still running; the state update still reads the X tile)
         if (a.out) {
           float d[32];
           tmem_ld16n<2>(tmD1 + lane_base + 64 + 32 * ehalf, d);
@@ -859,13 +914,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           if (a.out_bf16) {
 #pragma unroll
             for (int u = 0; u < 32; ++u)
-              *reinterpret_cast<__nv_bfloat16*>(sm + OFF_X + ((32 * ehalf + u) * D + ej) * 2) =
+              *reinterpret_cast<__nv_bfloat16*>(sm + OFF_S + ((32 * ehalf + u) * D + ej) * 2) =
                   __float2bfloat16_rn(d[u]);
           } else {
 #pragma unroll
             for (int u = 0; u < 32; ++u) reinterpret_cast<float*>(sm + OFF_KQ)[(32 * ehalf + u) * D + ej] = d[u];
           }
         }
+      }
+      if (!out_done || !mbar_wait_bounded(bar4, phase, kWaitLimitNs)) {
+        *s_abort = 1;
+        report(a.status, KDA_ERR_DEVICE_TIMEOUT);
+      } else {
+        tc_fence_after();
         // bf16 copy of the new state for the next chunk, into the TMEM A operand
         {
           const int i0 = 64 * ehalf;
@@ -890,14 +951,21 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       aborted = true;
       break;
     }
-    // flush the staged output rows of this chunk
+    // flush the staged output rows of this chunk: a full chunk of a bf16 output leaves through
+    // one tensor store (its source is read before (1) of the next chunk); a partial chunk row
+    // by row, so that no row of the next sequence is touched
     if (!a.out) {
+    } else if (a.out_bf16 && L == C) {
+      if (tid == kPfThread) {
+        tma_store_3d(&tm.out, sbase + OFF_S, 0, h, (int)c0);
+        bulk_commit();
+      }
     } else if (a.out_bf16) {
       for (int e = tid; e < C * 16; e += kThreads) {
         const int row = e >> 4, cc = e & 15;
         if (row < L)
           *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)(c0 + row) * a.Hv + h) * D +
-                                    cc * 8) = *reinterpret_cast<const uint4*>(sm + OFF_X + row * 256 + cc * 16);
+                                    cc * 8) = *reinterpret_cast<const uint4*>(sm + OFF_S + row * 256 + cc * 16);
       }
     } else {
       for (int e = tid; e < C * 32; e += kThreads) {
@@ -908,19 +976,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       }
     }
     } else {
-    // =============================== state side (segment build: both states, no readout)
+    // =============================== state side (segment build: both states; the first
+    // products were issued in the inverse)
     {
-      // D1_M = S_M^T (K o Gamma)^T and D1_U = S_U^T (K o Gamma)^T   (N = 64 each, K = 128)
-      if (tid == kMmaThread) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
-          mma_bf16_ts(tmD1u, tmSbu + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
-        }
-        mma_commit(bar0);
-      }
       if (!mbar_wait_bounded(bar0, phase, kWaitLimitNs)) {
         *s_abort = 1;
         report(a.status, KDA_ERR_DEVICE_TIMEOUT);
@@ -951,6 +1009,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       // Delta_M^T = Y_M^T T^T ;  Delta_U^T = V^T T^T + Y_U^T T^T
       if (tid == kMmaThread) {
         tc_fence_after();
+        if (!mbar_wait_bounded(bar_v, v_parity, kWaitLimitNs)) {  // this chunk's V has landed
+          *s_abort = 1;
+          report(a.status, KDA_ERR_DEVICE_TIMEOUT);
+        }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmD1, desc_sw128(sbase + OFF_XM + kk * 32), desc_sw128(sbase + OFF_T + kk * 32),
@@ -965,46 +1027,45 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
                    idesc_bf16_f32(64), 1);
         mma_commit(bar1);
       }
+      // decay both states while the second products run (they read neither state):
+      // S^T[j][i] *= Gamma_63[i]
+#pragma unroll 1
+      for (int st = 0; st < 2; ++st) {
+        const uint32_t tcol = (st ? tmSu : tmS) + lane_base + 64 * ehalf;
+        float sv[64];
+        tmem_ld16n<4>(tcol, sv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 64; u += 4) {
+          const float4 gv = *reinterpret_cast<const float4*>(sGC + 64 * ehalf + u);
+          sv[u] *= gv.x;
+          sv[u + 1] *= gv.y;
+          sv[u + 2] *= gv.z;
+          sv[u + 3] *= gv.w;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_st16(tcol + 16 * q, *reinterpret_cast<const float(*)[16]>(sv + 16 * q));
+      }
       if (!mbar_wait_bounded(bar1, phase, kWaitLimitNs)) {
         *s_abort = 1;
         report(a.status, KDA_ERR_DEVICE_TIMEOUT);
       } else {
         tc_fence_after();
-        {
-          float d[32], e[32];
-          tmem_ld16n<2>(tmD1 + lane_base + 32 * ehalf, d);
-          tmem_ld16n<2>(tmD1u + lane_base + 32 * ehalf, e);
-          tmem_wait_ld();
+        float d[32], e[32];
+        tmem_ld16n<2>(tmD1 + lane_base + 32 * ehalf, d);
+        tmem_ld16n<2>(tmD1u + lane_base + 32 * ehalf, e);
+        tmem_wait_ld();
 #pragma unroll
-          for (int r0 = 0; r0 < 32; r0 += 8) {
-            *reinterpret_cast<uint4*>(sm + OFF_XM + sw_off(ej, 32 * ehalf + r0, 128)) =
-                make_uint4(pack_bf16(d[r0], d[r0 + 1]), pack_bf16(d[r0 + 2], d[r0 + 3]),
-                           pack_bf16(d[r0 + 4], d[r0 + 5]), pack_bf16(d[r0 + 6], d[r0 + 7]));
-            *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(ej, 32 * ehalf + r0, 128)) =
-                make_uint4(pack_bf16(e[r0], e[r0 + 1]), pack_bf16(e[r0 + 2], e[r0 + 3]),
-                           pack_bf16(e[r0 + 4], e[r0 + 5]), pack_bf16(e[r0 + 6], e[r0 + 7]));
-          }
+        for (int r0 = 0; r0 < 32; r0 += 8) {
+          *reinterpret_cast<uint4*>(sm + OFF_XM + sw_off(ej, 32 * ehalf + r0, 128)) =
+              make_uint4(pack_bf16(d[r0], d[r0 + 1]), pack_bf16(d[r0 + 2], d[r0 + 3]),
+                         pack_bf16(d[r0 + 4], d[r0 + 5]), pack_bf16(d[r0 + 6], d[r0 + 7]));
+          *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(ej, 32 * ehalf + r0, 128)) =
+              make_uint4(pack_bf16(e[r0], e[r0 + 1]), pack_bf16(e[r0 + 2], e[r0 + 3]),
+                         pack_bf16(e[r0 + 4], e[r0 + 5]), pack_bf16(e[r0 + 6], e[r0 + 7]));
         }
-        // decay both states: S^T[j][i] *= Gamma_63[i]
-#pragma unroll 1
-        for (int st = 0; st < 2; ++st) {
-          const uint32_t tcol = (st ? tmSu : tmS) + lane_base + 64 * ehalf;
-          float sv[64];
-          tmem_ld16n<4>(tcol, sv);
-          tmem_wait_ld();
-#pragma unroll
-          for (int u = 0; u < 64; u += 4) {
-            const float4 gv = *reinterpret_cast<const float4*>(sGC + 64 * ehalf + u);
-            sv[u] *= gv.x;
-            sv[u + 1] *= gv.y;
-            sv[u + 2] *= gv.z;
-            sv[u + 3] *= gv.w;
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) tmem_st16(tcol + 16 * q, *reinterpret_cast<const float(*)[16]>(sv + 16 * q));
-        }
-        tmem_wait_st();
       }
+      tmem_wait_st();
       fence_async_smem();
       tc_fence_before();
       __syncthreads();
@@ -1012,8 +1073,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         aborted = true;
         break;
       }
-      // the V tile is free now that the second products completed
-      if (c0 + C < t1 && tid == kPfThread) issue_prefetch_v(c0 + C);
+      // the V tile is free now that the second products completed (and its copy was observed)
+      v_pending = false;
+      v_parity ^= 1u;
+      if (c0 + C < t1) {
+        if (tid == kPfThread) issue_prefetch_v(c0 + C);
+        v_pending = true;
+      }
 
       // [readouts: D_st = S_st,0^T (Q o Gamma)^T + Delta_st^T P^T -- the bf16 copies still hold the
       //  chunk's incoming states]   S_M^T += Delta_M^T K' ;  S_U^T += Delta_U^T K'
@@ -1034,6 +1100,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
               mma_bf16(dcol, desc_sw128(sbase + xoff + kk * 32), desc_sw128(sbase + OFF_P + kk * 32),
                        idesc_bf16_f32(64), 1);
           }
+          mma_commit(bar2);
         }
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -1043,26 +1110,34 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmSu, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128(sbase + OFF_KPT + kk * 32),
                    idesc_bf16_f32(128), 1);
-        mma_commit(bar2);
+        mma_commit(bar4);
       }
-      if (!mbar_wait_bounded(bar2, phase, kWaitLimitNs)) {
-        *s_abort = 1;
-        report(a.status, KDA_ERR_DEVICE_TIMEOUT);
-      } else {
+      // the next chunk's gates run on the CUDA cores while these products are on the tensor cores
+      if (c0 + C < t1) gate_phase(rows_of(c0 + C));
+      // the readouts are staged while the state updates still run
+      const bool read_done = !kRead || mbar_wait_bounded(bar2, phase, kWaitLimitNs);
+      if (read_done) {
         tc_fence_after();
         if constexpr (kRead) {
-          // readouts of both states, staged row-major bf16 in their (now free) X tiles
+          // readouts of both states, staged row-major bf16 in the K/Q tile (its last readers, the
+          // readout products, completed; the state updates still read both X tiles)
 #pragma unroll 1
           for (int st = 0; st < 2; ++st) {
             float d[32];
             tmem_ld16n<2>((st ? tmD1u : tmD1) + lane_base + 32 * ehalf, d);
             tmem_wait_ld();
-            uint8_t* stage = sm + (st ? OFF_X : OFF_XM);
+            uint8_t* stage = sm + OFF_KQ + st * 16384;
 #pragma unroll
             for (int u = 0; u < 32; ++u)
               *reinterpret_cast<__nv_bfloat16*>(stage + ((32 * ehalf + u) * D + ej) * 2) = __float2bfloat16_rn(d[u]);
           }
         }
+      }
+      if (!read_done || !mbar_wait_bounded(bar4, phase, kWaitLimitNs)) {
+        *s_abort = 1;
+        report(a.status, KDA_ERR_DEVICE_TIMEOUT);
+      } else {
+        tc_fence_after();
         // bf16 copies of both new states for the next chunk's first products
 #pragma unroll 1
         for (int st = 0; st < 2; ++st) {
@@ -1088,12 +1163,21 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         break;
       }
       if constexpr (kRead) {
+        // full chunks leave through two tensor stores (sources read before (1) of the next chunk)
+        if (L == C) {
+          if (tid == kPfThread) {
+            tma_store_3d(&tm.out, sbase + OFF_KQ, 0, h, (int)c0);
+            tma_store_3d(&tm.out2, sbase + OFF_KQ + 16384, 0, h, (int)c0);
+            bulk_commit();
+          }
+        } else {
         for (int e = tid; e < 2 * C * 16; e += kThreads) {
           const int st = e >> 10, row = (e >> 4) & 63, cc = e & 15;
           if (row < L)
             *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(st ? a.out2 : a.out) +
                                       ((size_t)(c0 + row) * a.Hv + h) * D + cc * 8) =
-                *reinterpret_cast<const uint4*>(sm + (st ? OFF_X : OFF_XM) + row * 256 + cc * 16);
+                *reinterpret_cast<const uint4*>(sm + OFF_KQ + st * 16384 + row * 256 + cc * 16);
+        }
         }
       }
     }
@@ -1126,6 +1210,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     }
   }
   if (pf_pending) mbar_wait_bounded(bar_pf, pf_parity, kWaitLimitNs);  // copies still in flight
+  if (v_pending) mbar_wait_bounded(bar_v, v_parity, kWaitLimitNs);
+  if (tid == kPfThread) bulk_wait_all();  // output tensor stores
   if (aborted && tid == kMmaThread) {
     // let any MMA still in flight finish before the tensor memory is released
     mma_commit(bar3);
@@ -1191,7 +1277,11 @@ cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream) {
                   encode_rows(&tm.q, a.q ? a.q : a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hk) &&
                   encode_rows(&tm.v, a.v ? a.v : a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv, 64,
                               CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!ok) return cudaErrorInvalidValue;
+  // bf16 outputs (the prefill output, or both readouts of the build) leave through tensor stores
+  const bool out_ok = rows == 0 || !a.out || !a.out_bf16 ||
+                      (encode_rows(&tm.out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv) &&
+                       (!a.out2 || encode_rows(&tm.out2, a.out2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv)));
+  if (!ok || !out_ok) return cudaErrorInvalidValue;
   dim3 grid(a.Hv, a.batch);
   if (a.build && a.out)
     fused_chunk_kernel<true, true><<<grid, kThreads, kSmemAlloc, stream>>>(a, tm);
