@@ -268,9 +268,9 @@ def run_reference(args):
 class Step:
     """One pass of the hot path on device-resident inputs; records per-call CUDA events."""
 
-    def __init__(self, w, stream):
+    def __init__(self, w, stream, public=False):
         import kimi_delta_attention_23_b200 as kda
-        self.kda, self.w, self.stream = kda, w, stream
+        self.kda, self.w, self.stream, self.public = kda, w, stream, public
         dev = w.q.device
         self.cp = w.seg_offsets is not None
         T, Hv, dv, dk = w.total_tokens, w.num_v_heads, w.dv, w.dk
@@ -287,8 +287,22 @@ class Step:
             self.inc = torch.empty((N, Hv, *st), device=dev)
             self.outg = torch.empty((N, Hv, *st), device=dev)
             self.fin = torch.empty((Hv, *st), device=dev)
-            self.rm = torch.empty((T, Hv, dv), dtype=torch.bfloat16, device=dev)
-            self.ru = torch.empty((T, Hv, dv), dtype=torch.bfloat16, device=dev)
+            # the library builds every segment as `pieces` chunk-aligned pieces (more chains than
+            # SMs' worth of segments); the step below makes the same calls as the prefill entry
+            self.pieces = kda.kda_context_parallel_pieces(T, N, Hv)
+            P = N * self.pieces
+            self.P = P
+            if public:
+                self.ws = torch.empty(max(kda.kda_context_parallel_workspace_preferred(T, N, Hv, dv), 1),
+                                      dtype=torch.uint8, device=dev)
+            else:
+                self.rm = torch.empty((T, Hv, dv), dtype=torch.bfloat16, device=dev)
+                self.ru = torch.empty((T, Hv, dv), dtype=torch.bfloat16, device=dev)
+                if self.pieces > 1:
+                    self.poffs = torch.empty(P + 1, dtype=torch.int32, device=dev)
+                    self.pM = torch.empty((P, Hv, dk, dk), device=dev)
+                    self.pU = torch.empty((P, Hv, *st), device=dev)
+                    self.pIn = torch.empty((P + 1, Hv, *st), device=dev)  # slot p + 1: outgoing of piece p
         self.pool = None if self.cp else w.state_pool.clone()
         self.events = []
 
@@ -298,30 +312,58 @@ class Step:
                     gate_lower_bound=w.gate_lower_bound, device_status=self.status, stream=self.stream)
 
     def launches(self):
-        return 3 if self.cp else 1  # segment build with readouts, scan, apply
+        if not self.cp:
+            return 1
+        # (piece boundaries,) segment build with readouts, scan, (composition,) apply
+        return 5 if self.pieces > 1 else 3
 
     def __call__(self, record=False):
         w, kda = self.w, self.kda
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if record else None
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if record else None
         if ev:
             ev[0].record(self.stream)
-        if self.cp:
+        if self.cp and self.public:
+            kda.kda_context_parallel_prefill(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias,
+                                             w.seg_offsets, self.init, self.out, final_state=self.fin, M=self.M,
+                                             U=self.U, incoming=self.inc, outgoing=self.outg, workspace=self.ws,
+                                             **self.kw())
+            for e in (ev or [])[1:]:
+                e.record(self.stream)
+        elif self.cp and self.pieces > 1:
+            kda.kda_context_parallel_piece_offsets(w.seg_offsets, self.pieces, out=self.poffs, stream=self.stream)
+            kda.kda_segment_summarize_and_scan(w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias,
+                                               self.poffs, self.init, M=self.pM, U=self.pU, incoming=self.pIn[:-1],
+                                               outgoing=self.pIn[1:], final_state=self.fin, q=w.q,
+                                               readout_m=self.rm, readout_u=self.ru, **self.kw())
+            if ev:
+                ev[1].record(self.stream)
+            kda.kda_segment_compose(self.pM, self.pU, self.pIn, self.fin, self.pieces, M=self.M, U=self.U,
+                                    incoming=self.inc, outgoing=self.outg, state_layout=w.state_layout,
+                                    stream=self.stream)
+            if ev:
+                ev[2].record(self.stream)
+            kda.kda_context_parallel_apply(self.rm, self.ru, self.pIn[:-1], self.poffs, self.out,
+                                           state_layout=w.state_layout, device_status=self.status,
+                                           stream=self.stream)
+        elif self.cp:
             kda.kda_segment_summarize_and_scan(w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias,
                                                w.seg_offsets, self.init, M=self.M, U=self.U, incoming=self.inc,
                                                outgoing=self.outg, final_state=self.fin, q=w.q, readout_m=self.rm,
                                                readout_u=self.ru, **self.kw())
             if ev:
                 ev[1].record(self.stream)
+                ev[2].record(self.stream)
             kda.kda_context_parallel_apply(self.rm, self.ru, self.inc, w.seg_offsets, self.out,
                                            state_layout=w.state_layout, device_status=self.status,
                                            stream=self.stream)
         else:
             if ev:
                 ev[1].record(self.stream)
+                ev[2].record(self.stream)
             kda.kda_chunk_fwd(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens,
                               self.pool, w.state_indices, self.out, **self.kw())
         if ev:
-            ev[2].record(self.stream)
+            ev[3].record(self.stream)
             self.events.append(ev)
 
 
@@ -364,7 +406,8 @@ def run_ours(args):
     barrier()
     ms_total = start.elapsed_time(stop)
     seg_ms = [e[0].elapsed_time(e[1]) for e in step.events]
-    pass_ms = [e[1].elapsed_time(e[2]) for e in step.events]
+    comp_ms = [e[1].elapsed_time(e[2]) for e in step.events]
+    pass_ms = [e[2].elapsed_time(e[3]) for e in step.events]
     ms_total = max_over_ranks(ms_total, pg, dev)
     ms_step = ms_total / args.steps
     tokens = w.total_tokens
@@ -382,10 +425,12 @@ def run_ours(args):
     ms_pass = statistics.mean(pass_ms)
     ms_seg = statistics.mean(seg_ms) if step.cp else 0.0
     if step.cp:
-        # dominant launch: the segment build with readouts (its call also runs the short scan)
+        # dominant launch: the segment build with readouts over the pieces (its call also runs the
+        # short scan; the piece boundaries are computed first, in a negligible launch)
         dom, bytes_dom, ms_dom = "fused_chunk_kernel<build,readout> + affine_scan_kernel", \
-            segment_build_bytes(w, step.N), ms_seg
-        breakdown = {"segment_build_and_scan": ms_seg, "context_parallel_apply": ms_pass}
+            segment_build_bytes(w, step.P), ms_seg
+        breakdown = {"segment_build_and_scan": ms_seg, "compose_pieces": statistics.mean(comp_ms),
+                     "context_parallel_apply": ms_pass}
     else:
         dom, bytes_dom, ms_dom = "fused_chunk_kernel<prefill>", chunk_fwd_bytes(w, w.batch), ms_pass
         breakdown = {"chunk_fwd": ms_pass}
@@ -399,10 +444,11 @@ def run_ours(args):
             "vs_baseline": None, "dtype": "bf16" if w.q.dtype == torch.bfloat16 else "f32", "data": "synthetic",
             "config": {"workload": args.workload, "tokens": tokens, "num_v_heads": w.num_v_heads,
                        "num_k_heads": w.num_k_heads, "dk": w.dk, "dv": w.dv, "batch": w.batch,
-                       "segments": step.N if step.cp else None, "gate_mode": w.gate_mode,
+                       "segments": step.N if step.cp else None,
+                       "pieces_per_segment": step.pieces if step.cp else None, "gate_mode": w.gate_mode,
                        "state_layout": w.state_layout, "parallelism": f"dp{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (%.2f GB read per step), no flush" % (
-                           (segment_build_bytes(w, step.N) if step.cp else chunk_fwd_bytes(w, w.batch)) / 1e9)},
+                           (segment_build_bytes(w, step.P) if step.cp else chunk_fwd_bytes(w, w.batch)) / 1e9)},
             "breakdown_ms": breakdown,
             "roofline": roof, "gpu_launches": step.launches() * args.steps, "clocks": clocks.summary()}
     if e2e is not None:
@@ -425,7 +471,7 @@ def measure_e2e(w, args, stream, pg):
     wd = W.Workload(**{k: getattr(w, k) for k in w.__dataclass_fields__})
     for n in names:
         setattr(wd, n, torch.empty_like(getattr(w, n)))
-    step = Step(wd, stream)
+    step = Step(wd, stream, public=True)
     out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
     fin_src = step.fin if step.cp else step.pool
     fin_host = torch.empty(fin_src.shape, dtype=fin_src.dtype).pin_memory()

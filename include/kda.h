@@ -188,7 +188,10 @@ KDA_API kda_status_t kda_context_parallel_apply(const void *readout_m, const voi
  *   M [N,Hv,dk,dk], U / incoming / outgoing [N,Hv,<state>] fp32, written (as in
  *     kda_segment_summarize_and_scan)
  *   workspace >= kda_context_parallel_workspace_size(T, num_v_heads, dv) bytes, 256-byte aligned
- *     device memory; its contents on return are unspecified
+ *     device memory; its contents on return are unspecified.  Given at least
+ *     kda_context_parallel_workspace_preferred(T, N, num_v_heads, dv) bytes, the build runs each
+ *     segment as several chunk-aligned pieces (more chains for the SMs; the results are the
+ *     same up to rounding) and composes each segment's M_i, U_i from its pieces'.
  * Supported: bf16 q/k/v with dk = dv = 128; otherwise KDA_ERR_UNSUPPORTED.
  */
 KDA_API kda_status_t kda_context_parallel_prefill(
@@ -228,6 +231,43 @@ KDA_API kda_status_t kda_context_parallel_prefill_static(
 
 /* Workspace bytes kda_context_parallel_prefill needs: the two bf16 readouts, 2 * T * Hv * dv * 2. */
 KDA_API size_t kda_context_parallel_workspace_size(int64_t T, int32_t num_v_heads, int32_t dv);
+
+/*
+ * kda_segment_compose -- summaries of segments from the summaries of their pieces: segment i
+ * consists of `pieces` consecutive pieces i*pieces .. i*pieces + pieces - 1 (as built by
+ * kda_segment_summarize_and_scan over the piece boundaries), and its map is their composition
+ * in order ("KDA Context Parallelism", Compose segments in sequence order:
+ * (M2, U2) o (M1, U1) = (M2 M1, M2 U1 + U2)).
+ *
+ *   M_pieces [N*pieces, Hv, dk, dk], U_pieces / incoming_pieces [N*pieces, Hv, <state>] fp32
+ *   final_state [Hv, <state>] (the scan's final state: the last segment's outgoing state)
+ *   M [N, Hv, dk, dk], U / incoming / outgoing [N, Hv, <state>] fp32, written: incoming[i] is
+ *     the incoming state of segment i's first piece, outgoing[i] that of segment i + 1's
+ *   flags: KDA_STATE_V_FIRST selects <state> = [dv, dk]; dk, dv <= 128 (fp32 CUDA-core kernel)
+ */
+KDA_API kda_status_t kda_segment_compose(const float *M_pieces, const float *U_pieces,
+                                         const float *incoming_pieces, const float *final_state,
+                                         int32_t num_segments, int32_t pieces, int32_t num_v_heads,
+                                         int32_t dk, int32_t dv, float *M, float *U, float *incoming,
+                                         float *outgoing, uint32_t flags, void *stream);
+
+/* Pieces per segment (1..8) that kda_context_parallel_prefill builds on the current device. */
+KDA_API int32_t kda_context_parallel_pieces(int64_t T, int32_t num_segments, int32_t num_v_heads);
+
+/* Piece boundaries: piece_offsets [N*pieces + 1] (device int32, written) from seg_offsets [N+1]:
+ * piece p of segment [s0, s1) with nch = ceil((s1 - s0) / 64) chunks starts at token
+ * s0 + 64 * floor(nch * p / pieces), capped at s1 (short segments give empty pieces); the last
+ * entry is seg_offsets[N].  Decreasing seg_offsets give decreasing piece offsets, which the
+ * segment build reports as KDA_ERR_DEVICE_CHECK. */
+KDA_API kda_status_t kda_context_parallel_piece_offsets(const int32_t *seg_offsets, int32_t num_segments,
+                                                        int32_t pieces, int32_t *piece_offsets, void *stream);
+
+/* Workspace bytes with which kda_context_parallel_prefill splits the segments into pieces on
+ * the current device (the readouts, plus per piece a transition, a contribution and an incoming
+ * state); equal to kda_context_parallel_workspace_size when no split pays off.  Depends on the
+ * current device's SM count: query it with the device current that will run the prefill. */
+KDA_API size_t kda_context_parallel_workspace_preferred(int64_t T, int32_t num_segments,
+                                                        int32_t num_v_heads, int32_t dv);
 
 /* Bytes of workspace kda_chunk_fwd / kda_segment_summarize_and_scan need for these extents
  * (0 for the current kernels). */

@@ -19,7 +19,9 @@ import os
 import torch
 
 __all__ = ["kda_chunk_fwd", "kda_segment_summarize_and_scan", "kda_context_parallel",
-           "kda_context_parallel_apply", "kda_context_parallel_prefill", "kda_context_parallel_workspace_size", "kda_workspace_size",
+           "kda_context_parallel_apply", "kda_context_parallel_prefill", "kda_context_parallel_workspace_size",
+           "kda_context_parallel_workspace_preferred", "kda_context_parallel_pieces",
+           "kda_context_parallel_piece_offsets", "kda_segment_compose", "kda_workspace_size",
            "kda_status_string", "load_library", "KdaError", "LIB_PATH"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +72,14 @@ def load_library():
                                                  ip, vp]
     lib.kda_context_parallel_workspace_size.restype = sz
     lib.kda_context_parallel_workspace_size.argtypes = [i64, i32, i32]
+    lib.kda_context_parallel_piece_offsets.restype = ctypes.c_int
+    lib.kda_context_parallel_piece_offsets.argtypes = [ip, i32, i32, ip, vp]
+    lib.kda_context_parallel_pieces.restype = i32
+    lib.kda_context_parallel_pieces.argtypes = [i64, i32, i32]
+    lib.kda_segment_compose.restype = ctypes.c_int
+    lib.kda_segment_compose.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, u32, vp]
+    lib.kda_context_parallel_workspace_preferred.restype = sz
+    lib.kda_context_parallel_workspace_preferred.argtypes = [i64, i32, i32, i32]
     lib.kda_workspace_size.restype = sz
     lib.kda_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32, i32, u32]
     lib.kda_status_string.restype = ctypes.c_char_p
@@ -322,6 +332,70 @@ def kda_context_parallel_workspace_size(T, num_v_heads, dv=128) -> int:
     return int(load_library().kda_context_parallel_workspace_size(T, num_v_heads, dv))
 
 
+def kda_context_parallel_pieces(T, num_segments, num_v_heads) -> int:
+    """Pieces per segment the context-parallel prefill builds on the current device."""
+    return int(load_library().kda_context_parallel_pieces(T, num_segments, num_v_heads))
+
+
+def kda_context_parallel_piece_offsets(seg_offsets, pieces, *, out=None, stream=None):
+    """Chunk-aligned boundaries of ``pieces`` pieces per segment (device int32 [N*pieces + 1])."""
+    lib = load_library()
+    dev = seg_offsets.device
+    _dev(seg_offsets, "seg_offsets", torch.int32, dev)
+    N = seg_offsets.numel() - 1
+    if out is None:
+        out = torch.empty(N * pieces + 1, dtype=torch.int32, device=dev)
+    _shape(_dev(out, "out", torch.int32, dev), "out", (N * pieces + 1,))
+    rc = lib.kda_context_parallel_piece_offsets(_ptr(seg_offsets), N, pieces, _ptr(out), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_context_parallel_piece_offsets")
+    return out
+
+
+def kda_segment_compose(M_pieces, U_pieces, incoming_pieces, final_state, pieces, *, M=None, U=None,
+                        incoming=None, outgoing=None, state_layout="K_FIRST", stream=None):
+    """Segment summaries (and incoming/outgoing states) composed from those of their pieces.
+
+    Returns dict(transition_matrices, local_contributions, incoming_states, outgoing_states).
+    """
+    lib = load_library()
+    dev = M_pieces.device
+    _dev(M_pieces, "M_pieces", torch.float32, dev)
+    NP, Hv, dk = M_pieces.shape[0], M_pieces.shape[1], M_pieces.shape[2]
+    if NP % pieces:
+        raise ValueError("the piece count must divide the number of pieces")
+    N = NP // pieces
+    st = tuple(U_pieces.shape[2:])
+    dv = st[1] if state_layout == "K_FIRST" else st[0]
+    _shape(_dev(U_pieces, "U_pieces", torch.float32, dev), "U_pieces", (NP, Hv, *st))
+    _dev(incoming_pieces, "incoming_pieces", torch.float32, dev)
+    if incoming_pieces.shape[0] < NP or tuple(incoming_pieces.shape[1:]) != (Hv, *st):
+        raise ValueError("incoming_pieces must be [>= N*pieces, Hv, <state>]")
+    _shape(_dev(final_state, "final_state", torch.float32, dev), "final_state", (Hv, *st))
+
+    def buf(t, name, shape):
+        if t is None:
+            return torch.empty(shape, dtype=torch.float32, device=dev)
+        _shape(_dev(t, name, torch.float32, dev), name, shape)
+        return t
+
+    M = buf(M, "M", (N, Hv, dk, dk))
+    U = buf(U, "U", (N, Hv, *st))
+    incoming = buf(incoming, "incoming", (N, Hv, *st))
+    outgoing = buf(outgoing, "outgoing", (N, Hv, *st))
+    rc = lib.kda_segment_compose(_ptr(M_pieces), _ptr(U_pieces), _ptr(incoming_pieces), _ptr(final_state), N,
+                                 pieces, Hv, dk, dv, _ptr(M), _ptr(U), _ptr(incoming), _ptr(outgoing),
+                                 _flags("original", "logits", state_layout), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_segment_compose")
+    return {"transition_matrices": M, "local_contributions": U, "incoming_states": incoming,
+            "outgoing_states": outgoing}
+
+
+def kda_context_parallel_workspace_preferred(T, num_segments, num_v_heads, dv=128) -> int:
+    return int(load_library().kda_context_parallel_workspace_preferred(T, num_segments, num_v_heads, dv))
+
+
 def kda_context_parallel_prefill(q, k, v, raw_gate, beta_logits, a_log, dt_bias, seg_offsets, initial_state,
                                  out=None, *, final_state=None, M=None, U=None, incoming=None, outgoing=None,
                                  workspace=None, output_dtype=None, gate_mode="original", beta_mode="logits",
@@ -330,7 +404,8 @@ def kda_context_parallel_prefill(q, k, v, raw_gate, beta_logits, a_log, dt_bias,
 
     Returns dict(out, final_state, incoming_states, outgoing_states, transition_matrices,
     local_contributions).  ``workspace`` (uint8 CUDA tensor of at least
-    kda_context_parallel_workspace_size bytes) is allocated when not given.
+    kda_context_parallel_workspace_size bytes) is allocated when not given, at the preferred size
+    (kda_context_parallel_workspace_preferred: enough to build the segments as pieces).
     """
     lib = load_library()
     dev = q.device
@@ -365,9 +440,10 @@ def kda_context_parallel_prefill(q, k, v, raw_gate, beta_logits, a_log, dt_bias,
     U = buf(U, "U", (N, Hv, *st))
     incoming = buf(incoming, "incoming", (N, Hv, *st))
     outgoing = buf(outgoing, "outgoing", (N, Hv, *st))
-    need = kda_context_parallel_workspace_size(T, Hv, dv)
     if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        with torch.cuda.device(dev):
+            pref = kda_context_parallel_workspace_preferred(T, N, Hv, dv)
+        workspace = torch.empty(max(pref, 1), dtype=torch.uint8, device=dev)
     _dev(workspace, "workspace", torch.uint8, dev)
     flags = _flags(gate_mode, beta_mode, state_layout)
     rc = lib.kda_context_parallel_prefill(_ptr(q), _ptr(k), _ptr(v), _BF16, _ptr(raw_gate), _ptr(beta_logits),

@@ -23,6 +23,40 @@ bool dtype_ok(kda_dtype_t t) { return t == KDA_F32 || t == KDA_BF16; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// Pieces per segment for the context-parallel segment build.  The fused kernel runs one chain
+// (segment piece, head) per SM, so N * Hv chains take ceil(N Hv / SMs) rounds of a whole
+// segment's length; k pieces per segment take ceil(k N Hv / SMs) rounds of 1/k of it.  The
+// smallest k (up to 8) that saves at least 3 % is taken, with pieces of four chunks or more on
+// average.
+int choose_pieces(int64_t T, int32_t N, int32_t Hv) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                 cudaSuccess || sms <= 0)
+    return 1;
+  const int64_t chains = (int64_t)N * Hv;
+  double best = (double)((chains + sms - 1) / sms);
+  int best_k = 1;
+  for (int k = 2; k <= 8; ++k) {
+    if (T < (int64_t)N * k * 256) break;
+    const double cost = (double)((chains * k + sms - 1) / sms) / k;
+    if (cost < best * 0.97) {
+      best = cost;
+      best_k = k;
+    }
+  }
+  return best_k;
+}
+
+// workspace bytes of the pieces: boundaries, transitions, contributions, incoming states (one
+// extra slot: the scan's outgoing state of piece p is the incoming state of piece p + 1)
+size_t pieces_bytes(int32_t N, int k, int32_t Hv, int32_t dk, int32_t dv) {
+  const size_t np = (size_t)N * k;
+  return round256((np + 1) * sizeof(int32_t)) + np * Hv * (size_t)dk * dk * sizeof(float) +
+         np * Hv * (size_t)dk * dv * sizeof(float) + (np + 1) * Hv * (size_t)dk * dv * sizeof(float);
+}
+
 }  // namespace
 
 extern "C" kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,
@@ -236,6 +270,57 @@ extern "C" size_t kda_context_parallel_workspace_size(int64_t T, int32_t num_v_h
   return (size_t)2 * (size_t)T * (size_t)num_v_heads * (size_t)dv * 2;
 }
 
+extern "C" int32_t kda_context_parallel_pieces(int64_t T, int32_t num_segments, int32_t num_v_heads) {
+  if (T < 0 || num_segments < 1 || num_v_heads <= 0) return 1;
+  return choose_pieces(T, num_segments, num_v_heads);
+}
+
+extern "C" kda_status_t kda_context_parallel_piece_offsets(const int32_t* seg_offsets, int32_t num_segments,
+                                                           int32_t pieces, int32_t* piece_offsets, void* stream) {
+  if (num_segments < 1 || pieces < 1 || !seg_offsets || !piece_offsets) return KDA_ERR_INVALID_ARG;
+  return kda::launch_split_offsets(seg_offsets, num_segments, pieces, piece_offsets,
+                                   reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KDA_OK
+             : KDA_ERR_CUDA;
+}
+
+extern "C" kda_status_t kda_segment_compose(const float* M_pieces, const float* U_pieces,
+                                            const float* incoming_pieces, const float* final_state,
+                                            int32_t num_segments, int32_t pieces, int32_t num_v_heads, int32_t dk,
+                                            int32_t dv, float* M, float* U, float* incoming, float* outgoing,
+                                            uint32_t flags, void* stream) {
+  if (num_segments < 1 || pieces < 1 || num_v_heads <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+  if ((flags & ~kKnownFlags) != 0) return KDA_ERR_INVALID_ARG;
+  if (!M_pieces || !U_pieces || !incoming_pieces || !final_state || !M || !U || !incoming || !outgoing)
+    return KDA_ERR_INVALID_ARG;
+  if (dk > 128 || dv > 128) return KDA_ERR_UNSUPPORTED;
+  kda::ComposeArgs ca{};
+  ca.M = M_pieces;
+  ca.U = U_pieces;
+  ca.inc = incoming_pieces;
+  ca.final_state = final_state;
+  ca.N = num_segments;
+  ca.k = pieces;
+  ca.H = num_v_heads;
+  ca.dk = dk;
+  ca.dv = dv;
+  ca.v_first = (flags & KDA_STATE_V_FIRST) ? 1 : 0;
+  ca.M_out = M;
+  ca.U_out = U;
+  ca.incoming = incoming;
+  ca.outgoing = outgoing;
+  return kda::launch_compose_pieces(ca, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? KDA_OK
+                                                                                                 : KDA_ERR_CUDA;
+}
+
+extern "C" size_t kda_context_parallel_workspace_preferred(int64_t T, int32_t num_segments, int32_t num_v_heads,
+                                                           int32_t dv) {
+  const size_t base = kda_context_parallel_workspace_size(T, num_v_heads, dv);
+  if (base == 0 || num_segments < 1) return base;
+  const int k = choose_pieces(T, num_segments, num_v_heads);
+  return k > 1 ? round256(base) + pieces_bytes(num_segments, k, num_v_heads, dv, dv) : base;
+}
+
 extern "C" kda_status_t kda_context_parallel_apply(const void* readout_m, const void* readout_u,
                                                    const float* incoming, const int32_t* seg_offsets,
                                                    int32_t num_segments, int64_t T, int32_t num_v_heads, int32_t dv,
@@ -280,6 +365,32 @@ extern "C" kda_status_t kda_context_parallel_prefill(
     return KDA_ERR_WORKSPACE;
   __nv_bfloat16_raw* o_m = reinterpret_cast<__nv_bfloat16_raw*>(workspace);
   __nv_bfloat16_raw* o_u = o_m + (size_t)T * num_v_heads * dv;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int kp = choose_pieces(T, num_segments, num_v_heads);
+  if (kp > 1 && workspace_bytes >= round256(need) + pieces_bytes(num_segments, kp, num_v_heads, dk, dv)) {
+    // more chains than segments: every segment is built as kp chunk-aligned pieces, the scan
+    // runs over the pieces, and each segment's summary is composed from its pieces'
+    const int32_t np = num_segments * kp;
+    uint8_t* w = reinterpret_cast<uint8_t*>(workspace) + round256(need);
+    int32_t* sub = reinterpret_cast<int32_t*>(w);
+    w += round256((size_t)(np + 1) * sizeof(int32_t));
+    float* pM = reinterpret_cast<float*>(w);
+    float* pU = pM + (size_t)np * num_v_heads * dk * dk;
+    float* pIn = pU + (size_t)np * num_v_heads * dk * dv;
+    const size_t blk = (size_t)num_v_heads * dk * dv;
+    kda_status_t st = kda_context_parallel_piece_offsets(seg_offsets, num_segments, kp, sub, stream);
+    if (st != KDA_OK) return st;
+    st = kda_segment_summarize_and_scan(
+        k, v, qkv_dtype, raw_gate, beta_logits, a_log, dt_bias, T, num_k_heads, num_v_heads, dk, dv, sub, np,
+        initial_state, pM, pU, pIn, pIn + blk, final_state, q, o_m, o_u, flags, gate_lower_bound, nullptr, 0,
+        device_status, stream);
+    if (st != KDA_OK) return st;
+    st = kda_segment_compose(pM, pU, pIn, final_state, num_segments, kp, num_v_heads, dk, dv, M, U, incoming,
+                             outgoing, flags & KDA_STATE_V_FIRST, stream);
+    if (st != KDA_OK) return st;
+    return kda_context_parallel_apply(o_m, o_u, pIn, sub, np, T, num_v_heads, dv, out, out_dtype,
+                                      flags & KDA_STATE_V_FIRST, device_status, stream);
+  }
   // every segment in parallel (M_i, U_i and both readouts), then the exclusive scan
   kda_status_t st = kda_segment_summarize_and_scan(k, v, qkv_dtype, raw_gate, beta_logits, a_log, dt_bias, T,
                                                    num_k_heads, num_v_heads, dk, dv, seg_offsets, num_segments,

@@ -94,7 +94,22 @@ struct ApplyArgs {
   int32_t* status;
 };
 
+// Summaries of segments split into k pieces each, rebuilt from the pieces' summaries.
+struct ComposeArgs {
+  const float* M;            // [N*k][H][dk][dk] the pieces' transitions (row-major)
+  const float* U;            // [N*k][H][state] the pieces' contributions
+  const float* inc;          // [N*k][H][state] the pieces' incoming states
+  const float* final_state;  // [H][state]
+  int32_t N, k, H, dk, dv, v_first;
+  float* M_out;              // [N][H][dk][dk]
+  float* U_out;              // [N][H][state]
+  float* incoming;           // [N][H][state]
+  float* outgoing;           // [N][H][state]
+};
+
 size_t simt_smem_bytes(int dk, int w);
+cudaError_t launch_split_offsets(const int32_t* offs, int32_t N, int32_t k, int32_t* sub, cudaStream_t stream);
+cudaError_t launch_compose_pieces(const ComposeArgs& a, cudaStream_t stream);
 cudaError_t launch_cp_apply(const ApplyArgs& a, cudaStream_t stream);
 cudaError_t launch_simt_chunk(const SimtArgs& a, cudaStream_t stream);
 cudaError_t launch_affine_scan(const ScanArgs& a, cudaStream_t stream);

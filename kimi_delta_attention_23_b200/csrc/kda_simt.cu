@@ -187,7 +187,7 @@ cudaError_t launch_simt_chunk(const SimtArgs& a, cudaStream_t stream) {
 // ------------------------------------------------------------------------------------------
 // Exclusive affine scan ("KDA Context Parallelism", Incoming and outgoing states):
 //   in_0 = S_initial;  out_i = M_i in_i + U_i;  in_{i+1} = out_i;  final = out_{N-1}.
-// One block per (head, 32-column tile of the state); the segment loop is serial.
+// One block per (head, 16-column tile of the state); the segment loop is serial.
 // ------------------------------------------------------------------------------------------
 constexpr int kScanCols = 16;
 constexpr int kScanThreads = 256;
@@ -263,7 +263,18 @@ __global__ void __launch_bounds__(kScanThreads) affine_scan_kernel(ScanArgs a) {
   }
 }
 
+bool tiles128(int dk, int dv);
+__global__ void affine_scan128_kernel(ScanArgs a);
+__global__ void compose128_kernel(ComposeArgs a);
+
 cudaError_t launch_affine_scan(const ScanArgs& a, cudaStream_t stream) {
+  if (tiles128(a.dk, a.dv)) {
+    const int smem = (2 * 128 * 132 + 128 * 32) * (int)sizeof(float);
+    cudaError_t err = cudaFuncSetAttribute(affine_scan128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    affine_scan128_kernel<<<dim3(a.H, a.dv / 32), 256, smem, stream>>>(a);
+    return cudaGetLastError();
+  }
   const size_t smem = ((size_t)a.dk * (a.dk + 1) + 2 * (size_t)a.dk * kScanCols) * sizeof(float);
   cudaError_t err = cudaFuncSetAttribute(affine_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -272,5 +283,283 @@ cudaError_t launch_affine_scan(const ScanArgs& a, cudaStream_t stream) {
   affine_scan_kernel<<<grid, kScanThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
+
+// ------------------------------------------------------------------------------------------
+// Segments split into pieces (more chains for the segment build than segments): the pieces'
+// boundaries, and each segment's summary rebuilt from its pieces' summaries by composing them
+// in order ("KDA Context Parallelism", Theory: (M2, U2) o (M1, U1) = (M2 M1, M2 U1 + U2)).
+// ------------------------------------------------------------------------------------------
+
+// Piece p of segment i covers chunk-aligned tokens [s0 + 64 floor(nch p / k), ...) of the
+// segment [s0, s1) (nch = its 64-token chunks); decreasing offsets stay decreasing.
+__global__ void split_offsets_kernel(const int32_t* offs, int32_t N, int32_t k, int32_t* sub) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e > N * k) return;
+  const int i = e / k, p = e % k;
+  if (i == N) {
+    sub[e] = offs[N];
+    return;
+  }
+  const int64_t s0 = offs[i], s1 = offs[i + 1];
+  const int64_t nch = s1 > s0 ? (s1 - s0 + 63) / 64 : 0;
+  const int64_t b = s0 + 64 * ((nch * p) / k);
+  sub[e] = (int32_t)(b < s1 ? b : (s1 > s0 ? s1 : s0));
+}
+
+cudaError_t launch_split_offsets(const int32_t* offs, int32_t N, int32_t k, int32_t* sub, cudaStream_t stream) {
+  const int n = N * k + 1;
+  split_offsets_kernel<<<(n + 255) / 256, 256, 0, stream>>>(offs, N, k, sub);
+  return cudaGetLastError();
+}
+
+// One block per (segment, head, 16-column tile): tiles of M_i (dk columns) carry the product of
+// the pieces' transitions from I; tiles of U_i (dv columns) carry the pieces' affine maps from
+// 0.  The U tiles also copy the segment's incoming state (its first piece's) and outgoing state
+// (the next segment's incoming state, or the final state).
+__global__ void __launch_bounds__(kScanThreads) compose_pieces_kernel(ComposeArgs a) {
+  extern __shared__ float sm[];
+  const int h = blockIdx.x, seg = blockIdx.z, tid = threadIdx.x;
+  const int dk = a.dk, dv = a.dv, H = a.H, k = a.k;
+  const int nbm = (dk + kScanCols - 1) / kScanCols;
+  const bool is_m = (int)blockIdx.y < nbm;
+  const int j0 = (is_m ? (int)blockIdx.y : (int)blockIdx.y - nbm) * kScanCols;
+  const int width = is_m ? dk : dv;
+  const int nc = min(kScanCols, width - j0);
+  float* Ms = sm;                   // [dk][dk + 1]
+  float* cur = Ms + dk * (dk + 1);  // [dk][kScanCols]
+  float* nxt = cur + dk * kScanCols;
+  const size_t st = (size_t)dk * dv;
+  for (int e = tid; e < dk * kScanCols; e += kScanThreads) {
+    const int i = e / kScanCols, jj = e % kScanCols;
+    cur[e] = (is_m && jj < nc && i == j0 + jj) ? 1.f : 0.f;
+  }
+  const int row = tid >> 1, c0 = (tid & 1) * 8;
+  for (int p = 0; p < k; ++p) {
+    const size_t piece = (size_t)seg * k + p;
+    const float* Mg = a.M + (piece * H + h) * (size_t)dk * dk;
+    __syncthreads();
+    for (int e = tid; e < dk * dk; e += kScanThreads) Ms[(e / dk) * (dk + 1) + e % dk] = Mg[e];
+    __syncthreads();
+    for (int r = row; r < dk; r += kScanThreads / 2) {
+      float acc[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+      const float* mrow = Ms + r * (dk + 1);
+      for (int l = 0; l < dk; ++l) {
+        const float m = mrow[l];
+        const float* cr = cur + l * kScanCols + c0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[u] = fmaf(m, cr[u], acc[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int jj = c0 + u;
+        if (jj >= nc) continue;
+        nxt[r * kScanCols + jj] =
+            is_m ? acc[u] : acc[u] + a.U[(piece * H + h) * st + state_off(r, j0 + jj, dk, dv, a.v_first)];
+      }
+    }
+    __syncthreads();
+    float* t = cur;
+    cur = nxt;
+    nxt = t;
+  }
+  for (int e = tid; e < dk * kScanCols; e += kScanThreads) {
+    const int i = e / kScanCols, jj = e % kScanCols;
+    if (jj >= nc) continue;
+    if (is_m) {
+      a.M_out[((size_t)seg * H + h) * (size_t)dk * dk + (size_t)i * dk + j0 + jj] = cur[e];
+    } else {
+      const size_t o = state_off(i, j0 + jj, dk, dv, a.v_first);
+      a.U_out[((size_t)seg * H + h) * st + o] = cur[e];
+      a.incoming[((size_t)seg * H + h) * st + o] = a.inc[((size_t)seg * k * H + h) * st + o];
+      a.outgoing[((size_t)seg * H + h) * st + o] =
+          seg + 1 < a.N ? a.inc[((size_t)(seg + 1) * k * H + h) * st + o] : a.final_state[(size_t)h * st + o];
+    }
+  }
+}
+
+cudaError_t launch_compose_pieces(const ComposeArgs& a, cudaStream_t stream) {
+  if (tiles128(a.dk, a.dv)) {
+    const int smem = (128 * 132 + 128 * 32) * (int)sizeof(float);
+    cudaError_t err = cudaFuncSetAttribute(compose128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    compose128_kernel<<<dim3(a.H, 4 + a.dv / 32, a.N), 256, smem, stream>>>(a);
+    return cudaGetLastError();
+  }
+  const size_t smem = ((size_t)a.dk * (a.dk + 1) + 2 * (size_t)a.dk * kScanCols) * sizeof(float);
+  cudaError_t err = cudaFuncSetAttribute(compose_pieces_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+  if (err != cudaSuccess) return err;
+  dim3 grid(a.H, (a.dk + kScanCols - 1) / kScanCols + (a.dv + kScanCols - 1) / kScanCols, a.N);
+  compose_pieces_kernel<<<grid, kScanThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------
+// dk = 128 forms of the scan and of the composition: 128 x 32 tiles, M staged row-major in
+// shared memory by 16-byte asynchronous copies (double-buffered along the scan), thread t owning
+// rows t/8 + 32 i (i < 4) and columns 4 (t % 8) .. + 3 (sixteen accumulators; each M element
+// read from shared memory feeds four of them, each float4 of the carried tile sixteen).
+// ------------------------------------------------------------------------------------------
+constexpr int kT = 32;          // tile columns
+constexpr int kLdM = 132;       // padded row of the staged M: 16-byte rows, conflict-free column reads
+constexpr int kTileThreads = 256;
+
+__device__ __forceinline__ void cp_async16_g2s(float* dst, const float* src) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_groups() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// M (128 x 128 fp32, row-major in global memory) into a padded shared tile
+__device__ __forceinline__ void stage_m(float* Ms, const float* Mg) {
+  for (int e = threadIdx.x; e < 128 * 32; e += kTileThreads) {
+    const int r = e >> 5, c = (e & 31) * 4;
+    cp_async16_g2s(Ms + r * kLdM + c, Mg + r * 128 + c);
+  }
+  cp_async_commit_group();
+}
+
+// acc[i][u] = sum_l Ms[rows_i][l] cur[l][c0 + u]
+__device__ __forceinline__ void tile_product(const float* Ms, const float* cur, float acc[4][4]) {
+  const int rb = threadIdx.x >> 3, c0 = (threadIdx.x & 7) * 4;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[i][u] = 0.f;
+#pragma unroll 4
+  for (int l = 0; l < 128; ++l) {
+    const float4 b = *reinterpret_cast<const float4*>(cur + l * kT + c0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float m = Ms[(rb + 32 * i) * kLdM + l];
+      acc[i][0] = fmaf(m, b.x, acc[i][0]);
+      acc[i][1] = fmaf(m, b.y, acc[i][1]);
+      acc[i][2] = fmaf(m, b.z, acc[i][2]);
+      acc[i][3] = fmaf(m, b.w, acc[i][3]);
+    }
+  }
+}
+
+// four consecutive columns j0 + c0 .. + 3 of row r of a state block in either layout
+__device__ __forceinline__ float4 load_state4(const float* blk, int r, int j, int dv, int v_first) {
+  if (!v_first) return *reinterpret_cast<const float4*>(blk + (size_t)r * dv + j);
+  return make_float4(blk[(size_t)j * 128 + r], blk[(size_t)(j + 1) * 128 + r], blk[(size_t)(j + 2) * 128 + r],
+                     blk[(size_t)(j + 3) * 128 + r]);
+}
+__device__ __forceinline__ void store_state4(float* blk, int r, int j, int dv, int v_first, float4 x) {
+  if (!v_first) {
+    *reinterpret_cast<float4*>(blk + (size_t)r * dv + j) = x;
+  } else {
+    blk[(size_t)j * 128 + r] = x.x;
+    blk[(size_t)(j + 1) * 128 + r] = x.y;
+    blk[(size_t)(j + 2) * 128 + r] = x.z;
+    blk[(size_t)(j + 3) * 128 + r] = x.w;
+  }
+}
+
+// the exclusive scan (as affine_scan_kernel) for dk = 128: one block per (head, 32 columns)
+__global__ void __launch_bounds__(kTileThreads, 1) affine_scan128_kernel(ScanArgs a) {
+  extern __shared__ __align__(16) float smf[];
+  float* Ms0 = smf;
+  float* Ms1 = Ms0 + 128 * kLdM;
+  float* cur = Ms1 + 128 * kLdM;  // [128][kT]
+  const int h = blockIdx.x, j0 = blockIdx.y * kT, H = a.H, dv = a.dv, vf = a.v_first;
+  const size_t st = (size_t)128 * dv;
+  const int rb = threadIdx.x >> 3, c0 = (threadIdx.x & 7) * 4;
+  if (a.N > 0) stage_m(Ms0, a.M + (size_t)h * 128 * 128);
+  float4 x[4];  // this thread's part of the carried state
+#pragma unroll
+  for (int i = 0; i < 4; ++i) x[i] = load_state4(a.initial + (size_t)h * st, rb + 32 * i, j0 + c0, dv, vf);
+  for (int s = 0; s < a.N; ++s) {
+    float* Ms = (s & 1) ? Ms1 : Ms0;
+    const size_t blk = ((size_t)s * H + h) * st;
+    float4 u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = rb + 32 * i;
+      *reinterpret_cast<float4*>(cur + r * kT + c0) = x[i];
+      if (a.incoming) store_state4(a.incoming + blk, r, j0 + c0, dv, vf, x[i]);
+      u[i] = load_state4(a.U + blk, r, j0 + c0, dv, vf);
+    }
+    if (s + 1 < a.N) {
+      stage_m((s & 1) ? Ms0 : Ms1, a.M + ((size_t)(s + 1) * H + h) * 128 * 128);
+      cp_async_wait_groups<1>();
+    } else {
+      cp_async_wait_groups<0>();
+    }
+    __syncthreads();  // M_s staged, the carried tile complete
+    float acc[4][4];
+    tile_product(Ms, cur, acc);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[i] = make_float4(acc[i][0] + u[i].x, acc[i][1] + u[i].y, acc[i][2] + u[i].z, acc[i][3] + u[i].w);
+      if (a.outgoing) store_state4(a.outgoing + blk, rb + 32 * i, j0 + c0, dv, vf, x[i]);
+    }
+    __syncthreads();  // every read of cur and of M_s is done
+  }
+  if (a.final_state)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) store_state4(a.final_state + (size_t)h * st, rb + 32 * i, j0 + c0, dv, vf, x[i]);
+}
+
+// the composition (as compose_pieces_kernel) for dk = 128: one block per (head, 32 columns of
+// M or of U, segment); the first piece's map is the starting tile
+__global__ void __launch_bounds__(kTileThreads, 2) compose128_kernel(ComposeArgs a) {
+  extern __shared__ __align__(16) float smf[];
+  float* Ms = smf;
+  float* cur = Ms + 128 * kLdM;
+  const int h = blockIdx.x, seg = blockIdx.z, H = a.H, dv = a.dv, vf = a.v_first, k = a.k;
+  const int nbm = 128 / kT;
+  const bool is_m = (int)blockIdx.y < nbm;
+  const int j0 = (is_m ? (int)blockIdx.y : (int)blockIdx.y - nbm) * kT;
+  const size_t st = (size_t)128 * dv;
+  const int rb = threadIdx.x >> 3, c0 = (threadIdx.x & 7) * 4;
+  const size_t first = (size_t)seg * k;
+  float4 x[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = rb + 32 * i;
+    x[i] = is_m ? *reinterpret_cast<const float4*>(a.M + (first * H + h) * 128 * 128 + (size_t)r * 128 + j0 + c0)
+                : load_state4(a.U + (first * H + h) * st, r, j0 + c0, dv, vf);
+  }
+  for (int p = 1; p < k; ++p) {
+    const size_t piece = first + p;
+    stage_m(Ms, a.M + (piece * H + h) * 128 * 128);
+    float4 u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = rb + 32 * i;
+      *reinterpret_cast<float4*>(cur + r * kT + c0) = x[i];
+      u[i] = is_m ? make_float4(0.f, 0.f, 0.f, 0.f) : load_state4(a.U + (piece * H + h) * st, r, j0 + c0, dv, vf);
+    }
+    cp_async_wait_groups<0>();
+    __syncthreads();
+    float acc[4][4];
+    tile_product(Ms, cur, acc);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      x[i] = make_float4(acc[i][0] + u[i].x, acc[i][1] + u[i].y, acc[i][2] + u[i].z, acc[i][3] + u[i].w);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = rb + 32 * i, j = j0 + c0;
+    const size_t ob = ((size_t)seg * H + h) * st;
+    if (is_m) {
+      *reinterpret_cast<float4*>(a.M_out + ((size_t)seg * H + h) * 128 * 128 + (size_t)r * 128 + j) = x[i];
+    } else {
+      store_state4(a.U_out + ob, r, j, dv, vf, x[i]);
+      store_state4(a.incoming + ob, r, j, dv, vf, load_state4(a.inc + (first * H + h) * st, r, j, dv, vf));
+      const float* nxt = seg + 1 < a.N ? a.inc + ((size_t)(seg + 1) * k * H + h) * st : a.final_state + (size_t)h * st;
+      store_state4(a.outgoing + ob, r, j, dv, vf, load_state4(nxt, r, j, dv, vf));
+    }
+  }
+}
+
+bool tiles128(int dk, int dv) { return dk == 128 && dv % kT == 0 && dv <= 128; }
 
 }  // namespace kda

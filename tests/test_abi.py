@@ -122,3 +122,28 @@ def test_context_parallel_host_checks(lib):
     args_f32[3] = 0
     assert lib.kda_context_parallel_prefill(*args_f32, p(256), 1 << 30, None, None) == 2
     assert kda.kda_context_parallel_workspace_size(100, 4, 128) == 2 * 100 * 4 * 128 * 2
+
+
+def test_piece_calls_host_checks(lib):
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
+    assert lib.kda_context_parallel_piece_offsets(None, 2, 2, p(16), None) == 1
+    assert lib.kda_context_parallel_piece_offsets(p(16), 0, 2, p(16), None) == 1
+    assert lib.kda_context_parallel_piece_offsets(p(16), 2, 0, p(16), None) == 1
+    args = [p(16)] * 4 + [2, 2, 2, 128, 128] + [p(16)] * 4 + [0, None]
+    bad_null = list(args)
+    bad_null[0] = None
+    assert lib.kda_segment_compose(*bad_null) == 1
+    bad_pieces = list(args)
+    bad_pieces[5] = 0
+    assert lib.kda_segment_compose(*bad_pieces) == 1
+    bad_dims = list(args)
+    bad_dims[7] = 256
+    assert lib.kda_segment_compose(*bad_dims) == 2
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="the split depends on the device's SM count")
+def test_without_a_device_nothing_is_split():
+    # no CUDA device here: one piece per segment, the preferred workspace is the minimum
+    assert kda.kda_context_parallel_pieces(1 << 17, 16, 32) == 1
+    assert kda.kda_context_parallel_workspace_preferred(1 << 17, 16, 32, 128) == \
+        kda.kda_context_parallel_workspace_size(1 << 17, 32, 128)

@@ -166,3 +166,87 @@ def test_full_size_context_parallel_prefill_sampled_heads():
                                       cpu(w.state_indices))
     assert rel_l2(res["out"][:, heads], o_ref) < 1e-2
     assert rel_l2(res["final_state"][heads], p_ref[0]) < 1e-2
+
+
+# ------------------------------------------------------------------------------------------
+# Segments built as pieces: boundaries, composition, and the split prefill
+# ------------------------------------------------------------------------------------------
+
+def _piece_rule(offs, k):
+    """The documented boundaries: piece p of [s0, s1) starts at s0 + 64 floor(nch p / k)."""
+    out = []
+    for i in range(len(offs) - 1):
+        s0, s1 = offs[i], offs[i + 1]
+        nch = (s1 - s0 + 63) // 64 if s1 > s0 else 0
+        out += [min(s0 + 64 * ((nch * p) // k), s1) if s1 > s0 else s0 for p in range(k)]
+    return out + [offs[-1]]
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 8])
+def test_piece_offsets_follow_the_documented_rule(k):
+    offs = [0, 0, 1, 64, 65, 1000, 8192, 8200]
+    d = torch.tensor(offs, dtype=torch.int32, device="cuda")
+    got = kda.kda_context_parallel_piece_offsets(d, k)
+    torch.cuda.synchronize()
+    assert got.cpu().tolist() == _piece_rule(offs, k)
+
+
+@pytest.mark.parametrize("dk,dv,layout", [(128, 128, "K_FIRST"), (40, 24, "V_FIRST")])
+def test_compose_matches_oracle_composition(dk, dv, layout):
+    rng = np.random.default_rng(dk + dv)
+    N, k, H = 3, 3, 2
+    st = (dk, dv) if layout == "K_FIRST" else (dv, dk)
+    Mp = rng.normal(size=(N * k, H, dk, dk)) / np.sqrt(dk)
+    Up = rng.normal(size=(N * k, H, *st))
+    Ip = rng.normal(size=(N * k + 1, H, *st))
+    fin = rng.normal(size=(H, *st))
+    cu = lambda x: torch.tensor(x, dtype=torch.float32, device="cuda")  # noqa: E731
+    res = kda.kda_segment_compose(cu(Mp), cu(Up), cu(Ip), cu(fin), k, state_layout=layout)
+    torch.cuda.synchronize()
+    kf = (lambda u: u) if layout == "K_FIRST" else (lambda u: u.T)  # noqa: E731
+    for i in range(N):
+        for h in range(H):
+            Mc, Uc = Mp[i * k, h], kf(Up[i * k, h])
+            for p in range(1, k):
+                Mc, Uc = oracle.kda_compose((Mp[i * k + p, h], kf(Up[i * k + p, h])), (Mc, Uc))
+            assert rel_l2(res["transition_matrices"][i, h], Mc) < 1e-5
+            assert rel_l2(kf(res["local_contributions"][i, h].cpu().double().numpy()), Uc) < 1e-5
+            assert torch.equal(res["incoming_states"][i, h].cpu(), cu(Ip[i * k, h]).cpu())
+            nxt = Ip[(i + 1) * k, h] if i + 1 < N else fin[h]
+            assert torch.equal(res["outgoing_states"][i, h].cpu(), cu(nxt).cpu())
+
+
+@pytest.mark.parametrize("layout", ["K_FIRST", "V_FIRST"])
+def test_split_prefill_matches_oracle_and_unsplit(layout):
+    """4096 tokens, 2 heads, 4 segments (one of a single token): 8 chains, so every segment is
+    built as several pieces; results against the oracle and against the unsplit prefill."""
+    T, H = 4096, 2
+    w = W.random_inputs([T], H, H, 128, 128, seed=12, state_std=0.1, state_layout=layout)
+    wd = w.to("cuda")
+    offs = torch.tensor([0, 1000, 1001, 2500, T], dtype=torch.int32, device="cuda")
+    N = offs.numel() - 1
+    pieces = kda.kda_context_parallel_pieces(T, N, H)
+    assert pieces > 1
+    init = wd.state_pool[0].contiguous()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    split = kda.kda_context_parallel_prefill(wd.q, wd.k, wd.v, wd.raw_gate, wd.beta_logits, wd.a_log, wd.dt_bias,
+                                             offs, init, state_layout=layout, device_status=status)
+    ws = torch.empty(kda.kda_context_parallel_workspace_size(T, H, 128), dtype=torch.uint8, device="cuda")
+    assert ws.numel() < kda.kda_context_parallel_workspace_preferred(T, N, H, 128)
+    whole = kda.kda_context_parallel_prefill(wd.q, wd.k, wd.v, wd.raw_gate, wd.beta_logits, wd.a_log, wd.dt_bias,
+                                             offs, init, state_layout=layout, workspace=ws, device_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    o_ref, p_ref = oracle.kda_forward(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens,
+                                      w.state_pool, w.state_indices, state_layout=layout)
+    M, U = oracle.kda_segment_summary(w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, offs.cpu(),
+                                      state_layout=layout)
+    scan = oracle.kda_affine_scan(M, U, w.state_pool[0].double().numpy(), state_layout=layout)
+    for res in (split, whole):
+        assert rel_l2(res["out"], o_ref) < 1e-2
+        assert rel_l2(res["final_state"], p_ref[0]) < 1e-2
+        assert rel_l2(res["transition_matrices"], M) < 1e-2
+        assert rel_l2(res["local_contributions"], U) < 1e-2
+        assert rel_l2(res["incoming_states"], scan["incoming_states"]) < 1e-2
+        assert rel_l2(res["outgoing_states"], scan["outgoing_states"]) < 1e-2
+    assert rel_l2(split["out"], whole["out"].double().cpu().numpy()) < 1e-2
