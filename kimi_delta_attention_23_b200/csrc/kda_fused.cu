@@ -559,6 +559,31 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         }
       }
     }
+    // the inverse of this 8-row block's diagonal part, X = (I + diag(beta) A_blk)^{-1} (unit
+    // lower triangular): lane j < 8 runs the forward substitution of column j; the strictly lower
+    // part goes to the block's upper triangle of sA (never read as A), transposed
+    __syncwarp();
+    if (lane < 8) {
+      const int j = lane, base = warp * 8;
+      float lb[8][8], bb[8];  // the block's strictly lower scores and its betas, loaded up front
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        bb[r] = sBeta[base + r];
+#pragma unroll
+        for (int c = 0; c < r; ++c) lb[r][c] = sA[(base + r) * kLdA + base + c];
+      }
+      float x[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < r; ++c) acc = fmaf(lb[r][c], x[c], acc);
+        x[r] = r < j ? 0.f : (r == j ? 1.f : -bb[r] * acc);
+      }
+#pragma unroll
+      for (int r = 1; r < 8; ++r)
+        if (r > j) sA[(base + j) * kLdA + base + r] = x[r];
+    }
     fence_async_smem();  // the operand tiles are read by the tensor cores
     __syncthreads();  // (2) operand tiles, block factors and diagonal scores in place
 
@@ -634,36 +659,35 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     __syncthreads();  // (3) A and P complete
 
     // =============================== k-side, part 3: T = (I + diag(beta) A)^{-1} diag(beta)
-    // X = (I + L)^{-1}, L = diag(beta) A strictly lower.  Diagonal 16-blocks by forward
-    // substitution (four threads per column); then two doubling levels on tf32 mma.sync --
+    // X = (I + L)^{-1}, L = diag(beta) A strictly lower.  Diagonal 8-blocks by forward
+    // substitution (in the diagonal phase), 16-blocks from them in fp32; then two doubling
+    // levels on tf32 mma.sync --
     // X10 and X32 from the 16-blocks, then the lower-left 32-block from the 32-blocks -- each as
     // X_ab = -X_aa (L_ab X_bb).  T is rounded to bf16 afterwards, so tf32 products suffice.
     {
       float* Xi = reinterpret_cast<float*>(sm + OFF_XI);
       float* Yb = reinterpret_cast<float*>(sm + OFF_Y);  // per-warp 16x8 tiles, then [32][32]
       {
-        const int col = (tid >> 2) & 15, q = tid & 3, base = 16 * (tid >> 6);
-        float lrow[16][4];  // L[base + r][base + 4j + q]
+        // the 16-blocks from their 8-blocks a = 2m, b = 2m + 1 (inverted in the diagonal phase,
+        // stored transposed above the diagonal of sA): X_ba = -X_bb (L_ba X_aa); thread ->
+        // (16-block m, row i, column j) of the 8 x 8 products
+        const int m = tid >> 6, i = (tid >> 3) & 7, j = tid & 7;
+        const int ra = 16 * m, rb8 = 16 * m + 8;
+        auto xblk = [&](int base, int r, int c) {  // unit lower triangular 8-block inverse
+          return r == c ? 1.f : (c < r ? sA[(base + c) * kLdA + base + r] : 0.f);
+        };
+        float y = 0.f;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          const float br = sBeta[base + r];
+        for (int l = 0; l < 8; ++l) y = fmaf(sA[(rb8 + i) * kLdA + ra + l], xblk(ra, l, j), y);
+        Yb[tid] = sBeta[rb8 + i] * y;  // (L_ba X_aa)[i][j]
+        __syncthreads();
+        float xv = 0.f;
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) lrow[r][jj] = br * sA[(base + r) * kLdA + base + 4 * jj + q];
-        }
-        float xq[4] = {0.f, 0.f, 0.f, 0.f};  // x[4 jj + q]: the entries this thread sums over
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          float part = 0.f;
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj)
-            if (4 * jj + q < r) part += lrow[r][jj] * xq[jj];
-          part += __shfl_xor_sync(0xffffffffu, part, 1);
-          part += __shfl_xor_sync(0xffffffffu, part, 2);
-          const float xr = (r == col) ? 1.f : (r < col ? 0.f : -part);
-          if ((r & 3) == q) xq[r >> 2] = xr;
-        }
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) Xi[(base + 4 * jj + q) * kLdA + base + col] = xq[jj];
+        for (int l = 0; l < 8; ++l) xv = fmaf(xblk(rb8, i, l), Yb[m * 64 + l * 8 + j], xv);
+        Xi[(rb8 + i) * kLdA + ra + j] = -xv;
+        Xi[(ra + i) * kLdA + ra + j] = xblk(ra, i, j);
+        Xi[(rb8 + i) * kLdA + rb8 + j] = xblk(rb8, i, j);
+        Xi[(ra + i) * kLdA + rb8 + j] = 0.f;
       }
       __syncthreads();
       const int g = lane >> 2, t = lane & 3;
@@ -913,9 +937,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           tmem_wait_ld();
           if (a.out_bf16) {
 #pragma unroll
-            for (int u = 0; u < 32; ++u)
-              *reinterpret_cast<__nv_bfloat16*>(sm + OFF_S + ((32 * ehalf + u) * D + ej) * 2) =
-                  __float2bfloat16_rn(d[u]);
+            for (int u = 0; u < 32; u += 2) {  // one conversion per row pair, two 16-bit stores
+              const uint32_t pk = pack_bf16(d[u], d[u + 1]);
+              *reinterpret_cast<uint16_t*>(sm + OFF_S + ((32 * ehalf + u) * D + ej) * 2) = (uint16_t)(pk & 0xffffu);
+              *reinterpret_cast<uint16_t*>(sm + OFF_S + ((32 * ehalf + u + 1) * D + ej) * 2) = (uint16_t)(pk >> 16);
+            }
           } else {
 #pragma unroll
             for (int u = 0; u < 32; ++u) reinterpret_cast<float*>(sm + OFF_KQ)[(32 * ehalf + u) * D + ej] = d[u];
@@ -1128,8 +1154,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
             tmem_wait_ld();
             uint8_t* stage = sm + OFF_KQ + st * 16384;
 #pragma unroll
-            for (int u = 0; u < 32; ++u)
-              *reinterpret_cast<__nv_bfloat16*>(stage + ((32 * ehalf + u) * D + ej) * 2) = __float2bfloat16_rn(d[u]);
+            for (int u = 0; u < 32; u += 2) {  // one conversion per row pair, two 16-bit stores
+              const uint32_t pk = pack_bf16(d[u], d[u + 1]);
+              *reinterpret_cast<uint16_t*>(stage + ((32 * ehalf + u) * D + ej) * 2) = (uint16_t)(pk & 0xffffu);
+              *reinterpret_cast<uint16_t*>(stage + ((32 * ehalf + u + 1) * D + ej) * 2) = (uint16_t)(pk >> 16);
+            }
           }
         }
       }
