@@ -516,11 +516,20 @@ def cpu_baseline(w, args):
 
 
 def profile_launches(args):
-    """Plain launches of the prefill kernel on one workload, nothing else (a target for ncu)."""
+    """Plain launches of one workload's step, nothing else (a target for ncu): the prefill kernel,
+    or for a context-parallel workload the step's calls (build over the pieces, scan, composition,
+    apply)."""
     import kimi_delta_attention_23_b200 as kda
     from kimi_delta_attention_23_b200 import build as kbuild
     kbuild.build()
     w = W.make(args.workload, device="cuda")
+    if w.seg_offsets is not None:
+        step = Step(w, torch.cuda.current_stream())
+        for _ in range(args.profile_launches):
+            step()
+        torch.cuda.synchronize()
+        print("launched", args.profile_launches, "context-parallel steps; pieces per segment", step.pieces)
+        return 0
     for _ in range(args.profile_launches):
         pool = w.state_pool.clone()
         kda.kda_chunk_fwd(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens, pool,

@@ -147,6 +147,7 @@ WORKLOADS = (
     "long_T131072_H32_cp16",
     "batch64_T2048_H16_safe",
     "batch4_T2048_H32",  # one wave of 128 chains, inputs 404 MB (> L2): the profiling case
+    "long_T16384_H32_cp2",  # context-parallel profiling case: 2 segments of 8192, inputs 420 MB
 )
 
 
@@ -175,6 +176,9 @@ def make(name: str, device="cpu", seed: Optional[int] = None) -> Workload:
                           device=device, name=name)
     elif name == "batch4_T2048_H32":
         w = random_inputs([2048] * 4, 32, 32, 128, 128, seed=s, state_std=0.1, device=device, name=name)
+    elif name == "long_T16384_H32_cp2":
+        w = random_inputs([16384], 32, 32, 128, 128, seed=s, state_std=0.1, device=device, name=name)
+        w.seg_offsets = (torch.arange(3, dtype=torch.int32) * 8192).to(device)
     else:  # pragma: no cover
         raise KeyError(name)
     return w
