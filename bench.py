@@ -304,6 +304,12 @@ class Step:
                     self.pU = torch.empty((P, Hv, *st), device=dev)
                     self.pIn = torch.empty((P + 1, Hv, *st), device=dev)  # slot p + 1: outgoing of piece p
         self.pool = None if self.cp else w.state_pool.clone()
+        if not self.cp:
+            # the prefill's optional workspace: with it, a batch of few or uneven sequences may
+            # take the split route (decided on the device by the library's planner)
+            Hk = w.k.shape[1]
+            need = kda.kda_workspace_size(T, w.batch, Hk, Hv, dk, dv) if w.q.dtype == torch.bfloat16 else 0
+            self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
         self.events = []
 
     def kw(self):
@@ -313,7 +319,8 @@ class Step:
 
     def launches(self):
         if not self.cp:
-            return 1
+            # split route: planner, plain kernel (gated), build, pool scan, apply; else one kernel
+            return 5 if self.ws.numel() > 0 else 1
         # (piece boundaries,) segment build with readouts, scan, (composition,) apply
         return 5 if self.pieces > 1 else 3
 
@@ -361,7 +368,7 @@ class Step:
                 ev[1].record(self.stream)
                 ev[2].record(self.stream)
             kda.kda_chunk_fwd(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens,
-                              self.pool, w.state_indices, self.out, **self.kw())
+                              self.pool, w.state_indices, self.out, workspace=self.ws, **self.kw())
         if ev:
             ev[3].record(self.stream)
             self.events.append(ev)
@@ -432,7 +439,9 @@ def run_ours(args):
         breakdown = {"segment_build_and_scan": ms_seg, "compose_pieces": statistics.mean(comp_ms),
                      "context_parallel_apply": ms_pass}
     else:
-        dom, bytes_dom, ms_dom = "fused_chunk_kernel<prefill>", chunk_fwd_bytes(w, w.batch), ms_pass
+        dom = "fused_chunk_kernel<prefill>" if step.ws.numel() == 0 else \
+            "kda_chunk_fwd (planner; pieces: build with readouts, pool scan, apply; or the prefill kernel)"
+        bytes_dom, ms_dom = chunk_fwd_bytes(w, w.batch), ms_pass
         breakdown = {"chunk_fwd": ms_pass}
     achieved = bytes_dom / (ms_dom / 1e3) / 1e9
     roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",

@@ -101,7 +101,17 @@ enum {
  *   state_indices [batch]                           int32 pool slot of each sequence
  *   out           [total_tokens, num_v_heads, dv]   out_dtype; rows outside every sequence untouched
  *   gate_lower_bound                                used only with KDA_GATE_SAFE
- *   workspace     unused by the current kernels (kda_workspace_size() returns 0); may be NULL
+ *   workspace     optional device scratch, 256-byte aligned.  With at least kda_workspace_size()
+ *                 bytes, a bf16 batch of few or uneven sequences (fewer than three chains, i.e.
+ *                 sequence-heads, per SM) may take the split route: every sequence is cut into
+ *                 chunk-aligned pieces, the pieces are built in parallel (transition,
+ *                 contribution and readouts, as in the context-parallel prefill), applied in order
+ *                 from the sequence's pool slot, and the outputs formed from the readouts
+ *                 ("KDA Context Parallelism": any cut is a segment boundary).  A planner kernel
+ *                 on the device keeps the plain route when, with the real lengths, the pieces would
+ *                 not shorten the schedule, or when an offset or a slot is bad (the plain route
+ *                 then reports it as usual).  Results agree with the plain route up to rounding.
+ *                 NULL or a smaller workspace: the plain route.
  *
  * Supported groupings: (qkv F32, out F32) for any 1 <= dk, dv <= 128 on the fp32 CUDA-core
  * kernel; (qkv BF16, out BF16 or F32) with dk = dv = 128 on the fused tensor-core kernel, or on
@@ -269,8 +279,10 @@ KDA_API kda_status_t kda_context_parallel_piece_offsets(const int32_t *seg_offse
 KDA_API size_t kda_context_parallel_workspace_preferred(int64_t T, int32_t num_segments,
                                                         int32_t num_v_heads, int32_t dv);
 
-/* Bytes of workspace kda_chunk_fwd / kda_segment_summarize_and_scan need for these extents
- * (0 for the current kernels). */
+/* Bytes of workspace with which kda_chunk_fwd may take its split route on the current device
+ * (0 when the batch has chains enough for the SMs, for dk or dv other than 128, or with
+ * KDA_FORCE_SIMT; the workspace is optional either way).  kda_segment_summarize_and_scan needs
+ * none.  num_segments is unused. */
 KDA_API size_t kda_workspace_size(int64_t total_tokens, int32_t batch, int32_t num_k_heads,
                           int32_t num_v_heads, int32_t dk, int32_t dv, int32_t num_segments,
                           uint32_t flags);

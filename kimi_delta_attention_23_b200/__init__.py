@@ -148,13 +148,15 @@ def _stream(stream, device):
 def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, state_pool, state_indices,
                   out=None, *, output_dtype=None, use_computebound=False, gate_mode="original",
                   beta_mode="logits", state_layout="K_FIRST", gate_lower_bound=-5.0, force_simt=False,
-                  device_status=None, stream=None):
+                  workspace=None, device_status=None, stream=None):
     """Chunk-parallel KDA prefill (``max.nn.state_space.kda_chunk`` semantics).
 
     Shapes: q,k [T,Hk,dk]; v [T,Hv,dv]; raw_gate [T,Hv,dk] f32; beta_logits [T,Hv] f32;
     a_log [Hv] f32; dt_bias [Hv,dk] f32; cu_seqlens [B+1] i32; state_pool [slots,Hv,dk,dv]
     (K_FIRST) or [slots,Hv,dv,dk] (V_FIRST) f32, mutated in place; state_indices [B] i32.
-    Returns out [T,Hv,dv] in ``output_dtype`` (default: the dtype of v).
+    Returns out [T,Hv,dv] in ``output_dtype`` (default: the dtype of v).  ``workspace`` (uint8
+    CUDA tensor) enables the split route for batches of few or uneven sequences; it is
+    allocated at kda_workspace_size bytes when not given (pass an empty tensor to disable).
     """
     lib = load_library()
     dev = q.device
@@ -189,10 +191,18 @@ def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, st
     if device_status is not None:
         _shape(_dev(device_status, "device_status", torch.int32, dev), "device_status", (1,))
     flags = _flags(gate_mode, beta_mode, state_layout, use_computebound, force_simt)
+    if workspace is None:
+        need = 0
+        if q.dtype == torch.bfloat16 and not force_simt:
+            with torch.cuda.device(dev):
+                need = kda_workspace_size(T, B, Hk, Hv, dk, dv, 0, flags)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _dev(workspace, "workspace", torch.uint8, dev)
     rc = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], _ptr(raw_gate), _ptr(beta_logits),
                            _ptr(a_log), _ptr(dt_bias), _ptr(cu_seqlens), B, T, Hk, Hv, dk, dv,
                            _ptr(state_pool), state_pool.shape[0], _ptr(state_indices), _ptr(out),
-                           _DTYPES[output_dtype], flags, float(gate_lower_bound), None, 0,
+                           _DTYPES[output_dtype], flags, float(gate_lower_bound),
+                           _ptr(workspace) if workspace.numel() else None, workspace.numel(),
                            _ptr(device_status), _stream(stream, dev))
     if rc != 0:
         raise KdaError(rc, "kda_chunk_fwd")

@@ -57,6 +57,50 @@ size_t pieces_bytes(int32_t N, int k, int32_t Hv, int32_t dk, int32_t dv) {
          np * Hv * (size_t)dk * dv * sizeof(float) + (np + 1) * Hv * (size_t)dk * dv * sizeof(float);
 }
 
+int sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return sms;
+}
+
+// Piece length (tokens, a multiple of 64) for the split route of kda_chunk_fwd, or 0 when the
+// batch has chains (sequence-heads) enough for the SMs -- more than half as many as SMs -- and
+// runs as it is.  Estimated time in chunk steps for piece length P, with sequences of the mean
+// length: rounds of chains on the SMs (one chain per SM) times P / 64, plus 0.35 chunk steps
+// for every piece the scan applies in order.  The planner on the device still keeps the plain
+// route when, with the real lengths, the pieces would not pay.
+int choose_piece_len(int64_t T, int32_t batch, int32_t Hv) {
+  const int sms = sm_count();
+  if (sms <= 0 || T <= 0 || batch <= 0 || 2 * (int64_t)batch * Hv > (int64_t)sms) return 0;
+  const int64_t mean = (T + batch - 1) / batch;
+  const int64_t top = ((mean + 63) / 64) * 64;
+  int best_p = 0;
+  double best = 0.0;
+  for (int64_t P = 256; P <= top && P <= ((int64_t)1 << 30); P += (P < 4096 ? 64 : P / 16 / 64 * 64)) {
+    const int64_t per_seq = (mean + P - 1) / P;
+    const int64_t chains = (int64_t)batch * per_seq * Hv;
+    const double est = (double)((chains + sms - 1) / sms) * (double)(P / 64) + 0.35 * (double)per_seq;
+    if (best_p == 0 || est < best) {
+      best = est;
+      best_p = (int)P;
+    }
+  }
+  return best_p;
+}
+
+int32_t max_pieces_of(int64_t T, int32_t batch, int P) { return batch + (int32_t)((T + P - 1) / P); }
+
+// workspace of the split route: readouts, the pieces' transitions, contributions and incoming
+// states, piece boundaries, first piece per sequence, the fallback flag
+size_t split_bytes(int64_t T, int32_t batch, int32_t Hv, int P) {
+  const size_t np = (size_t)max_pieces_of(T, batch, P);
+  const size_t blk = (size_t)Hv * 128 * 128 * sizeof(float);
+  return round256((size_t)2 * T * Hv * 128 * 2) + 3 * np * blk + round256((np + 1) * sizeof(int32_t)) +
+         round256(((size_t)batch + 1) * sizeof(int32_t)) + 256;
+}
+
 }  // namespace
 
 extern "C" kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,
@@ -146,7 +190,94 @@ extern "C" kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* 
   f.flags = flags;
   f.lb = gate_lower_bound;
   f.status = device_status;
-  return kda::launch_fused_chunk(f, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  const int P = choose_piece_len(total_tokens, batch, num_v_heads);
+  if (P == 0 || !workspace || workspace_bytes < split_bytes(total_tokens, batch, num_v_heads, P) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return kda::launch_fused_chunk(f, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+
+  // Split route: sequences cut into pieces of at most P tokens, the pieces built in parallel
+  // (transition, contribution, readouts), applied in order from each sequence's pool slot, then
+  // the outputs formed from the readouts.  A planner kernel lays the pieces out and, if an
+  // offset or a slot is bad or the pieces would not shorten the schedule, sets the fallback
+  // flag: then only the plain launch runs.
+  const int32_t np = max_pieces_of(total_tokens, batch, P);
+  const size_t blk = (size_t)num_v_heads * 128 * 128;
+  uint8_t* w = reinterpret_cast<uint8_t*>(workspace);
+  __nv_bfloat16_raw* o_m = reinterpret_cast<__nv_bfloat16_raw*>(w);
+  __nv_bfloat16_raw* o_u = o_m + (size_t)total_tokens * num_v_heads * 128;
+  w += round256((size_t)2 * total_tokens * num_v_heads * 128 * 2);
+  float* pM = reinterpret_cast<float*>(w);
+  float* pU = pM + (size_t)np * blk;
+  float* pIn = pU + (size_t)np * blk;
+  w += 3 * (size_t)np * blk * sizeof(float);
+  int32_t* piece_offs = reinterpret_cast<int32_t*>(w);
+  w += round256(((size_t)np + 1) * sizeof(int32_t));
+  int32_t* seq_first = reinterpret_cast<int32_t*>(w);
+  w += round256(((size_t)batch + 1) * sizeof(int32_t));
+  int32_t* fallback = reinterpret_cast<int32_t*>(w);
+
+  kda::PlanArgs pa{};
+  pa.cu = cu_seqlens;
+  pa.slots = state_indices;
+  pa.batch = batch;
+  pa.total_tokens = total_tokens;
+  pa.max_slots = max_slots;
+  pa.piece_len = P;
+  pa.max_pieces = np;
+  pa.num_heads = num_v_heads;
+  pa.num_sms = sm_count();
+  pa.piece_offs = piece_offs;
+  pa.seq_first = seq_first;
+  pa.fallback = fallback;
+  if (kda::launch_plan_pieces(pa, s) != cudaSuccess) return KDA_ERR_CUDA;
+  // plain route (runs only on fallback)
+  f.gate_flag = fallback;
+  f.gate_run_if = 1;
+  if (kda::launch_fused_chunk(f, s) != cudaSuccess) return KDA_ERR_CUDA;
+  // the pieces: both states and both readouts in one launch
+  kda::FusedArgs bf = f;
+  bf.cu = piece_offs;
+  bf.batch = np;
+  bf.state_in = nullptr;
+  bf.max_slots = np;
+  bf.slots = nullptr;
+  bf.init_mode = 0;
+  bf.values_zero = 0;
+  bf.build = 1;
+  bf.state_out = pM;
+  bf.state_out2 = pU;
+  bf.out = o_m;
+  bf.out2 = o_u;
+  bf.out_bf16 = 1;
+  bf.gate_run_if = 0;
+  if (kda::launch_fused_chunk(bf, s) != cudaSuccess) return KDA_ERR_CUDA;
+  kda::PoolScanArgs ps{};
+  ps.M = pM;
+  ps.U = pU;
+  ps.seq_first = seq_first;
+  ps.slots = state_indices;
+  ps.fallback = fallback;
+  ps.batch = batch;
+  ps.H = num_v_heads;
+  ps.dv = 128;
+  ps.v_first = f.v_first;
+  ps.pool = state_pool;
+  ps.incoming = pIn;
+  if (kda::launch_pool_scan(ps, s) != cudaSuccess) return KDA_ERR_CUDA;
+  kda::ApplyArgs ap{};
+  ap.seg_offsets = piece_offs;
+  ap.num_segments = np;
+  ap.total_tokens = total_tokens;
+  ap.Hv = num_v_heads;
+  ap.incoming = pIn;
+  ap.v_first = f.v_first;
+  ap.o_m = o_m;
+  ap.o_u = o_u;
+  ap.out = out;
+  ap.out_bf16 = out_dtype == KDA_BF16;
+  ap.status = device_status;
+  ap.skip_flag = fallback;
+  return kda::launch_cp_apply(ap, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 extern "C" kda_status_t kda_segment_summarize_and_scan(
@@ -405,15 +536,13 @@ extern "C" kda_status_t kda_context_parallel_prefill(
 extern "C" size_t kda_workspace_size(int64_t total_tokens, int32_t batch, int32_t num_k_heads,
                                      int32_t num_v_heads, int32_t dk, int32_t dv, int32_t num_segments,
                                      uint32_t flags) {
-  (void)total_tokens;
-  (void)batch;
   (void)num_k_heads;
-  (void)num_v_heads;
-  (void)dk;
-  (void)dv;
   (void)num_segments;
-  (void)flags;
-  return 0;
+  // the split route of kda_chunk_fwd (bf16 fast path only; unused otherwise)
+  if (dk != 128 || dv != 128 || (flags & KDA_FORCE_SIMT) || total_tokens < 0 || batch <= 0 || num_v_heads <= 0)
+    return 0;
+  const int P = choose_piece_len(total_tokens, batch, num_v_heads);
+  return P > 0 ? split_bytes(total_tokens, batch, num_v_heads, P) : 0;
 }
 
 extern "C" const char* kda_status_string(kda_status_t status) {

@@ -43,6 +43,7 @@ struct TilePos {
 };
 
 __global__ void __launch_bounds__(kThreads, 2) cp_apply_kernel(ApplyArgs a) {
+  if (a.skip_flag && *a.skip_flag) return;
   extern __shared__ __align__(16) uint8_t smem[];
   __nv_bfloat16* sB = reinterpret_cast<__nv_bfloat16*>(smem);  // [j][j'] = S_in[j'][j]
   __nv_bfloat16* sM = sB + D * kLd;                              // 2 x [r][j'] readout through M

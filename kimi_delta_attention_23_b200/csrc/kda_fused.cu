@@ -125,6 +125,7 @@ struct InputMaps {
 // in prefill; in the build, the readouts of both states (local outputs of the segment).
 template <bool kBuild, bool kRead>
 __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArgs a, const __grid_constant__ InputMaps tm) {
+  if (a.gate_flag && *a.gate_flag != a.gate_run_if) return;  // this launch is not the one that runs
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;

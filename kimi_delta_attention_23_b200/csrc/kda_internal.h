@@ -77,6 +77,9 @@ struct FusedArgs {
   uint32_t flags;
   float lb;
   int32_t* status;
+  // launch gate (nullable): the kernel runs only if *gate_flag == gate_run_if
+  const int32_t* gate_flag;
+  int32_t gate_run_if;
 };
 
 // Context-parallel prefill, last step: out = O_M . S_in(segment) + O_U.
@@ -92,6 +95,39 @@ struct ApplyArgs {
   void* out;                   // [T][Hv][128]
   int32_t out_bf16;
   int32_t* status;
+  const int32_t* skip_flag;  // nullable: the kernel does nothing if *skip_flag != 0
+};
+
+// A varlen batch cut into pieces of at most piece_len tokens (chunk-aligned, at least one per
+// sequence): piece boundaries and each sequence's first piece, or the fallback flag (1) when an
+// offset or a slot is out of range or the pieces would not shorten the schedule (the plain
+// kernel then handles the batch).
+struct PlanArgs {
+  const int32_t* cu;
+  const int32_t* slots;  // nullable: sequence b uses slot b
+  int32_t batch;
+  int64_t total_tokens;
+  int32_t max_slots;
+  int32_t piece_len;
+  int32_t max_pieces;
+  int32_t num_heads;     // value heads (chains per piece)
+  int32_t num_sms;       // SMs of the device (one chain each at a time)
+  int32_t* piece_offs;   // [max_pieces + 1]
+  int32_t* seq_first;    // [batch + 1]
+  int32_t* fallback;     // [1]
+};
+
+// The pieces' summaries applied in order from each sequence's pool slot (dk = 128): the
+// incoming state of every piece, and the final state written back to the slot.
+struct PoolScanArgs {
+  const float* M;        // [pieces][H][128][128]
+  const float* U;        // [pieces][H][state]
+  const int32_t* seq_first;
+  const int32_t* slots;  // nullable
+  const int32_t* fallback;
+  int32_t batch, H, dv, v_first;
+  float* pool;           // [slots][H][state]
+  float* incoming;       // [pieces][H][state]
 };
 
 // Summaries of segments split into k pieces each, rebuilt from the pieces' summaries.
@@ -110,6 +146,8 @@ struct ComposeArgs {
 size_t simt_smem_bytes(int dk, int w);
 cudaError_t launch_split_offsets(const int32_t* offs, int32_t N, int32_t k, int32_t* sub, cudaStream_t stream);
 cudaError_t launch_compose_pieces(const ComposeArgs& a, cudaStream_t stream);
+cudaError_t launch_plan_pieces(const PlanArgs& a, cudaStream_t stream);
+cudaError_t launch_pool_scan(const PoolScanArgs& a, cudaStream_t stream);
 cudaError_t launch_cp_apply(const ApplyArgs& a, cudaStream_t stream);
 cudaError_t launch_simt_chunk(const SimtArgs& a, cudaStream_t stream);
 cudaError_t launch_affine_scan(const ScanArgs& a, cudaStream_t stream);

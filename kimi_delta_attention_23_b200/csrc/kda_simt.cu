@@ -562,4 +562,164 @@ __global__ void __launch_bounds__(kTileThreads, 2) compose128_kernel(ComposeArgs
 
 bool tiles128(int dk, int dv) { return dk == 128 && dv % kT == 0 && dv <= 128; }
 
+// ------------------------------------------------------------------------------------------
+// A varlen batch as pieces: every sequence cut into chunk-aligned pieces of at most piece_len
+// tokens (an empty sequence keeps one empty piece), so that a prefill of few or uneven
+// sequences has as many chains as the SMs need; the pieces are built, applied in order from
+// each sequence's pool slot, and read out ("KDA Context Parallelism": any cut is a segment
+// boundary).
+// ------------------------------------------------------------------------------------------
+constexpr int kPlanThreads = 1024;
+
+__global__ void __launch_bounds__(kPlanThreads) plan_pieces_kernel(PlanArgs a) {
+  __shared__ int s_bad;
+  __shared__ int s_carry;
+  __shared__ int s_warp[kPlanThreads / 32];
+  __shared__ unsigned long long s_chunks;
+  __shared__ int s_max_chunks;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  if (tid == 0) {
+    s_bad = 0;
+    s_carry = 0;
+    s_chunks = 0;
+    s_max_chunks = 0;
+  }
+  __syncthreads();
+  for (int b = tid; b < a.batch; b += kPlanThreads) {
+    const int64_t t0 = a.cu[b], t1 = a.cu[b + 1];
+    const int32_t slot = a.slots ? a.slots[b] : b;
+    if (t0 < 0 || t1 < t0 || t1 > a.total_tokens || slot < 0 || slot >= a.max_slots) {
+      s_bad = 1;
+    } else {
+      const int nch = (int)((t1 - t0 + 63) / 64);
+      atomicAdd(&s_chunks, (unsigned long long)nch);
+      atomicMax(&s_max_chunks, nch);
+    }
+  }
+  __syncthreads();
+  // chunk steps on the SMs (one chain per SM): the plain schedule cannot beat its longest
+  // sequence nor the total work; the pieces are no longer than piece_len, but a piece's chunk
+  // carries two states and two readouts (taken as 1.25 chunk steps) and the scan and the apply
+  // add about 12 chunk steps
+  const double work = (double)s_chunks * a.num_heads / a.num_sms;
+  const double plain = fmax((double)s_max_chunks, work);
+  const double split = 1.25 * fmax((double)(a.piece_len / 64), work) + 12.0;
+  if (s_bad || !(split < 0.9 * plain)) {  // the plain kernel runs instead (and reports what is wrong)
+    if (tid == 0) *a.fallback = 1;
+    return;
+  }
+  const int P = a.piece_len;
+  for (int base = 0; base < a.batch; base += kPlanThreads) {
+    const int b = base + tid;
+    int n = 0;
+    int64_t t0 = 0, len = 0;
+    if (b < a.batch) {
+      t0 = a.cu[b];
+      len = a.cu[b + 1] - t0;
+      n = len > 0 ? (int)((len + P - 1) / P) : 1;
+    }
+    // inclusive block scan of n
+    int x = n;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, d);
+      if (lane >= d) x += y;
+    }
+    if (lane == 31) s_warp[w] = x;
+    __syncthreads();
+    if (w == 0) {
+      int v = s_warp[lane];
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, v, d);
+        if (lane >= d) v += y;
+      }
+      s_warp[lane] = v;
+    }
+    __syncthreads();
+    const int incl = x + (w > 0 ? s_warp[w - 1] : 0);
+    const int first = s_carry + incl - n;
+    if (b < a.batch) {
+      a.seq_first[b] = first;
+      for (int j = 0; j < n && first + j < a.max_pieces; ++j) a.piece_offs[first + j] = (int32_t)(t0 + (int64_t)j * P);
+    }
+    __syncthreads();
+    if (tid == kPlanThreads - 1) s_carry += incl;
+    __syncthreads();
+  }
+  const int total = s_carry;
+  if (total > a.max_pieces) {  // cannot happen for max_pieces >= batch + ceil(total_tokens / piece_len)
+    if (tid == 0) *a.fallback = 1;
+    return;
+  }
+  if (tid == 0) {
+    a.seq_first[a.batch] = total;
+    *a.fallback = 0;
+  }
+  const int32_t end = a.batch > 0 ? a.cu[a.batch] : 0;
+  for (int i = total + tid; i <= a.max_pieces; i += kPlanThreads) a.piece_offs[i] = end;
+}
+
+cudaError_t launch_plan_pieces(const PlanArgs& a, cudaStream_t stream) {
+  plan_pieces_kernel<<<1, kPlanThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+// one block per (head, 32 columns, sequence): the sequence's pieces applied in order to its
+// pool state, each piece's incoming state recorded, the final state written back
+__global__ void __launch_bounds__(kTileThreads, 1) pool_scan128_kernel(PoolScanArgs a) {
+  if (*a.fallback) return;
+  extern __shared__ __align__(16) float smf[];
+  float* Ms0 = smf;
+  float* Ms1 = Ms0 + 128 * kLdM;
+  float* cur = Ms1 + 128 * kLdM;
+  const int h = blockIdx.x, j0 = blockIdx.y * kT, b = blockIdx.z, H = a.H, dv = a.dv, vf = a.v_first;
+  const size_t st = (size_t)128 * dv;
+  const int rb = threadIdx.x >> 3, c0 = (threadIdx.x & 7) * 4;
+  const int p0 = a.seq_first[b], p1 = a.seq_first[b + 1];
+  const int32_t slot = a.slots ? a.slots[b] : b;
+  float* blk = a.pool + ((size_t)slot * H + h) * st;
+  if (p1 > p0) stage_m(Ms0, a.M + ((size_t)p0 * H + h) * 128 * 128);
+  float4 x[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) x[i] = load_state4(blk, rb + 32 * i, j0 + c0, dv, vf);
+  for (int p = p0; p < p1; ++p) {
+    const int s = p - p0;
+    float* Ms = (s & 1) ? Ms1 : Ms0;
+    const size_t pb = ((size_t)p * H + h) * st;
+    float4 u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = rb + 32 * i;
+      *reinterpret_cast<float4*>(cur + r * kT + c0) = x[i];
+      store_state4(a.incoming + pb, r, j0 + c0, dv, vf, x[i]);
+      u[i] = load_state4(a.U + pb, r, j0 + c0, dv, vf);
+    }
+    if (p + 1 < p1) {
+      stage_m((s & 1) ? Ms0 : Ms1, a.M + ((size_t)(p + 1) * H + h) * 128 * 128);
+      cp_async_wait_groups<1>();
+    } else {
+      cp_async_wait_groups<0>();
+    }
+    __syncthreads();
+    float acc[4][4];
+    tile_product(Ms, cur, acc);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      x[i] = make_float4(acc[i][0] + u[i].x, acc[i][1] + u[i].y, acc[i][2] + u[i].z, acc[i][3] + u[i].w);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) store_state4(blk, rb + 32 * i, j0 + c0, dv, vf, x[i]);
+}
+
+cudaError_t launch_pool_scan(const PoolScanArgs& a, cudaStream_t stream) {
+  const int smem = (2 * 128 * kLdM + 128 * kT) * (int)sizeof(float);
+  cudaError_t err = cudaFuncSetAttribute(pool_scan128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  if (a.batch == 0) return cudaSuccess;
+  pool_scan128_kernel<<<dim3(a.H, a.dv / kT, a.batch), kTileThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
 }  // namespace kda
