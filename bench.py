@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 import kda_workloads as W  # noqa: E402
 
 METRIC = "KDA prefill tokens/s (H=32,dk=dv=128,bf16) and % of roofline on 1 B200"
+DECODE_METRIC = "KDA decode tokens/s (one token per sequence, dk=dv=128) and % of roofline on 1 B200"
 DEFAULT_WORKLOAD = "long_T131072_H32_cp16"
 
 
@@ -55,6 +56,16 @@ def chunk_fwd_bytes(w, num_seqs, dk=128, dv=128):
     qkv = 2 if w.q.dtype == torch.bfloat16 else 4
     ob = 2 if w.output_dtype == torch.bfloat16 else 4
     return th * io_bytes_per_token_head(qkv, ob, dk, dv, group) + num_seqs * w.num_v_heads * 2 * dk * dv * 4
+
+
+def decode_bytes(w):
+    """One token per (sequence, head): the state block read and written once, plus the token's
+    q, k, v, gate, beta and output."""
+    group = w.num_v_heads // w.num_k_heads
+    qkv = 2 if w.q.dtype == torch.bfloat16 else 4
+    ob = 2 if w.output_dtype == torch.bfloat16 else 4
+    th = w.batch * w.num_v_heads
+    return th * (io_bytes_per_token_head(qkv, ob, w.dk, w.dv, group) + 2 * w.dk * w.dv * 4)
 
 
 def segment_build_bytes(w, N, dk=128, dv=128):
@@ -219,10 +230,13 @@ def oracle_time_sample(w, n_tokens):
     cu_s = [c for c in cu if c < n] + [n]
     B = len(cu_s) - 1
     cpu = lambda t: t.detach().cpu()  # noqa: E731
+    # only the slots the sampled sequences name (the oracle touches no other slot)
+    idx = cpu(w.state_indices)[:B].long()
+    pool = cpu(w.state_pool)[idx]
     t0 = time.perf_counter()
     oracle.kda_forward(cpu(w.q)[:n], cpu(w.k)[:n], cpu(w.v)[:n], cpu(w.raw_gate)[:n], cpu(w.beta_logits)[:n],
                        cpu(w.a_log), cpu(w.dt_bias), torch.tensor(cu_s, dtype=torch.int32),
-                       cpu(w.state_pool), cpu(w.state_indices)[:B], gate_mode=w.gate_mode, beta_mode=w.beta_mode,
+                       pool, torch.arange(B, dtype=torch.int32), gate_mode=w.gate_mode, beta_mode=w.beta_mode,
                        state_layout=w.state_layout, gate_lower_bound=w.gate_lower_bound)
     return time.perf_counter() - t0, n
 
@@ -249,7 +263,8 @@ def run_reference(args):
     times = [oracle_time_sample(w, n)[0] for _ in range(args.steps)]
     total = sum(times)
     value = n * args.steps / total
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+    line = {"impl": "reference", "metric": DECODE_METRIC if w.notes.get("decode") else METRIC, "value": value,
+            "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": args.workload, "tokens_per_step": n,
@@ -273,6 +288,7 @@ class Step:
         self.kda, self.w, self.stream, self.public = kda, w, stream, public
         dev = w.q.device
         self.cp = w.seg_offsets is not None
+        self.decode = bool(w.notes.get("decode"))
         T, Hv, dv, dk = w.total_tokens, w.num_v_heads, w.dv, w.dk
         self.out = torch.empty((T, Hv, dv), dtype=w.output_dtype, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -304,7 +320,9 @@ class Step:
                     self.pU = torch.empty((P, Hv, *st), device=dev)
                     self.pIn = torch.empty((P + 1, Hv, *st), device=dev)  # slot p + 1: outgoing of piece p
         self.pool = None if self.cp else w.state_pool.clone()
-        if not self.cp:
+        if self.decode:
+            self.ws = torch.empty(0, dtype=torch.uint8, device=dev)
+        elif not self.cp:
             # the prefill's optional workspace: with it, a batch of few or uneven sequences may
             # take the split route (decided on the device by the library's planner)
             Hk = w.k.shape[1]
@@ -318,6 +336,8 @@ class Step:
                     gate_lower_bound=w.gate_lower_bound, device_status=self.status, stream=self.stream)
 
     def launches(self):
+        if self.decode:
+            return 1
         if not self.cp:
             # split route: planner, plain kernel (gated), build, pool scan, apply; else one kernel
             return 5 if self.ws.numel() > 0 else 1
@@ -363,6 +383,12 @@ class Step:
             kda.kda_context_parallel_apply(self.rm, self.ru, self.inc, w.seg_offsets, self.out,
                                            state_layout=w.state_layout, device_status=self.status,
                                            stream=self.stream)
+        elif self.decode:
+            if ev:
+                ev[1].record(self.stream)
+                ev[2].record(self.stream)
+            kda.kda_decode(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, self.pool,
+                           w.state_indices, self.out, **self.kw())
         else:
             if ev:
                 ev[1].record(self.stream)
@@ -438,6 +464,9 @@ def run_ours(args):
             segment_build_bytes(w, step.P), ms_seg
         breakdown = {"segment_build_and_scan": ms_seg, "compose_pieces": statistics.mean(comp_ms),
                      "context_parallel_apply": ms_pass}
+    elif step.decode:
+        dom, bytes_dom, ms_dom = "decode_kernel", decode_bytes(w), ms_pass
+        breakdown = {"decode": ms_pass}
     else:
         dom = "fused_chunk_kernel<prefill>" if step.ws.numel() == 0 else \
             "kda_chunk_fwd (planner; pieces: build with readouts, pool scan, apply; or the prefill kernel)"
@@ -448,8 +477,8 @@ def run_ours(args):
             "frac": achieved / pk["hbm_gbs"], "traffic": recorded_traffic(dom),
             "algorithmic_bytes_per_launch": bytes_dom, "ms_per_launch": ms_dom,
             "peak_source": pk["source"]}
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+    line = {"metric": DECODE_METRIC if step.decode else METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.q.dtype == torch.bfloat16 else "f32", "data": "synthetic",
             "config": {"workload": args.workload, "tokens": tokens, "num_v_heads": w.num_v_heads,
                        "num_k_heads": w.num_k_heads, "dk": w.dk, "dv": w.dv, "batch": w.batch,
@@ -457,7 +486,8 @@ def run_ours(args):
                        "pieces_per_segment": step.pieces if step.cp else None, "gate_mode": w.gate_mode,
                        "state_layout": w.state_layout, "parallelism": f"dp{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (%.2f GB read per step), no flush" % (
-                           (segment_build_bytes(w, step.P) if step.cp else chunk_fwd_bytes(w, w.batch)) / 1e9)},
+                           (segment_build_bytes(w, step.P) if step.cp else
+                            decode_bytes(w) if step.decode else chunk_fwd_bytes(w, w.batch)) / 1e9)},
             "breakdown_ms": breakdown,
             "roofline": roof, "gpu_launches": step.launches() * args.steps, "clocks": clocks.summary()}
     if e2e is not None:
@@ -538,6 +568,15 @@ def profile_launches(args):
             step()
         torch.cuda.synchronize()
         print("launched", args.profile_launches, "context-parallel steps; pieces per segment", step.pieces)
+        return 0
+    if w.notes.get("decode"):
+        pool = w.state_pool.clone()
+        for _ in range(args.profile_launches):
+            kda.kda_decode(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, pool, w.state_indices,
+                           output_dtype=w.output_dtype, gate_mode=w.gate_mode, beta_mode=w.beta_mode,
+                           state_layout=w.state_layout, gate_lower_bound=w.gate_lower_bound)
+        torch.cuda.synchronize()
+        print("launched", args.profile_launches, "decode steps")
         return 0
     for _ in range(args.profile_launches):
         pool = w.state_pool.clone()

@@ -1,7 +1,7 @@
 /*
  * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention prefill library (libkda.so).
  *
- * Two operations:
+ * The operations:
  *
  *  kda_chunk_fwd
  *    The chunk-parallel KDA prefill ("max.nn.state_space.kda_chunk": the same recurrence as
@@ -18,6 +18,10 @@
  *    S (dk x dv, fp32) starts as state_pool[state_indices[b], h] and is written back there
  *    when the sequence ends.  The key head used by value head h is h / (Hv / Hk).  No query
  *    scaling is applied (GStar Assignment 2: the formulas omit it; scale = 1).
+ *
+ *  kda_decode
+ *    The same step for one token of each sequence in a batch (the single-token path that
+ *    "max.nn.state_space.kda_chunk" names kda_decode), in place on the state pool.
  *
  *  kda_segment_summarize_and_scan
  *    Context-parallel segment summary and exclusive scan ("KDA Context Parallelism"): a
@@ -125,6 +129,35 @@ KDA_API kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, 
                            const int32_t *state_indices, void *out, kda_dtype_t out_dtype,
                            uint32_t flags, float gate_lower_bound, void *workspace,
                            size_t workspace_bytes, int32_t *device_status, void *stream);
+
+/*
+ * kda_decode -- one token of each sequence in a batch, in place on the state pool
+ * ("max.nn.state_space.kda_chunk": single-token decode is the kda_decode path of the same
+ * recurrence; "nx_nofloat_kda.nx source", kda_step: decay, delta write, readout).  For every
+ * sequence b and value head h, with S = state_pool[state_indices[b], h]:
+ *     S = Diag(exp(g)) S;   S = S + k (beta (v - k^T S))^T;   out[b,h,:] = q^T S
+ * with g and beta as in kda_chunk_fwd.  The result equals kda_chunk_fwd on a batch whose every
+ * sequence has one token (cu_seqlens = 0, 1, ..., batch).
+ *
+ *   q, k          [batch, num_k_heads, dk]   qkv_dtype
+ *   v             [batch, num_v_heads, dv]   qkv_dtype
+ *   raw_gate      [batch, num_v_heads, dk]   fp32;   beta_logits [batch, num_v_heads] fp32
+ *   a_log [num_v_heads], dt_bias [num_v_heads, dk]   fp32
+ *   state_pool    as kda_chunk_fwd (K_FIRST or V_FIRST), read and written in place
+ *   state_indices [batch] int32;  out [batch, num_v_heads, dv] out_dtype
+ *   flags         KDA_GATE_SAFE, KDA_BETA_PROB, KDA_STATE_V_FIRST (others: KDA_ERR_INVALID_ARG)
+ *
+ * Supported: 1 <= dk, dv <= 128; (qkv F32, out F32) or (qkv BF16, out BF16 or F32); fp32
+ * arithmetic throughout.  A slot outside [0, max_slots) is reported in device_status and that
+ * sequence is skipped (its output row is not written).  batch = 0 does nothing.
+ */
+KDA_API kda_status_t kda_decode(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                                const float *raw_gate, const float *beta_logits, const float *a_log,
+                                const float *dt_bias, int32_t batch, int32_t num_k_heads,
+                                int32_t num_v_heads, int32_t dk, int32_t dv, float *state_pool,
+                                int32_t max_slots, const int32_t *state_indices, void *out,
+                                kda_dtype_t out_dtype, uint32_t flags, float gate_lower_bound,
+                                int32_t *device_status, void *stream);
 
 /*
  * kda_segment_summarize_and_scan -- segment summaries and the exclusive affine scan of ONE

@@ -148,6 +148,8 @@ WORKLOADS = (
     "batch64_T2048_H16_safe",
     "batch4_T2048_H32",  # one wave of 128 chains, inputs 404 MB (> L2): the profiling case
     "long_T16384_H32_cp2",  # context-parallel profiling case: 2 segments of 8192, inputs 420 MB
+    "decode_B256_H32",  # single-token step: 256 sequences x 32 heads, pool 537 MB (> L2)
+    "decode_B64_H16_safe",  # single-token step on the large-batch prefill's pool shape, safe gate
 )
 
 
@@ -179,6 +181,17 @@ def make(name: str, device="cpu", seed: Optional[int] = None) -> Workload:
     elif name == "long_T16384_H32_cp2":
         w = random_inputs([16384], 32, 32, 128, 128, seed=s, state_std=0.1, device=device, name=name)
         w.seg_offsets = (torch.arange(3, dtype=torch.int32) * 8192).to(device)
+    elif name == "decode_B256_H32":
+        g = torch.Generator().manual_seed(1000 + s)
+        idxs = torch.randperm(256, generator=g).to(torch.int32)
+        w = random_inputs([1] * 256, 32, 32, 128, 128, seed=s, state_std=0.1, max_slots=256,
+                          state_indices=idxs, device=device, name=name)
+        w.notes["decode"] = True
+    elif name == "decode_B64_H16_safe":
+        w = random_inputs([1] * 64, 16, 16, 128, 128, seed=s, raw_std=2.0, beta_mean=2.0, beta_std=1.0,
+                          state_std=0.1, gate_mode="safe", gate_lower_bound=-5.0, state_layout="V_FIRST",
+                          device=device, name=name)
+        w.notes["decode"] = True
     else:  # pragma: no cover
         raise KeyError(name)
     return w

@@ -6,6 +6,7 @@ memory and streams.  There is no CPU path: if ``libkda.so`` is missing, every ca
 
 Public calls (same names as the C ABI):
   kda_chunk_fwd(...)                      chunk-parallel prefill, mutates state_pool in place
+  kda_decode(...)                         one token per sequence, mutates state_pool in place
   kda_segment_summarize_and_scan(...)     segment (M_i, U_i) summaries + exclusive scan
   kda_context_parallel(M, U, initial)     the scan alone, returning exactly incoming_states,
                                           outgoing_states and final_state
@@ -18,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_segment_summarize_and_scan", "kda_context_parallel",
+__all__ = ["kda_chunk_fwd", "kda_decode", "kda_segment_summarize_and_scan", "kda_context_parallel",
            "kda_context_parallel_apply", "kda_context_parallel_prefill", "kda_context_parallel_workspace_size",
            "kda_context_parallel_workspace_preferred", "kda_context_parallel_pieces",
            "kda_context_parallel_piece_offsets", "kda_segment_compose", "kda_workspace_size",
@@ -60,6 +61,9 @@ def load_library():
     lib.kda_chunk_fwd.restype = ctypes.c_int
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, ctypes.c_int, fp, fp, fp, fp, ip, i32, i64, i32, i32, i32,
                                   i32, fp, i32, ip, vp, ctypes.c_int, u32, f32, vp, sz, ip, vp]
+    lib.kda_decode.restype = ctypes.c_int
+    lib.kda_decode.argtypes = [vp, vp, vp, ctypes.c_int, fp, fp, fp, fp, i32, i32, i32, i32, i32, fp, i32, ip,
+                               vp, ctypes.c_int, u32, f32, ip, vp]
     lib.kda_segment_summarize_and_scan.restype = ctypes.c_int
     lib.kda_segment_summarize_and_scan.argtypes = [vp, vp, ctypes.c_int, fp, fp, fp, fp, i64, i32, i32,
                                                    i32, i32, ip, i32, fp, fp, fp, fp, fp, fp, vp, vp, vp, u32,
@@ -206,6 +210,56 @@ def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, st
                            _ptr(device_status), _stream(stream, dev))
     if rc != 0:
         raise KdaError(rc, "kda_chunk_fwd")
+    return out
+
+
+def kda_decode(q, k, v, raw_gate, beta_logits, a_log, dt_bias, state_pool, state_indices, out=None, *,
+               output_dtype=None, gate_mode="original", beta_mode="logits", state_layout="K_FIRST",
+               gate_lower_bound=-5.0, device_status=None, stream=None):
+    """One KDA step for one token of each sequence (the kda_decode path of kda_chunk's recurrence).
+
+    Shapes: q,k [B,Hk,dk]; v [B,Hv,dv]; raw_gate [B,Hv,dk] f32; beta_logits [B,Hv] f32; a_log [Hv];
+    dt_bias [Hv,dk]; state_pool [slots,Hv,dk,dv] (K_FIRST) or [slots,Hv,dv,dk] (V_FIRST) f32,
+    mutated in place; state_indices [B] i32.  Returns out [B,Hv,dv] in ``output_dtype``.
+    """
+    lib = load_library()
+    dev = q.device
+    _dev(q, "q", device=dev)
+    if q.dtype not in _DTYPES:
+        raise ValueError("q/k/v must be float32 or bfloat16")
+    if q.dim() != 3:
+        raise ValueError(f"q has shape {tuple(q.shape)}, expected [B, Hk, dk]")
+    B, Hk, dk = q.shape
+    _shape(_dev(k, "k", q.dtype, dev), "k", (B, Hk, dk))
+    _dev(v, "v", q.dtype, dev)
+    if v.dim() != 3 or v.shape[0] != B:
+        raise ValueError(f"v has shape {tuple(v.shape)}, expected [{B}, Hv, dv]")
+    Hv, dv = v.shape[1], v.shape[2]
+    _shape(_dev(raw_gate, "raw_gate", torch.float32, dev), "raw_gate", (B, Hv, dk))
+    _shape(_dev(beta_logits, "beta_logits", torch.float32, dev), "beta_logits", (B, Hv))
+    _shape(_dev(a_log, "a_log", torch.float32, dev), "a_log", (Hv,))
+    _shape(_dev(dt_bias, "dt_bias", torch.float32, dev), "dt_bias", (Hv, dk))
+    _shape(_dev(state_indices, "state_indices", torch.int32, dev), "state_indices", (B,))
+    _dev(state_pool, "state_pool", torch.float32, dev)
+    blk = (Hv, dk, dv) if state_layout == "K_FIRST" else (Hv, dv, dk)
+    if state_pool.dim() != 4 or tuple(state_pool.shape[1:]) != blk:
+        raise ValueError(f"state_pool has shape {tuple(state_pool.shape)}, expected [slots, {blk}]")
+    if output_dtype is None:
+        output_dtype = v.dtype if out is None else out.dtype
+    if output_dtype not in _DTYPES:
+        raise ValueError("output_dtype must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty((B, Hv, dv), dtype=output_dtype, device=dev)
+    _shape(_dev(out, "out", output_dtype, dev), "out", (B, Hv, dv))
+    if device_status is not None:
+        _shape(_dev(device_status, "device_status", torch.int32, dev), "device_status", (1,))
+    flags = _flags(gate_mode, beta_mode, state_layout)
+    rc = lib.kda_decode(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], _ptr(raw_gate), _ptr(beta_logits), _ptr(a_log),
+                        _ptr(dt_bias), B, Hk, Hv, dk, dv, _ptr(state_pool), state_pool.shape[0],
+                        _ptr(state_indices), _ptr(out), _DTYPES[output_dtype], flags, float(gate_lower_bound),
+                        _ptr(device_status), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_decode")
     return out
 
 

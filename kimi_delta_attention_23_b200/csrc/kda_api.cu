@@ -280,6 +280,48 @@ extern "C" kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* 
   return kda::launch_cp_apply(ap, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+extern "C" kda_status_t kda_decode(const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype,
+                                   const float* raw_gate, const float* beta_logits, const float* a_log,
+                                   const float* dt_bias, int32_t batch, int32_t num_k_heads, int32_t num_v_heads,
+                                   int32_t dk, int32_t dv, float* state_pool, int32_t max_slots,
+                                   const int32_t* state_indices, void* out, kda_dtype_t out_dtype, uint32_t flags,
+                                   float gate_lower_bound, int32_t* device_status, void* stream) {
+  if (batch < 0 || num_k_heads <= 0 || num_v_heads <= 0 || dk <= 0 || dv <= 0 || max_slots <= 0)
+    return KDA_ERR_INVALID_ARG;
+  if (num_v_heads % num_k_heads != 0) return KDA_ERR_INVALID_ARG;
+  if ((flags & ~(uint32_t)(KDA_GATE_SAFE | KDA_BETA_PROB | KDA_STATE_V_FIRST)) != 0) return KDA_ERR_INVALID_ARG;
+  if (!state_pool || !state_indices || !a_log || !dt_bias) return KDA_ERR_INVALID_ARG;
+  if (batch > 0 && (!q || !k || !v || !raw_gate || !beta_logits || !out)) return KDA_ERR_INVALID_ARG;
+  if (!dtype_ok(qkv_dtype) || !dtype_ok(out_dtype)) return KDA_ERR_UNSUPPORTED;
+  if (qkv_dtype == KDA_F32 && out_dtype != KDA_F32) return KDA_ERR_UNSUPPORTED;
+  if (dk > 128 || dv > 128) return KDA_ERR_UNSUPPORTED;
+  if (batch == 0) return KDA_OK;
+  kda::DecodeArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.in_bf16 = qkv_dtype == KDA_BF16;
+  a.raw_gate = raw_gate;
+  a.beta = beta_logits;
+  a.a_log = a_log;
+  a.dt_bias = dt_bias;
+  a.batch = batch;
+  a.Hk = num_k_heads;
+  a.Hv = num_v_heads;
+  a.dk = dk;
+  a.dv = dv;
+  a.pool = state_pool;
+  a.max_slots = max_slots;
+  a.slots = state_indices;
+  a.v_first = (flags & KDA_STATE_V_FIRST) ? 1 : 0;
+  a.out = out;
+  a.out_bf16 = out_dtype == KDA_BF16;
+  a.flags = flags;
+  a.lb = gate_lower_bound;
+  a.status = device_status;
+  return kda::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 extern "C" kda_status_t kda_segment_summarize_and_scan(
     const void* k, const void* v, kda_dtype_t kv_dtype, const float* raw_gate, const float* beta_logits,
     const float* a_log, const float* dt_bias, int64_t T, int32_t num_k_heads, int32_t num_v_heads,

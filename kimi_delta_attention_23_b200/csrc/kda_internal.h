@@ -143,6 +143,29 @@ struct ComposeArgs {
   float* outgoing;           // [N][H][state]
 };
 
+// Single-token step of a batch of sequences (one token each), in place on the pool.
+struct DecodeArgs {
+  const void* q;            // [batch,Hk,dk]
+  const void* k;            // [batch,Hk,dk]
+  const void* v;            // [batch,Hv,dv]
+  int32_t in_bf16;
+  const float* raw_gate;    // [batch,Hv,dk]
+  const float* beta;        // [batch,Hv]
+  const float* a_log;       // [Hv]
+  const float* dt_bias;     // [Hv,dk]
+  int32_t batch;
+  int32_t Hk, Hv, dk, dv;
+  float* pool;              // [max_slots][Hv][dk][dv] (K_FIRST) or [..][dv][dk] (V_FIRST)
+  int32_t max_slots;
+  const int32_t* slots;     // [batch]
+  int32_t v_first;
+  void* out;                // [batch,Hv,dv]
+  int32_t out_bf16;
+  uint32_t flags;
+  float lb;
+  int32_t* status;
+};
+
 size_t simt_smem_bytes(int dk, int w);
 cudaError_t launch_split_offsets(const int32_t* offs, int32_t N, int32_t k, int32_t* sub, cudaStream_t stream);
 cudaError_t launch_compose_pieces(const ComposeArgs& a, cudaStream_t stream);
@@ -151,5 +174,6 @@ cudaError_t launch_pool_scan(const PoolScanArgs& a, cudaStream_t stream);
 cudaError_t launch_cp_apply(const ApplyArgs& a, cudaStream_t stream);
 cudaError_t launch_simt_chunk(const SimtArgs& a, cudaStream_t stream);
 cudaError_t launch_affine_scan(const ScanArgs& a, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace kda

@@ -140,6 +140,17 @@ def kda_forward(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, stat
     return out, pool
 
 
+def kda_decode(q, k, v, raw_gate, beta_logits, a_log, dt_bias, state_pool, state_indices=None, *,
+               gate_mode="original", beta_mode="logits", state_layout="K_FIRST", gate_lower_bound=-5.0):
+    """One token per sequence: the token-by-token definition on a batch of one-token sequences
+    (q, k [B,Hk,dk], v [B,Hv,dv], ...).  Returns (out [B,Hv,dv], new_state_pool)."""
+    B = int(np.asarray(q.shape)[0])
+    cu = np.arange(B + 1, dtype=np.int32)
+    return kda_forward(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu, state_pool, state_indices,
+                       gate_mode=gate_mode, beta_mode=beta_mode, state_layout=state_layout,
+                       gate_lower_bound=gate_lower_bound)
+
+
 def kda_segment_summary(k, v, raw_gate, beta_logits, a_log, dt_bias, seg_offsets, *,
                         num_v_heads=None, gate_mode="original", beta_mode="logits",
                         state_layout="K_FIRST", gate_lower_bound=-5.0):

@@ -147,3 +147,30 @@ def test_without_a_device_nothing_is_split():
     assert kda.kda_context_parallel_pieces(1 << 17, 16, 32) == 1
     assert kda.kda_context_parallel_workspace_preferred(1 << 17, 16, 32, 128) == \
         kda.kda_context_parallel_workspace_size(1 << 17, 32, 128)
+
+
+def _decode(lib, **over):
+    args = dict(q=1, k=1, v=1, qkv=1, raw=1, beta=1, a_log=1, dt_bias=1, batch=3, Hk=2, Hv=4, dk=128, dv=128,
+                pool=1, slots=4, idx=1, out=1, out_dtype=1, flags=0)
+    args.update(over)
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731  (never dereferenced: checks fail first)
+    return lib.kda_decode(p(args["q"]), p(args["k"]), p(args["v"]), args["qkv"], p(args["raw"]), p(args["beta"]),
+                          p(args["a_log"]), p(args["dt_bias"]), args["batch"], args["Hk"], args["Hv"], args["dk"],
+                          args["dv"], p(args["pool"]), args["slots"], p(args["idx"]), p(args["out"]),
+                          args["out_dtype"], args["flags"], -5.0, None, None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(batch=-1), 1), (dict(Hk=0), 1), (dict(Hv=5), 1), (dict(dk=0), 1), (dict(dv=-2), 1), (dict(slots=0), 1),
+    (dict(flags=kda.FUSED), 1), (dict(flags=kda.SEG_SCAN_ONLY), 1), (dict(flags=1 << 9), 1), (dict(q=0), 1),
+    (dict(v=0), 1), (dict(raw=0), 1), (dict(pool=0), 1), (dict(idx=0), 1), (dict(out=0), 1), (dict(dt_bias=0), 1),
+    (dict(qkv=5), 2), (dict(out_dtype=3), 2),
+    (dict(qkv=0, out_dtype=1), 2),                                  # fp32 inputs need fp32 output
+    (dict(dk=129), 2), (dict(dv=256), 2),                           # head dims beyond the kernel
+])
+def test_decode_host_checks(lib, over, code):
+    assert _decode(lib, **over) == code
+
+
+def test_decode_empty_batch_is_a_no_op(lib):
+    assert _decode(lib, batch=0, q=0, k=0, v=0, raw=0, beta=0, out=0) == 0

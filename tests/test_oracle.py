@@ -402,6 +402,25 @@ def test_split_call_resumes_from_pool():
         assert rel(p_b, pool) < 1e-14
 
 
+def test_decode_steps_equal_the_prefill():
+    # kda_decode is the single-token path of the same recurrence ("max.nn.state_space.kda_chunk"):
+    # stepping each sequence one token at a time through its pool slot equals one prefill call
+    w = tiny([9, 9, 9], Hk=1, Hv=2, dk=5, dv=4, seed=31, max_slots=4,
+             state_indices=torch.tensor([3, 0, 2], dtype=torch.int32), state_layout="V_FIRST")
+    out, pool = run(w)
+    p = w.state_pool
+    steps = []
+    for t in range(9):
+        rows = [0 + t, 9 + t, 18 + t]
+        o, p = oracle.kda_decode(w.q[rows], w.k[rows], w.v[rows], w.raw_gate[rows], w.beta_logits[rows], w.a_log,
+                                 w.dt_bias, p, w.state_indices, state_layout="V_FIRST")
+        steps.append(o)
+    got = np.stack(steps, axis=1).reshape(27, 2, 4)
+    assert rel(got, out) < 1e-14
+    assert rel(p, pool) < 1e-14
+    assert np.array_equal(p[1], np.asarray(w.state_pool[1], np.float64))  # unnamed slot untouched
+
+
 @pytest.mark.parametrize("chunk", [1, 2, 4, 16])
 @pytest.mark.parametrize("gate_mode,raw_std", [("original", 1.0), ("original", 3.0), ("safe", 2.0)])
 def test_chunked_algebra_equals_recurrence(chunk, gate_mode, raw_std):
