@@ -127,13 +127,16 @@ template <bool kBuild, bool kRead>
 __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArgs a, const __grid_constant__ InputMaps tm) {
   if (a.gate_flag && *a.gate_flag != a.gate_run_if) return;  // this launch is not the one that runs
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-aligned base, offset from the shared array itself so that every pointer derived from it
+  // stays in the shared window (32-bit shared addressing instead of generic pointers)
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.x, b = blockIdx.y;
   const int kh = h / (a.Hv / a.Hk);
   const bool safe = a.flags & KDA_GATE_SAFE, prob = a.flags & KDA_BETA_PROB;
 
-  const int64_t t0 = a.cu[b], t1 = a.cu[b + 1];
+  const int t0 = a.cu[b], t1 = a.cu[b + 1];  // token offsets (int32 like cu_seqlens)
   const int32_t slot = a.slots ? a.slots[b] : b;
   if (t0 < 0 || t1 < t0 || t1 > a.total_tokens || slot < 0 || slot >= a.max_slots) {
     if (tid == 0) report(a.status, KDA_ERR_DEVICE_CHECK);
@@ -185,13 +188,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   const uint32_t gkq_bytes = 32768u + 16384u * (1u + (qb ? 1u : 0u));
   // gate, k and q land in the score scratch (free once the chunk's inverse is done); V lands
   // in its operand tile (free once the chunk's second product completed)
-  auto issue_prefetch_gkq = [&](int64_t c0n) {
+  auto issue_prefetch_gkq = [&](int c0n) {
     mbar_arrive_expect_tx(bar_pf, gkq_bytes);
     tma_load_3d(sbase + PF_RAW, &tm.raw, 0, h, (int)c0n, bar_pf);
     tma_load_3d(sbase + PF_K, &tm.k, 0, kh, (int)c0n, bar_pf);
     if (qb) tma_load_3d(sbase + PF_Q, &tm.q, 0, kh, (int)c0n, bar_pf);
   };
-  auto issue_prefetch_v = [&](int64_t c0n) {
+  auto issue_prefetch_v = [&](int c0n) {
     if (has_v) {
       mbar_arrive_expect_tx(bar_v, 16384u);
       tma_load_3d(sbase + OFF_V, &tm.v, 0, h, (int)c0n, bar_v);
@@ -265,8 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
 
   // beta of the next chunk is read one chunk ahead (lanes 0..7 of each warp, one row each)
   float beta_raw = 0.f;
-  auto load_beta = [&](int64_t c0n) {
-    const int64_t t = c0n + warp * 8 + lane;
+  auto load_beta = [&](int c0n) {
+    const int t = c0n + warp * 8 + lane;
     if (lane < 8 && t < t1) beta_raw = __ldg(a.beta + (size_t)t * a.Hv + h);
   };
   // gates of the chunk whose inputs are in the prefetch region (Ln valid rows): the decay alpha
@@ -304,13 +307,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       sBeta[row] = row < Ln ? beta_f32(beta_raw, prob) : 0.f;
     }
   };
-  auto rows_of = [&](int64_t c0n) { return (int)((t1 - c0n) < C ? (t1 - c0n) : C); };
+  auto rows_of = [&](int c0n) { return (t1 - c0n) < C ? (t1 - c0n) : C; };
   load_beta(t0);
   if (t1 > t0) gate_phase(rows_of(t0));
   uint32_t phase = 0;
   bool aborted = false;
 #pragma unroll 1
-  for (int64_t c0 = t0; c0 < t1; c0 += C, phase ^= 1u) {
+  for (int c0 = t0; c0 < t1; c0 += C, phase ^= 1u) {
     const int L = rows_of(c0);
 
     // =============================== k-side, part 1: in-block products (the gates were done
