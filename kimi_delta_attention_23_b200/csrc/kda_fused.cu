@@ -255,6 +255,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     }
     tmem_wait_st();
   }
+  // P's upper triangle must read as zero (A's upper triangle is never read); no chunk writes
+  // there, so it is cleared once
+  if constexpr (kRead)
+    for (int e = tid; e < 8192 / 16; e += kThreads) reinterpret_cast<uint4*>(sm + OFF_P)[e] = make_uint4(0, 0, 0, 0);
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -336,9 +340,116 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         q2[r] = make_uint2(0u, 0u);
       }
     }
-    // P's upper triangle must read as zero (A's upper triangle is never read)
-    if constexpr (kRead)
-      for (int e = tid; e < 8192 / 16; e += kThreads) reinterpret_cast<uint4*>(sm + OFF_P)[e] = make_uint4(0, 0, 0, 0);
+    // k and q of my rows in fp32, kept for the diagonal blocks and the operand tiles
+    float kf[8][4], qf[8][4];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const float2 k01 = unpack_bf16(k2[r].x), k23 = unpack_bf16(k2[r].y);
+      const float2 q01 = unpack_bf16(q2[r].x), q23 = unpack_bf16(q2[r].y);
+      kf[r][0] = k01.x;
+      kf[r][1] = k01.y;
+      kf[r][2] = k23.x;
+      kf[r][3] = k23.y;
+      qf[r][0] = q01.x;
+      qf[r][1] = q01.y;
+      qf[r][2] = q23.x;
+      qf[r][3] = q23.y;
+    }
+    // the diagonal 8x8 score blocks need only this block's rows: formed before (1)
+    // diagonal 8x8 blocks on CUDA cores: partial sums over my 4 channels of
+    //   A_rs (r > s, slots 0..27) and P_rs (r >= s, slots 28..63), then a butterfly
+    //   reduce-scatter over the 32 lanes leaves slots 2*lane and 2*lane+1 in this lane
+    //   (build: A only, 32 slots, slot lane in this lane)
+    if constexpr (!kRead) {
+      float acc[32];
+#pragma unroll
+      for (int i = 28; i < 32; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        float w[4] = {kf[s][0], kf[s][1], kf[s][2], kf[s][3]};
+#pragma unroll
+        for (int r = s + 1; r < 8; ++r) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) w[c] *= al[r][c];
+          acc[r * (r - 1) / 2 + s] = kf[r][0] * w[0] + kf[r][1] * w[1] + kf[r][2] * w[2] + kf[r][3] * w[3];
+        }
+      }
+#pragma unroll
+      for (int half = 16; half >= 1; half >>= 1) {
+        const bool hi = (lane & half) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const float send = hi ? acc[i] : acc[i + half];
+          const float keep = hi ? acc[i + half] : acc[i];
+          acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+        }
+      }
+      if (lane < 28) {
+        const int rs = kDiagPair[lane], r = rs >> 3, sc = rs & 7;
+        sA[(warp * 8 + r) * kLdA + warp * 8 + sc] = acc[0];
+      }
+    } else {
+      float acc[64];
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        float w[4] = {kf[s][0], kf[s][1], kf[s][2], kf[s][3]};
+        acc[28 + s * (s + 1) / 2 + s] = qf[s][0] * w[0] + qf[s][1] * w[1] + qf[s][2] * w[2] + qf[s][3] * w[3];
+#pragma unroll
+        for (int r = s + 1; r < 8; ++r) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) w[c] *= al[r][c];
+          acc[r * (r - 1) / 2 + s] = kf[r][0] * w[0] + kf[r][1] * w[1] + kf[r][2] * w[2] + kf[r][3] * w[3];
+          acc[28 + r * (r + 1) / 2 + s] = qf[r][0] * w[0] + qf[r][1] * w[1] + qf[r][2] * w[2] + qf[r][3] * w[3];
+        }
+      }
+#pragma unroll
+      for (int half = 32; half >= 2; half >>= 1) {
+        const int bit = half >> 1;  // 16, 8, 4, 2, 1
+        const bool hi = (lane & bit) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+          const float send = hi ? acc[i] : acc[i + half];
+          const float keep = hi ? acc[i + half] : acc[i];
+          acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int idx = 2 * lane + u;
+        const int rs = kDiagPair[idx], r = rs >> 3, sc = rs & 7;
+        if (idx < 28) {
+          sA[(warp * 8 + r) * kLdA + warp * 8 + sc] = acc[u];
+        } else {
+          *reinterpret_cast<__nv_bfloat16*>(sm + OFF_P + sw_off(warp * 8 + r, warp * 8 + sc, 64)) =
+              __float2bfloat16_rn(acc[u]);
+        }
+      }
+    }
+    // the inverse of this 8-row block's diagonal part, X = (I + diag(beta) A_blk)^{-1} (unit
+    // lower triangular): lane j < 8 runs the forward substitution of column j; the strictly lower
+    // part goes to the block's upper triangle of sA (never read as A), transposed
+    __syncwarp();
+    if (lane < 8) {
+      const int j = lane, base = warp * 8;
+      float lb[8][8], bb[8];  // the block's strictly lower scores and its betas, loaded up front
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        bb[r] = sBeta[base + r];
+#pragma unroll
+        for (int c = 0; c < r; ++c) lb[r][c] = sA[(base + r) * kLdA + base + c];
+      }
+      float x[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < r; ++c) acc = fmaf(lb[r][c], x[c], acc);
+        x[r] = r < j ? 0.f : (r == j ? 1.f : -bb[r] * acc);
+      }
+#pragma unroll
+      for (int r = 1; r < 8; ++r)
+        if (r > j) sA[(base + j) * kLdA + base + r] = x[r];
+    }
     // in-block products: p8 inclusive prefix from the block start, s8 exclusive suffix
     float p8[8][4], s8[8][4];
 #pragma unroll
@@ -409,48 +520,46 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       *reinterpret_cast<float4*>(sMp + 4 * D + ch) = make_float4(t16b[0], t16b[1], t16b[2], t16b[3]);
       *reinterpret_cast<float4*>(sMp + 5 * D + ch) = one;
     }
-    // operand tiles
+    // operand tiles.  The block-local products are formed once per row -- kp = k o p8 (prefix
+    // from the block start), qp = q o p8, ks = k o s8 (suffix to the block end) -- and every tile
+    // is one of them, possibly scaled once more: K o Gamma = kp o pre, K o pi = kp (o prevb in an
+    // upper half), K o kappa = ks (o nextb in a lower half), K' = ks o suf, the 8-level halves
+    // kp / qp (upper) and ks (lower).
     float kpv[8][4];  // K' values of my 8 rows x 4 channels (packed pairwise below)
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int row = warp * 8 + r;
-      const float2 k01 = unpack_bf16(k2[r].x), k23 = unpack_bf16(k2[r].y);
-      const float2 q01 = unpack_bf16(q2[r].x), q23 = unpack_bf16(q2[r].y);
-      const float kf[4] = {k01.x, k01.y, k23.x, k23.y};
-      const float qf[4] = {q01.x, q01.y, q23.x, q23.y};
-      float g[4], pi[4], ka[4], kp[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        g[c] = pre[c] * p8[r][c];
-        pi[c] = upper ? prevb[c] * p8[r][c] : p8[r][c];
-        ka[c] = upper ? s8[r][c] : s8[r][c] * nextb[c];
-        kp[c] = kf[c] * s8[r][c] * suf[c];
-      }
+      const float kp[4] = {kf[r][0] * p8[r][0], kf[r][1] * p8[r][1], kf[r][2] * p8[r][2], kf[r][3] * p8[r][3]};
+      const float qp[4] = {qf[r][0] * p8[r][0], qf[r][1] * p8[r][1], qf[r][2] * p8[r][2], qf[r][3] * p8[r][3]};
+      const float ks[4] = {kf[r][0] * s8[r][0], kf[r][1] * s8[r][1], kf[r][2] * s8[r][2], kf[r][3] * s8[r][3]};
       *reinterpret_cast<uint2*>(sm + OFF_KQ + sw_off(row, ch, 128)) =
-          pack4(kf[0] * g[0], kf[1] * g[1], kf[2] * g[2], kf[3] * g[3]);
+          pack4(kp[0] * pre[0], kp[1] * pre[1], kp[2] * pre[2], kp[3] * pre[3]);
       if constexpr (kRead)
         *reinterpret_cast<uint2*>(sm + OFF_KQ + sw_off(64 + row, ch, 128)) =
-            pack4(qf[0] * g[0], qf[1] * g[1], qf[2] * g[2], qf[3] * g[3]);
-      *reinterpret_cast<uint2*>(sm + OFF_KPI + sw_off(row, ch, 64)) =
-          pack4(kf[0] * pi[0], kf[1] * pi[1], kf[2] * pi[2], kf[3] * pi[3]);
-      if constexpr (kRead)
-        *reinterpret_cast<uint2*>(sm + OFF_QPI + sw_off(row, ch, 64)) =
-            pack4(qf[0] * pi[0], qf[1] * pi[1], qf[2] * pi[2], qf[3] * pi[3]);
-      *reinterpret_cast<uint2*>(sm + OFF_KC + sw_off(row, ch, 64)) =
-          pack4(kf[0] * ka[0], kf[1] * ka[1], kf[2] * ka[2], kf[3] * ka[3]);
+            pack4(qp[0] * pre[0], qp[1] * pre[1], qp[2] * pre[2], qp[3] * pre[3]);
       const int r32 = b16 * 8 + r;
       if (upper) {
-        *reinterpret_cast<uint2*>(sm + OFF_KPI8 + sw_off(r32, ch, 32)) =
-            pack4(kf[0] * p8[r][0], kf[1] * p8[r][1], kf[2] * p8[r][2], kf[3] * p8[r][3]);
-        if constexpr (kRead)
-          *reinterpret_cast<uint2*>(sm + OFF_QPI8 + sw_off(r32, ch, 32)) =
-              pack4(qf[0] * p8[r][0], qf[1] * p8[r][1], qf[2] * p8[r][2], qf[3] * p8[r][3]);
+        const uint2 kp_b = pack4(kp[0], kp[1], kp[2], kp[3]);
+        *reinterpret_cast<uint2*>(sm + OFF_KPI + sw_off(row, ch, 64)) =
+            pack4(kp[0] * prevb[0], kp[1] * prevb[1], kp[2] * prevb[2], kp[3] * prevb[3]);
+        *reinterpret_cast<uint2*>(sm + OFF_KPI8 + sw_off(r32, ch, 32)) = kp_b;
+        if constexpr (kRead) {
+          *reinterpret_cast<uint2*>(sm + OFF_QPI + sw_off(row, ch, 64)) =
+              pack4(qp[0] * prevb[0], qp[1] * prevb[1], qp[2] * prevb[2], qp[3] * prevb[3]);
+          *reinterpret_cast<uint2*>(sm + OFF_QPI8 + sw_off(r32, ch, 32)) = pack4(qp[0], qp[1], qp[2], qp[3]);
+        }
+        *reinterpret_cast<uint2*>(sm + OFF_KC + sw_off(row, ch, 64)) = pack4(ks[0], ks[1], ks[2], ks[3]);
       } else {
-        *reinterpret_cast<uint2*>(sm + OFF_KK8 + sw_off(r32, ch, 32)) =
-            pack4(kf[0] * s8[r][0], kf[1] * s8[r][1], kf[2] * s8[r][2], kf[3] * s8[r][3]);
+        const uint2 ks_b = pack4(ks[0], ks[1], ks[2], ks[3]);
+        *reinterpret_cast<uint2*>(sm + OFF_KPI + sw_off(row, ch, 64)) = pack4(kp[0], kp[1], kp[2], kp[3]);
+        if constexpr (kRead)
+          *reinterpret_cast<uint2*>(sm + OFF_QPI + sw_off(row, ch, 64)) = pack4(qp[0], qp[1], qp[2], qp[3]);
+        *reinterpret_cast<uint2*>(sm + OFF_KC + sw_off(row, ch, 64)) =
+            pack4(ks[0] * nextb[0], ks[1] * nextb[1], ks[2] * nextb[2], ks[3] * nextb[3]);
+        *reinterpret_cast<uint2*>(sm + OFF_KK8 + sw_off(r32, ch, 32)) = ks_b;
       }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) kpv[r][c] = kp[c];
+      for (int c = 0; c < 4; ++c) kpv[r][c] = ks[c] * suf[c];
     }
     // K'^T: channel rows, token columns; pairs of consecutive tokens pack into one word
     uint32_t kpt[4][4];
@@ -471,123 +580,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       *reinterpret_cast<uint4*>(sm + OFF_KPT + sw_off(ch + c, warp * 8, 128)) = val;
     }
 
-    // diagonal 8x8 blocks on CUDA cores: partial sums over my 4 channels of
-    //   A_rs (r > s, slots 0..27) and P_rs (r >= s, slots 28..63), then a butterfly
-    //   reduce-scatter over the 32 lanes leaves slots 2*lane and 2*lane+1 in this lane
-    //   (build: A only, 32 slots, slot lane in this lane)
-    if constexpr (!kRead) {
-      float acc[32];
-      float kf[8][4];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const float2 k01 = unpack_bf16(k2[r].x), k23 = unpack_bf16(k2[r].y);
-        kf[r][0] = k01.x;
-        kf[r][1] = k01.y;
-        kf[r][2] = k23.x;
-        kf[r][3] = k23.y;
-      }
-#pragma unroll
-      for (int i = 28; i < 32; ++i) acc[i] = 0.f;
-#pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        float w[4] = {kf[s][0], kf[s][1], kf[s][2], kf[s][3]};
-#pragma unroll
-        for (int r = s + 1; r < 8; ++r) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) w[c] *= al[r][c];
-          acc[r * (r - 1) / 2 + s] = kf[r][0] * w[0] + kf[r][1] * w[1] + kf[r][2] * w[2] + kf[r][3] * w[3];
-        }
-      }
-#pragma unroll
-      for (int half = 16; half >= 1; half >>= 1) {
-        const bool hi = (lane & half) != 0;
-#pragma unroll
-        for (int i = 0; i < half; ++i) {
-          const float send = hi ? acc[i] : acc[i + half];
-          const float keep = hi ? acc[i + half] : acc[i];
-          acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
-        }
-      }
-      if (lane < 28) {
-        const int rs = kDiagPair[lane], r = rs >> 3, sc = rs & 7;
-        sA[(warp * 8 + r) * kLdA + warp * 8 + sc] = acc[0];
-      }
-    } else {
-      float acc[64];
-      float kf[8][4], qf[8][4];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const float2 k01 = unpack_bf16(k2[r].x), k23 = unpack_bf16(k2[r].y);
-        const float2 q01 = unpack_bf16(q2[r].x), q23 = unpack_bf16(q2[r].y);
-        kf[r][0] = k01.x;
-        kf[r][1] = k01.y;
-        kf[r][2] = k23.x;
-        kf[r][3] = k23.y;
-        qf[r][0] = q01.x;
-        qf[r][1] = q01.y;
-        qf[r][2] = q23.x;
-        qf[r][3] = q23.y;
-      }
-#pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        float w[4] = {kf[s][0], kf[s][1], kf[s][2], kf[s][3]};
-        acc[28 + s * (s + 1) / 2 + s] = qf[s][0] * w[0] + qf[s][1] * w[1] + qf[s][2] * w[2] + qf[s][3] * w[3];
-#pragma unroll
-        for (int r = s + 1; r < 8; ++r) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) w[c] *= al[r][c];
-          acc[r * (r - 1) / 2 + s] = kf[r][0] * w[0] + kf[r][1] * w[1] + kf[r][2] * w[2] + kf[r][3] * w[3];
-          acc[28 + r * (r + 1) / 2 + s] = qf[r][0] * w[0] + qf[r][1] * w[1] + qf[r][2] * w[2] + qf[r][3] * w[3];
-        }
-      }
-#pragma unroll
-      for (int half = 32; half >= 2; half >>= 1) {
-        const int bit = half >> 1;  // 16, 8, 4, 2, 1
-        const bool hi = (lane & bit) != 0;
-#pragma unroll
-        for (int i = 0; i < half; ++i) {
-          const float send = hi ? acc[i] : acc[i + half];
-          const float keep = hi ? acc[i + half] : acc[i];
-          acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int idx = 2 * lane + u;
-        const int rs = kDiagPair[idx], r = rs >> 3, sc = rs & 7;
-        if (idx < 28) {
-          sA[(warp * 8 + r) * kLdA + warp * 8 + sc] = acc[u];
-        } else {
-          *reinterpret_cast<__nv_bfloat16*>(sm + OFF_P + sw_off(warp * 8 + r, warp * 8 + sc, 64)) =
-              __float2bfloat16_rn(acc[u]);
-        }
-      }
-    }
-    // the inverse of this 8-row block's diagonal part, X = (I + diag(beta) A_blk)^{-1} (unit
-    // lower triangular): lane j < 8 runs the forward substitution of column j; the strictly lower
-    // part goes to the block's upper triangle of sA (never read as A), transposed
-    __syncwarp();
-    if (lane < 8) {
-      const int j = lane, base = warp * 8;
-      float lb[8][8], bb[8];  // the block's strictly lower scores and its betas, loaded up front
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        bb[r] = sBeta[base + r];
-#pragma unroll
-        for (int c = 0; c < r; ++c) lb[r][c] = sA[(base + r) * kLdA + base + c];
-      }
-      float x[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        float acc = 0.f;
-#pragma unroll
-        for (int c = 0; c < r; ++c) acc = fmaf(lb[r][c], x[c], acc);
-        x[r] = r < j ? 0.f : (r == j ? 1.f : -bb[r] * acc);
-      }
-#pragma unroll
-      for (int r = 1; r < 8; ++r)
-        if (r > j) sA[(base + j) * kLdA + base + r] = x[r];
-    }
     fence_async_smem();  // the operand tiles are read by the tensor cores
     __syncthreads();  // (2) operand tiles, block factors and diagonal scores in place
 
@@ -1151,11 +1143,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         if constexpr (kRead) {
           // readouts of both states, staged row-major bf16 in the K/Q tile (its last readers, the
           // readout products, completed; the state updates still read both X tiles)
-#pragma unroll 1
+          float dd[2][32];  // both states' readouts loaded before one wait
+          tmem_ld16n<2>(tmD1 + lane_base + 32 * ehalf, dd[0]);
+          tmem_ld16n<2>(tmD1u + lane_base + 32 * ehalf, dd[1]);
+          tmem_wait_ld();
+#pragma unroll
           for (int st = 0; st < 2; ++st) {
-            float d[32];
-            tmem_ld16n<2>((st ? tmD1u : tmD1) + lane_base + 32 * ehalf, d);
-            tmem_wait_ld();
+            const float* d = dd[st];
             uint8_t* stage = sm + OFF_KQ + st * 16384;
 #pragma unroll
             for (int u = 0; u < 32; u += 2) {  // one conversion per row pair, two 16-bit stores
