@@ -430,16 +430,24 @@ __device__ __forceinline__ void tile_product(const float* Ms, const float* cur, 
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int u = 0; u < 4; ++u) acc[i][u] = 0.f;
-#pragma unroll 4
-  for (int l = 0; l < 128; ++l) {
-    const float4 b = *reinterpret_cast<const float4*>(cur + l * kT + c0);
+  // four columns of M per step: one 16-byte load per row (conflict-free with the 132-float
+  // padding), four 16-byte loads of the carried tile, 64 fused multiply-adds
+#pragma unroll 2
+  for (int l = 0; l < 128; l += 4) {
+    float4 mr[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float m = Ms[(rb + 32 * i) * kLdM + l];
-      acc[i][0] = fmaf(m, b.x, acc[i][0]);
-      acc[i][1] = fmaf(m, b.y, acc[i][1]);
-      acc[i][2] = fmaf(m, b.z, acc[i][2]);
-      acc[i][3] = fmaf(m, b.w, acc[i][3]);
+    for (int i = 0; i < 4; ++i) mr[i] = *reinterpret_cast<const float4*>(Ms + (rb + 32 * i) * kLdM + l);
+#pragma unroll
+    for (int dl = 0; dl < 4; ++dl) {
+      const float4 b = *reinterpret_cast<const float4*>(cur + (l + dl) * kT + c0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float m = dl == 0 ? mr[i].x : dl == 1 ? mr[i].y : dl == 2 ? mr[i].z : mr[i].w;
+        acc[i][0] = fmaf(m, b.x, acc[i][0]);
+        acc[i][1] = fmaf(m, b.y, acc[i][1]);
+        acc[i][2] = fmaf(m, b.z, acc[i][2]);
+        acc[i][3] = fmaf(m, b.w, acc[i][3]);
+      }
     }
   }
 }
