@@ -34,8 +34,9 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // persistent grid of two blocks per SM splits it into equal contiguous ranges, so a block
 // touches only one or two (segment, head) pairs and loads each pair's incoming state once
 // (bf16, as the B operand).  The next tile's two readout tiles are copied asynchronously while
-// the current one is multiplied; warp w computes rows 16 (w % 4) .. +16 and columns
-// 64 (w / 4) .. +64 of a tile and adds the contribution readout.  A bf16 result overwrites the
+// the current one is multiplied; warp w computes rows 32 (w % 2) .. +32 and columns
+// 32 (w / 2) .. +32 of a tile -- its share of the incoming state stays in registers as B
+// fragments for all tiles of a pair -- and adds the contribution readout.  A bf16 result overwrites the
 // contribution tile in place (each thread rewrites exactly the elements it read) and leaves in
 // 16-byte row stores.
 struct TilePos {
@@ -118,7 +119,11 @@ __global__ void __launch_bounds__(kThreads, 2) cp_apply_kernel(ApplyArgs a) {
   TilePos cur{s_pos[0], s_pos[1], s_pos[2]};
   issue_tile(cur, 0);
   const int g = lane >> 2, t = lane & 3, m = lane >> 3;
-  const int r0 = 16 * (warp & 3), n0 = 64 * (warp >> 2);
+  // warp tile: rows r0 .. +32 (two 16-row MMA tiles), columns n0 .. +32 (four 8-column tiles);
+  // its B fragments (the incoming state, the same for every tile of a (segment, head) pair)
+  // stay in registers, so only the readout tiles are read from shared memory per tile
+  const int r0 = 32 * (warp & 1), n0 = 32 * (warp >> 1);
+  uint32_t bfrag[8][2][4];
   int loaded_seg = -1, loaded_h = -1, buf = 0;
 #pragma unroll 1
   for (int64_t i = 0; i < count; ++i, buf ^= 1) {
@@ -143,39 +148,50 @@ __global__ void __launch_bounds__(kThreads, 2) cp_apply_kernel(ApplyArgs a) {
       loaded_seg = cur.seg;
       loaded_h = cur.h;
       __syncthreads();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+          const int br = n0 + 16 * np + (m >> 1) * 8 + (lane & 7), bk = 16 * kk + (m & 1) * 8;
+          ldsm_x4(sB_addr + (br * kLd + bk) * 2, bfrag[kk][np][0], bfrag[kk][np][1], bfrag[kk][np][2],
+                  bfrag[kk][np][3]);
+        }
     }
     const int64_t c0 = offs[cur.seg] + (int64_t)kTile * cur.tile, s1 = offs[cur.seg + 1];
     const int L = (int)((s1 - c0) < kTile ? (s1 - c0) : kTile);
-    float acc[8][4];
+    float acc[2][4][4];
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int u = 0; u < 4; ++u) acc[nt][u] = 0.f;
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[mt][nt][u] = 0.f;
     const uint32_t aM = sM_addr + (uint32_t)(buf * kTile * kLd * 2);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-      uint32_t a0, a1, a2, a3;
-      const int ar = r0 + (m & 1) * 8 + (lane & 7), ak = 16 * kk + (m >> 1) * 8;
-      ldsm_x4(aM + (ar * kLd + ak) * 2, a0, a1, a2, a3);
 #pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t b00, b01, b10, b11;
-        const int br = n0 + 16 * np + (m >> 1) * 8 + (lane & 7), bk = 16 * kk + (m & 1) * 8;
-        ldsm_x4(sB_addr + (br * kLd + bk) * 2, b00, b01, b10, b11);
-        mma16816(acc[2 * np], a0, a1, a2, a3, b00, b01);
-        mma16816(acc[2 * np + 1], a0, a1, a2, a3, b10, b11);
+      for (int mt = 0; mt < 2; ++mt) {
+        uint32_t a0, a1, a2, a3;
+        const int ar = r0 + 16 * mt + (m & 1) * 8 + (lane & 7), ak = 16 * kk + (m >> 1) * 8;
+        ldsm_x4(aM + (ar * kLd + ak) * 2, a0, a1, a2, a3);
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+          mma16816(acc[mt][2 * np], a0, a1, a2, a3, bfrag[kk][np][0], bfrag[kk][np][1]);
+          mma16816(acc[mt][2 * np + 1], a0, a1, a2, a3, bfrag[kk][np][2], bfrag[kk][np][3]);
+        }
       }
     }
     __nv_bfloat16* tU = sU + buf * kTile * kLd;
     float* out32 = reinterpret_cast<float*>(a.out);
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
+    for (int q = 0; q < 8; ++q) {
+      const int mt = q >> 2, nt = q & 3;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        const int r = r0 + g + 8 * hh, j = n0 + 8 * nt + 2 * t;
+        const int r = r0 + 16 * mt + g + 8 * hh, j = n0 + 8 * nt + 2 * t;
         uint32_t* cell = reinterpret_cast<uint32_t*>(tU + r * kLd + j);
         const float2 u = unpack_bf16(*cell);
-        const float y0 = acc[nt][2 * hh] + u.x, y1 = acc[nt][2 * hh + 1] + u.y;
+        const float y0 = acc[mt][nt][2 * hh] + u.x, y1 = acc[mt][nt][2 * hh + 1] + u.y;
         if (a.out_bf16)
           *cell = pack_bf16(y0, y1);
         else if (r < L)
