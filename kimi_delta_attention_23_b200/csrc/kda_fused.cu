@@ -582,8 +582,29 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
 
     fence_async_smem();  // the operand tiles are read by the tensor cores
     __syncthreads();  // (2) operand tiles, block factors and diagonal scores in place
-
-
+    // the first state-side product needs only [K o Gamma ; Q o Gamma] and the chunk's incoming
+    // state(s): it runs under the off-diagonal scores (sharing the tensor pipe with them costs
+    // less than issuing it later, under the inverse's own products)
+    if (tid == kMmaThread) {
+      tc_fence_after();
+      if constexpr (!kBuild) {
+        // D1 = S^T [K o Gamma ; Q o Gamma]^T   (M = 128, N = 128, K = 128)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(128), kk > 0);
+        }
+      } else {
+        // D1_M = S_M^T (K o Gamma)^T and D1_U = S_U^T (K o Gamma)^T   (N = 64 each, K = 128)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
+          mma_bf16_ts(tmD1u, tmSbu + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
+        }
+      }
+      mma_commit(bar0);
+    }
     // =============================== k-side, part 2: off-diagonal scores on mma.sync
     {
       const int g = lane >> 2, t = lane & 3, m = lane >> 3;
@@ -689,29 +710,30 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       const int g = lane >> 2, t = lane & 3;
       auto lval = [&](int r, int c) { return sBeta[r] * sA[r * kLdA + c]; };
       if (warp >= 4) {
-        // warps 4..7 have no part in the first doubling level: one thread issues the first
-        // state-side product, which needs only [K o Gamma ; Q o Gamma] (complete since (2))
-        // and the chunk's incoming state(s); it runs while the inverse is finished
-        if (tid == kMmaThread) {
+        // warps 4..7 have no part in the first doubling level: they run the state side's first
+        // epilogue (the first product was issued after (2)); warp -> TMEM lane quadrant warp % 4,
+        // all 64 columns.  Y^T[j][r] = -D1[j][r] = -((K o Gamma) S0)^T into the X tile(s); V
+        // enters in the next product
+        if (!mbar_wait_bounded(bar0, phase, kWaitLimitNs)) {
+          *s_abort = 1;
+          report(a.status, KDA_ERR_DEVICE_TIMEOUT);
+        } else {
           tc_fence_after();
-          if constexpr (!kBuild) {
-            // D1 = S^T [K o Gamma ; Q o Gamma]^T   (M = 128, N = 128, K = 128)
+#pragma unroll 1
+          for (int st = 0; st < (kBuild ? 2 : 1); ++st) {
+            float d[64];
+            tmem_ld16n<4>((st ? tmD1u : tmD1) + lane_base, d);
+            tmem_wait_ld();
+            const uint32_t xoff = (kBuild && st == 0) ? OFF_XM : OFF_X;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(128), kk > 0);
-            }
-          } else {
-            // D1_M = S_M^T (K o Gamma)^T and D1_U = S_U^T (K o Gamma)^T   (N = 64 each, K = 128)
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
-              mma_bf16_ts(tmD1u, tmSbu + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
-            }
+            for (int r0 = 0; r0 < 64; r0 += 8)
+              *reinterpret_cast<uint4*>(sm + xoff + sw_off(ej, r0, 128)) =
+                  make_uint4(pack_bf16(-d[r0], -d[r0 + 1]), pack_bf16(-d[r0 + 2], -d[r0 + 3]),
+                             pack_bf16(-d[r0 + 4], -d[r0 + 5]), pack_bf16(-d[r0 + 6], -d[r0 + 7]));
           }
-          mma_commit(bar0);
         }
+        fence_async_smem();
+        tc_fence_before();
       } else {
         // level 1: warp -> (problem, 8-column tile); problem 0 = X10, problem 1 = X32
         const int ra = (warp >> 1) ? 3 : 1, cb = 16 * (ra - 1), R0 = 16 * ra, n0 = 8 * (warp & 1);
@@ -804,29 +826,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     }
 
     if constexpr (!kBuild) {
-    // =============================== state side (the first product was issued in the inverse)
-    {
-      // epilogues run on all eight warps: warps w and w + 4 share TMEM lane quadrant w % 4
-      // (state row j) and split the columns
-      if (!mbar_wait_bounded(bar0, phase, kWaitLimitNs)) {
-        *s_abort = 1;
-        report(a.status, KDA_ERR_DEVICE_TIMEOUT);
-      } else {
-        tc_fence_after();
-        // Y^T[j][r] = -D1[j][r] = -((K o Gamma) S0)^T; V enters in the next product
-        float d[32];
-        tmem_ld16n<2>(tmD1 + lane_base + 32 * ehalf, d);
-        tmem_wait_ld();
-#pragma unroll
-        for (int r0 = 0; r0 < 32; r0 += 8)
-          *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(ej, 32 * ehalf + r0, 128)) =
-              make_uint4(pack_bf16(-d[r0], -d[r0 + 1]), pack_bf16(-d[r0 + 2], -d[r0 + 3]),
-                         pack_bf16(-d[r0 + 4], -d[r0 + 5]), pack_bf16(-d[r0 + 6], -d[r0 + 7]));
-      }
-      fence_async_smem();
-      tc_fence_before();
-    }
-    __syncthreads();
+    // =============================== state side (the first product was issued after (2) and its
+    // epilogue ran during the inverse)
     if (*s_abort) {
       aborted = true;
       break;
@@ -999,30 +1000,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     }
     } else {
     // =============================== state side (segment build: both states; the first
-    // products were issued in the inverse)
+    // products were issued after (2) and their epilogues ran during the inverse)
     {
-      if (!mbar_wait_bounded(bar0, phase, kWaitLimitNs)) {
-        *s_abort = 1;
-        report(a.status, KDA_ERR_DEVICE_TIMEOUT);
-      } else {
-        tc_fence_after();
-        float d[32], e[32];
-        tmem_ld16n<2>(tmD1 + lane_base + 32 * ehalf, d);
-        tmem_ld16n<2>(tmD1u + lane_base + 32 * ehalf, e);
-        tmem_wait_ld();
-#pragma unroll
-        for (int r0 = 0; r0 < 32; r0 += 8) {
-          *reinterpret_cast<uint4*>(sm + OFF_XM + sw_off(ej, 32 * ehalf + r0, 128)) =
-              make_uint4(pack_bf16(-d[r0], -d[r0 + 1]), pack_bf16(-d[r0 + 2], -d[r0 + 3]),
-                         pack_bf16(-d[r0 + 4], -d[r0 + 5]), pack_bf16(-d[r0 + 6], -d[r0 + 7]));
-          *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(ej, 32 * ehalf + r0, 128)) =
-              make_uint4(pack_bf16(-e[r0], -e[r0 + 1]), pack_bf16(-e[r0 + 2], -e[r0 + 3]),
-                         pack_bf16(-e[r0 + 4], -e[r0 + 5]), pack_bf16(-e[r0 + 6], -e[r0 + 7]));
-        }
-      }
-      fence_async_smem();
-      tc_fence_before();
-      __syncthreads();
       if (*s_abort) {
         aborted = true;
         break;
