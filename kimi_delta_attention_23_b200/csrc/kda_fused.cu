@@ -93,6 +93,18 @@ __device__ __forceinline__ uint32_t sw_off(int row, int k, int rows) {
                     ((kin & 7) << 1));
 }
 
+__device__ __forceinline__ void put_t1(uint8_t* sm_t, int r, int s, float v) {
+  *reinterpret_cast<__nv_bfloat16*>(sm_t + sw_off(r, s, 64)) = __float2bfloat16_rn(v);
+}
+__device__ __forceinline__ void put_t2(uint8_t* sm_t, int r, int s, float v0, float v1) {
+  *reinterpret_cast<uint32_t*>(sm_t + sw_off(r, s, 64)) = pack_bf16(v0, v1);
+}
+
+// T = X diag(beta) is written in bf16 as each block of the inverse X is completed; one entry, or
+// two consecutive ones (s even), of the 64 x 64 tile (K-major, 128B swizzle)
+__device__ __forceinline__ void put_t1(uint8_t* sm_t, int r, int s, float v);
+__device__ __forceinline__ void put_t2(uint8_t* sm_t, int r, int s, float v0, float v1);
+
 __device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
   return make_uint2(pack_bf16(a, b), pack_bf16(c, d));
 }
@@ -259,6 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   // there, so it is cleared once
   if constexpr (kRead)
     for (int e = tid; e < 8192 / 16; e += kThreads) reinterpret_cast<uint4*>(sm + OFF_P)[e] = make_uint4(0, 0, 0, 0);
+  // likewise T's upper triangle: the inverse writes only entries s <= r
+  for (int e = tid; e < 8192 / 16; e += kThreads) reinterpret_cast<uint4*>(sm + OFF_T)[e] = make_uint4(0, 0, 0, 0);
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -701,10 +715,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         float xv = 0.f;
 #pragma unroll
         for (int l = 0; l < 8; ++l) xv = fmaf(xblk(rb8, i, l), Yb[m * 64 + l * 8 + j], xv);
+        const float xa = xblk(ra, i, j), xb = xblk(rb8, i, j);
         Xi[(rb8 + i) * kLdA + ra + j] = -xv;
-        Xi[(ra + i) * kLdA + ra + j] = xblk(ra, i, j);
-        Xi[(rb8 + i) * kLdA + rb8 + j] = xblk(rb8, i, j);
+        Xi[(ra + i) * kLdA + ra + j] = xa;
+        Xi[(rb8 + i) * kLdA + rb8 + j] = xb;
         Xi[(ra + i) * kLdA + rb8 + j] = 0.f;
+        // this 16-block of T = X diag(beta) (its upper triangle stays zero from the launch)
+        put_t1(sm + OFF_T, rb8 + i, ra + j, -xv * sBeta[ra + j]);
+        if (j <= i) {
+          put_t1(sm + OFF_T, ra + i, ra + j, xa * sBeta[ra + j]);
+          put_t1(sm + OFF_T, rb8 + i, rb8 + j, xb * sBeta[rb8 + j]);
+        }
       }
       __syncthreads();
       const int g = lane >> 2, t = lane & 3;
@@ -765,6 +786,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         Xi[(R0 + g) * kLdA + cb + n0 + 2 * t + 1] = -xo[1];
         Xi[(R0 + g + 8) * kLdA + cb + n0 + 2 * t] = -xo[2];
         Xi[(R0 + g + 8) * kLdA + cb + n0 + 2 * t + 1] = -xo[3];
+        const int s0 = cb + n0 + 2 * t;
+        const float b0 = sBeta[s0], b1 = sBeta[s0 + 1];
+        put_t2(sm + OFF_T, R0 + g, s0, -xo[0] * b0, -xo[1] * b1);
+        put_t2(sm + OFF_T, R0 + g + 8, s0, -xo[2] * b0, -xo[3] * b1);
       }
       __syncthreads();
       {
@@ -797,24 +822,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
                        to_tf32(Xi[(R0 + g + 8) * kLdA + 32 + k0 + t + 4]), to_tf32(Y2[(k0 + t) * 32 + n0 + g]),
                        to_tf32(Y2[(k0 + t + 4) * 32 + n0 + g]));
         }
-        Xi[(R0 + g) * kLdA + n0 + 2 * t] = -xo[0];
-        Xi[(R0 + g) * kLdA + n0 + 2 * t + 1] = -xo[1];
-        Xi[(R0 + g + 8) * kLdA + n0 + 2 * t] = -xo[2];
-        Xi[(R0 + g + 8) * kLdA + n0 + 2 * t + 1] = -xo[3];
-      }
-      __syncthreads();
-      // T[r][s] = X[r][s] beta_s for s <= r, else 0; bf16 tile [r][s]
-      for (int idx = tid; idx < 64 * 8; idx += kThreads) {
-        const int r = idx >> 3, sc = idx & 7;
-        float tv[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int s = sc * 8 + u;
-          tv[u] = s <= r ? Xi[r * kLdA + s] * sBeta[s] : 0.f;
-        }
-        *reinterpret_cast<uint4*>(sm + OFF_T + sw_off(r, sc * 8, 64)) =
-            make_uint4(pack_bf16(tv[0], tv[1]), pack_bf16(tv[2], tv[3]), pack_bf16(tv[4], tv[5]),
-                       pack_bf16(tv[6], tv[7]));
+        // the last block of X: only T is needed from here on
+        const int s0 = n0 + 2 * t;
+        const float b0 = sBeta[s0], b1 = sBeta[s0 + 1];
+        put_t2(sm + OFF_T, R0 + g, s0, -xo[0] * b0, -xo[1] * b1);
+        put_t2(sm + OFF_T, R0 + g + 8, s0, -xo[2] * b0, -xo[3] * b1);
       }
     }
     fence_async_smem();
