@@ -134,11 +134,14 @@ __global__ void __launch_bounds__(kThreads, 2) cp_apply_kernel(ApplyArgs a) {
     if (cur.seg != loaded_seg || cur.h != loaded_h) {
       const float4* S = reinterpret_cast<const float4*>(a.incoming + ((size_t)cur.seg * Hv + cur.h) * (size_t)(D * D));
       for (int e = tid; e < D * D / 4; e += kThreads) {
-        const float4 x = S[e];
-        const int row = e >> 5, col = (e & 31) * 4;  // four consecutive elements of one stored row
-        if (a.v_first) {  // stored [j][j']: a row of sB
+        if (a.v_first) {  // stored [j][j']: four consecutive elements of a row of sB
+          const float4 x = S[e];
+          const int row = e >> 5, col = (e & 31) * 4;
           *reinterpret_cast<uint2*>(sB + row * kLd + col) = make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
-        } else {  // stored [j'][j]: a column of sB
+        } else {  // stored [j'][j]: columns of sB; consecutive lanes take consecutive stored rows,
+                  // so each 2-byte store instruction hits 32 consecutive elements of a row of sB
+          const int row = e & (D - 1), col = (e >> 7) * 4;
+          const float4 x = S[row * (D / 4) + (col >> 2)];
           sB[(col + 0) * kLd + row] = __float2bfloat16_rn(x.x);
           sB[(col + 1) * kLd + row] = __float2bfloat16_rn(x.y);
           sB[(col + 2) * kLd + row] = __float2bfloat16_rn(x.z);
