@@ -1042,22 +1042,25 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       }
       // decay both states while the second products run (they read neither state):
       // S^T[j][i] *= Gamma_63[i]
-#pragma unroll 1
-      for (int st = 0; st < 2; ++st) {
-        const uint32_t tcol = (st ? tmSu : tmS) + lane_base + 64 * ehalf;
-        float sv[64];
-        tmem_ld16n<4>(tcol, sv);
+      {
+        float sm_[64], su_[64];  // both states' 64 columns, one wide load each, one wait
+        tmem_ld64(tmS + lane_base + 64 * ehalf, sm_);
+        tmem_ld64(tmSu + lane_base + 64 * ehalf, su_);
         tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 64; u += 4) {
           const float4 gv = *reinterpret_cast<const float4*>(sGC + 64 * ehalf + u);
-          sv[u] *= gv.x;
-          sv[u + 1] *= gv.y;
-          sv[u + 2] *= gv.z;
-          sv[u + 3] *= gv.w;
+          sm_[u] *= gv.x;
+          sm_[u + 1] *= gv.y;
+          sm_[u + 2] *= gv.z;
+          sm_[u + 3] *= gv.w;
+          su_[u] *= gv.x;
+          su_[u + 1] *= gv.y;
+          su_[u + 2] *= gv.z;
+          su_[u + 3] *= gv.w;
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_st16(tcol + 16 * q, *reinterpret_cast<const float(*)[16]>(sv + 16 * q));
+        tmem_st64(tmS + lane_base + 64 * ehalf, sm_);
+        tmem_st64(tmSu + lane_base + 64 * ehalf, su_);
       }
       if (!mbar_wait_bounded(bar1, phase, kWaitLimitNs)) {
         *s_abort = 1;
@@ -1157,19 +1160,20 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       } else {
         tc_fence_after();
         // bf16 copies of both new states for the next chunk's first products
-#pragma unroll 1
-        for (int st = 0; st < 2; ++st) {
+        {
           const int i0 = 64 * ehalf;
-          float sv[64];
-          tmem_ld16n<4>((st ? tmSu : tmS) + lane_base + i0, sv);
+          float sm_[64], su_[64];  // both states' 64 columns, one wide load each, one wait
+          tmem_ld64(tmS + lane_base + i0, sm_);
+          tmem_ld64(tmSu + lane_base + i0, su_);
           tmem_wait_ld();
+          uint32_t pm[32], pu[32];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t pk[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) pk[u] = pack_bf16(sv[16 * q + 2 * u], sv[16 * q + 2 * u + 1]);
-            tmem_st8u((st ? tmSbu : tmSb) + lane_base + i0 / 2 + 8 * q, pk);
+          for (int u = 0; u < 32; ++u) {
+            pm[u] = pack_bf16(sm_[2 * u], sm_[2 * u + 1]);
+            pu[u] = pack_bf16(su_[2 * u], su_[2 * u + 1]);
           }
+          tmem_st32u(tmSb + lane_base + i0 / 2, pm);
+          tmem_st32u(tmSbu + lane_base + i0 / 2, pu);
         }
         tmem_wait_st();
       }
