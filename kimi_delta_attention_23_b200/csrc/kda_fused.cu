@@ -870,7 +870,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       {
         const int i0 = 64 * ehalf;
         float sv[64];
-        tmem_ld16n<4>(tmS + lane_base + i0, sv);
+        tmem_ld64(tmS + lane_base + i0, sv);
         tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 64; u += 4) {
@@ -880,9 +880,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           sv[u + 2] *= gv.z;
           sv[u + 3] *= gv.w;
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          tmem_st16(tmS + lane_base + i0 + 16 * q, *reinterpret_cast<const float(*)[16]>(sv + 16 * q));
+        tmem_st64(tmS + lane_base + i0, sv);
       }
       if (!mbar_wait_bounded(bar1, phase, kWaitLimitNs)) {
         *s_abort = 1;
@@ -966,15 +964,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         {
           const int i0 = 64 * ehalf;
           float sv[64];
-          tmem_ld16n<4>(tmS + lane_base + i0, sv);
+          tmem_ld64(tmS + lane_base + i0, sv);
           tmem_wait_ld();
+          uint32_t pk[32];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t pk[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) pk[u] = pack_bf16(sv[16 * q + 2 * u], sv[16 * q + 2 * u + 1]);
-            tmem_st8u(tmSb + lane_base + i0 / 2 + 8 * q, pk);
-          }
+          for (int u = 0; u < 32; ++u) pk[u] = pack_bf16(sv[2 * u], sv[2 * u + 1]);
+          tmem_st32u(tmSb + lane_base + i0 / 2, pk);
           tmem_wait_st();
         }
       }
