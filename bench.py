@@ -108,10 +108,21 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_source_hash():
+# the sources each recorded kernel is built from (its DRAM traffic holds while they are unchanged)
+KERNEL_SOURCES = {
+    "fused_chunk_kernel<build,readout> + affine_scan_kernel": [
+        "kda_fused.cu", "kda_simt.cu", "kda_api.cu", "kda_sm100.cuh", "kda_common.cuh", "kda_internal.h"],
+    "fused_chunk_kernel<prefill>": ["kda_fused.cu", "kda_api.cu", "kda_sm100.cuh", "kda_common.cuh",
+                                    "kda_internal.h"],
+    "decode_kernel": ["kda_decode.cu", "kda_api.cu", "kda_common.cuh", "kda_internal.h"],
+}
+
+
+def kernel_source_hash(kernel=None):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kimi_delta_attention_23_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    names = KERNEL_SOURCES.get(kernel) or sorted(os.listdir(csrc))
+    for name in sorted(names):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -125,7 +136,7 @@ def recorded_traffic(kernel):
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return float(e["dram_bytes_per_launch"])
 
