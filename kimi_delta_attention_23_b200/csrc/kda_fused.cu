@@ -312,8 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const float x = xs[c];
-          // softplus(x) in log2 units, then alpha = exp(-exp(a_log) softplus(x)) = 2^(-c sp2)
-          const float sp2 = fmaxf(x, 0.f) * kLog2e + fast_lg2(1.f + fast_ex2(-fabsf(x) * kLog2e));
+          // softplus(x) in log2 units, log2(1 + 2^(x log2 e)), then alpha = exp(-exp(a_log)
+          // softplus(x)) = 2^(-c sp2); the limits come out right on both sides (x large: the power
+          // overflows to inf and alpha = 0; x very negative: it flushes to 0 and alpha = 1)
+          const float sp2 = fast_lg2(1.f + fast_ex2(x * kLog2e));
           const float al_c = fast_ex2(-cexp * sp2);
           o[c] = safe ? fmaxf(al_c, alpha_floor) : al_c;
         }
@@ -438,31 +440,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
               __float2bfloat16_rn(acc[u]);
         }
       }
-    }
-    // the inverse of this 8-row block's diagonal part, X = (I + diag(beta) A_blk)^{-1} (unit
-    // lower triangular): lane j < 8 runs the forward substitution of column j; the strictly lower
-    // part goes to the block's upper triangle of sA (never read as A), transposed
-    __syncwarp();
-    if (lane < 8) {
-      const int j = lane, base = warp * 8;
-      float lb[8][8], bb[8];  // the block's strictly lower scores and its betas, loaded up front
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        bb[r] = sBeta[base + r];
-#pragma unroll
-        for (int c = 0; c < r; ++c) lb[r][c] = sA[(base + r) * kLdA + base + c];
-      }
-      float x[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        float acc = 0.f;
-#pragma unroll
-        for (int c = 0; c < r; ++c) acc = fmaf(lb[r][c], x[c], acc);
-        x[r] = r < j ? 0.f : (r == j ? 1.f : -bb[r] * acc);
-      }
-#pragma unroll
-      for (int r = 1; r < 8; ++r)
-        if (r > j) sA[(base + j) * kLdA + base + r] = x[r];
     }
     // in-block products: p8 inclusive prefix from the block start, s8 exclusive suffix
     float p8[8][4], s8[8][4];
@@ -662,6 +639,32 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
                   pack_bf16(accP[nt][2 * hlf], accP[nt][2 * hlf + 1]);
           }
         }
+        if (warp == 0 || warp == 2) {
+          // the inverses of the diagonal 8x8 blocks, X = (I + diag(beta) A_blk)^{-1} (unit lower
+          // triangular), on the two warps whose score pairs are adjacent (the lightest): four
+          // blocks per warp, lane -> (block, column j) runs the forward substitution of column j;
+          // the strictly lower part goes to the block's upper triangle of sA (never read as A),
+          // transposed
+          const int j = lane & 7, base = 8 * ((warp >> 1) * 4 + (lane >> 3));
+          float lb[8][8], bb[8];  // the block's strictly lower scores and its betas, loaded up front
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            bb[r] = sBeta[base + r];
+#pragma unroll
+            for (int c = 0; c < r; ++c) lb[r][c] = sA[(base + r) * kLdA + base + c];
+          }
+          float x[8];
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            float acc = 0.f;
+#pragma unroll
+            for (int c = 0; c < r; ++c) acc = fmaf(lb[r][c], x[c], acc);
+            x[r] = r < j ? 0.f : (r == j ? 1.f : -bb[r] * acc);
+          }
+#pragma unroll
+          for (int r = 1; r < 8; ++r)
+            if (r > j) sA[(base + j) * kLdA + base + r] = x[r];
+        }
       } else {
         // rows 8..15 x columns 0..7 inside each 16-block, reference point between the halves
 #pragma unroll 1
@@ -699,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       float* Xi = reinterpret_cast<float*>(sm + OFF_XI);
       float* Yb = reinterpret_cast<float*>(sm + OFF_Y);  // per-warp 16x8 tiles, then [32][32]
       {
-        // the 16-blocks from their 8-blocks a = 2m, b = 2m + 1 (inverted in the diagonal phase,
+        // the 16-blocks from their 8-blocks a = 2m, b = 2m + 1 (inverted during the off-diagonal scores,
         // stored transposed above the diagonal of sA): X_ba = -X_bb (L_ba X_aa); thread ->
         // (16-block m, row i, column j) of the 8 x 8 products
         const int m = tid >> 6, i = (tid >> 3) & 7, j = tid & 7;
