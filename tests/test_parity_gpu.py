@@ -137,6 +137,36 @@ def test_bf16_fp32_output():
     check(w, out, pool, TOL_BF16)
 
 
+def test_bf16_grouped_heads_v_first():
+    # two key heads shared by eight value heads ("max.nn.state_space.kda_chunk": num_key_heads for
+    # q/k, num_value_heads for v, gates, beta and state); key head of value head h is h // 4
+    w = W.random_inputs([150, 70, 64], 2, 8, 128, 128, seed=41, state_std=0.1, state_layout="V_FIRST",
+                        max_slots=5, state_indices=torch.tensor([4, 0, 2], dtype=torch.int32))
+    out, pool = gpu_forward(w)
+    check(w, out, pool, TOL_BF16)
+
+
+def test_bf16_strong_decay_original_gate():
+    # raw_gate ~ N(0, 3) with exp(a_log) up to 16: single steps decay by e^-60 and more, so
+    # in-chunk decay products span far beyond the fp32 range -- every factor the kernel forms
+    # is a product of decays (<= 1) and must neither overflow nor lose the surviving terms
+    w = W.random_inputs([333, 190], 2, 2, 128, 128, seed=42, state_std=0.1, raw_std=3.0)
+    out, pool = gpu_forward(w)
+    check(w, out, pool, TOL_BF16)
+
+
+def test_bf16_unit_query_equals_key_with_beta_one_reads_back_v():
+    # closed form of the step: with q_t = k_t (unit) and beta = 1 the readout after the delta write
+    # is k_t^T S_t = v_t exactly, whatever the decay and the earlier state
+    w = W.random_inputs([200, 77], 2, 2, 128, 128, seed=43, state_std=0.3, raw_std=1.0)
+    w.q = w.k.clone()
+    w.beta_mode = "probability"
+    w.beta_logits = torch.ones_like(w.beta_logits)
+    out, _ = gpu_forward(w)
+    v = w.v.double().numpy()
+    assert rel_l2(out.double().cpu().numpy(), v) <= TOL_BF16
+
+
 # ------------------------------------------------------------------------------------------
 # Full-size workloads (the benchmark's launch configuration), sampled heads
 # ------------------------------------------------------------------------------------------
