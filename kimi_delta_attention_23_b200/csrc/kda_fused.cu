@@ -460,6 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     }
     *reinterpret_cast<float4*>(sTau + warp * D + ch) = make_float4(p8[7][0], p8[7][1], p8[7][2], p8[7][3]);
     if (tid == kPfThread) bulk_wait_read_all();  // the previous chunk's staged outputs were read
+    tmem_wait_st();  // the previous chunk's bf16 state copies have landed in TMEM
+    tc_fence_before();
     __syncthreads();  // (1) block products visible; prefetched inputs consumed; output flushed
     if (*s_abort) {
       aborted = true;
@@ -973,7 +975,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
 #pragma unroll
           for (int u = 0; u < 32; ++u) pk[u] = pack_bf16(sv[2 * u], sv[2 * u + 1]);
           tmem_st32u(tmSb + lane_base + i0 / 2, pk);
-          tmem_wait_st();
+          // (completion is awaited before barrier (1) of the next chunk: its first product is
+          // issued after (2))
         }
       }
       fence_async_smem();
@@ -1172,8 +1175,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           }
           tmem_st32u(tmSb + lane_base + i0 / 2, pm);
           tmem_st32u(tmSbu + lane_base + i0 / 2, pu);
+          // (completion is awaited before barrier (1) of the next chunk: its first products are
+          // issued after (2))
         }
-        tmem_wait_st();
       }
       fence_async_smem();
       tc_fence_before();
@@ -1229,6 +1233,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       }
     }
   }
+  tmem_wait_st();  // the last bf16 state copies
   if (pf_pending) mbar_wait_bounded(bar_pf, pf_parity, kWaitLimitNs);  // copies still in flight
   if (v_pending) mbar_wait_bounded(bar_v, v_parity, kWaitLimitNs);
   if (tid == kPfThread) bulk_wait_all();  // output tensor stores
