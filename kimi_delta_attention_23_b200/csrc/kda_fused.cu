@@ -43,7 +43,12 @@ using namespace sm100;
 constexpr int C = 64;          // chunk length
 constexpr int D = 128;         // dk = dv
 constexpr int kThreads = 256;
-constexpr int kMmaThread = 128;
+// the tensor-core products of a chunk are issued by four threads in four warps, so that no
+// warp carries all of the issue work (one thread per group of products; each commits its own)
+constexpr int kIssueFirst = 192;   // D1 = S^T [K o Gamma ; Q o Gamma]^T          (warp 6)
+constexpr int kIssueDelta = 224;   // Delta = (V - (K o Gamma) S0) T             (warp 7)
+constexpr int kIssueRead = 128;    // readouts / outputs                          (warp 4)
+constexpr int kIssueUpdate = 160;  // state updates S += K'^T Delta               (warp 5)
 constexpr int kPfThread = 160;
 constexpr uint32_t kTmemCols = 512;  // D1 [0,128), S fp32 [128,256), S bf16 A operand [256,320)
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far beyond any legitimate wait
@@ -170,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     mbar_init(bar0, 1);
     mbar_init(bar1, 1);
     mbar_init(bar2, 1);
-    mbar_init(bar3, 1);
+    mbar_init(bar3, 4);
     mbar_init(bar_pf, 1);
     mbar_init(bar4, 1);
     mbar_init(bar_v, 1);
@@ -578,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     // the first state-side product needs only [K o Gamma ; Q o Gamma] and the chunk's incoming
     // state(s): it runs under the off-diagonal scores (sharing the tensor pipe with them costs
     // less than issuing it later, under the inverse's own products)
-    if (tid == kMmaThread) {
+    if (tid == kIssueFirst) {
       tc_fence_after();
       if constexpr (!kBuild) {
         // D1 = S^T [K o Gamma ; Q o Gamma]^T   (M = 128, N = 128, K = 128)
@@ -851,7 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     }
 
     // D1[:, 0:64] = V^T T^T + Y^T T^T = (V - (K o Gamma) S0)^T T^T = Delta^T   (N = 64, K = 64)
-    if (tid == kMmaThread) {
+    if (tid == kIssueDelta) {
       tc_fence_after();
       if (has_v && !mbar_wait_bounded(bar_v, v_parity, kWaitLimitNs)) {  // this chunk's V has landed
         *s_abort = 1;
@@ -920,14 +925,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       v_pending = has_v;
     }
 
-    // D1[:, 64:128] += Delta^T P^T ;  S^T += Delta^T K'   (accumulate)
-    if (tid == kMmaThread) {
+    // D1[:, 64:128] += Delta^T P^T ;  S^T += Delta^T K'   (accumulate; two issuing threads)
+    if (tid == kIssueRead) {
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmD1 + 64, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128(sbase + OFF_P + kk * 32),
                  idesc_bf16_f32(64), 1);
       mma_commit(bar2);
+    }
+    if (tid == kIssueUpdate) {
+      tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmS, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128(sbase + OFF_KPT + kk * 32),
@@ -1021,7 +1029,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       }
 
       // Delta_M^T = Y_M^T T^T ;  Delta_U^T = V^T T^T + Y_U^T T^T
-      if (tid == kMmaThread) {
+      if (tid == kIssueDelta) {
         tc_fence_after();
         if (!mbar_wait_bounded(bar_v, v_parity, kWaitLimitNs)) {  // this chunk's V has landed
           *s_abort = 1;
@@ -1100,7 +1108,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
 
       // [readouts: D_st = S_st,0^T (Q o Gamma)^T + Delta_st^T P^T -- the bf16 copies still hold the
       //  chunk's incoming states]   S_M^T += Delta_M^T K' ;  S_U^T += Delta_U^T K'
-      if (tid == kMmaThread) {
+      if (kRead && tid == kIssueRead) {
         tc_fence_after();
         if constexpr (kRead) {
 #pragma unroll 1
@@ -1119,6 +1127,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           }
           mma_commit(bar2);
         }
+      }
+      if (tid == kIssueUpdate) {
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(tmS, desc_sw128(sbase + OFF_XM + kk * 32), desc_sw128(sbase + OFF_KPT + kk * 32),
@@ -1237,8 +1248,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   if (pf_pending) mbar_wait_bounded(bar_pf, pf_parity, kWaitLimitNs);  // copies still in flight
   if (v_pending) mbar_wait_bounded(bar_v, v_parity, kWaitLimitNs);
   if (tid == kPfThread) bulk_wait_all();  // output tensor stores
-  if (aborted && tid == kMmaThread) {
-    // let any MMA still in flight finish before the tensor memory is released
+  if (aborted && (tid == kIssueFirst || tid == kIssueDelta || tid == kIssueRead || tid == kIssueUpdate)) {
+    // let any MMA still in flight finish before the tensor memory is released (bar3 counts the
+    // four issuing threads' commits)
     mma_commit(bar3);
     mbar_wait_bounded(bar3, 0, kWaitLimitNs);
   }
