@@ -174,10 +174,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   if (tid == 0) {
     mbar_init(bar0, 1);
     mbar_init(bar1, 1);
-    mbar_init(bar2, 1);
+    mbar_init(bar2, kBuild ? 2 : 1);  // build: one commit per state
     mbar_init(bar3, 4);
     mbar_init(bar_pf, 1);
-    mbar_init(bar4, 1);
+    mbar_init(bar4, kBuild ? 2 : 1);
     mbar_init(bar_v, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -1108,36 +1108,33 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
 
       // [readouts: D_st = S_st,0^T (Q o Gamma)^T + Delta_st^T P^T -- the bf16 copies still hold the
       //  chunk's incoming states]   S_M^T += Delta_M^T K' ;  S_U^T += Delta_U^T K'
-      if (kRead && tid == kIssueRead) {
+      // one issuing thread per state for each group (warps 4 / 6 the readouts of M / U, warps
+      // 5 / 7 their updates); bar2 and bar4 count the two commits of their group
+      if (kRead && (tid == kIssueRead || tid == kIssueFirst)) {
         tc_fence_after();
         if constexpr (kRead) {
-#pragma unroll 1
-          for (int st = 0; st < 2; ++st) {
-            const uint32_t dcol = st ? tmD1u : tmD1, acol = st ? tmSbu : tmSb;
-            const uint32_t xoff = st ? OFF_X : OFF_XM;
+          const int st = tid == kIssueFirst ? 1 : 0;
+          const uint32_t dcol = st ? tmD1u : tmD1, acol = st ? tmSbu : tmSb;
+          const uint32_t xoff = st ? OFF_X : OFF_XM;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32 + 8192;  // rows 64..127: Q o Gamma
-              mma_bf16_ts(dcol, acol + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
-            }
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(dcol, desc_sw128(sbase + xoff + kk * 32), desc_sw128(sbase + OFF_P + kk * 32),
-                       idesc_bf16_f32(64), 1);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32 + 8192;  // rows 64..127: Q o Gamma
+            mma_bf16_ts(dcol, acol + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
           }
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(dcol, desc_sw128(sbase + xoff + kk * 32), desc_sw128(sbase + OFF_P + kk * 32),
+                     idesc_bf16_f32(64), 1);
           mma_commit(bar2);
         }
       }
-      if (tid == kIssueUpdate) {
+      if (tid == kIssueUpdate || tid == kIssueDelta) {
         tc_fence_after();
+        const bool u = tid == kIssueDelta;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmS, desc_sw128(sbase + OFF_XM + kk * 32), desc_sw128(sbase + OFF_KPT + kk * 32),
-                   idesc_bf16_f32(128), 1);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(tmSu, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128(sbase + OFF_KPT + kk * 32),
-                   idesc_bf16_f32(128), 1);
+          mma_bf16(u ? tmSu : tmS, desc_sw128(sbase + (u ? OFF_X : OFF_XM) + kk * 32),
+                   desc_sw128(sbase + OFF_KPT + kk * 32), idesc_bf16_f32(128), 1);
         mma_commit(bar4);
       }
       // the next chunk's gates run on the CUDA cores while these products are on the tensor cores
