@@ -17,6 +17,7 @@
 // values it yields the transition M_i; started at 0 with the real values it yields U_i.
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "kda_sm100.cuh"
 
 namespace kda {
 
@@ -269,7 +270,7 @@ __global__ void compose128_kernel(ComposeArgs a);
 
 cudaError_t launch_affine_scan(const ScanArgs& a, cudaStream_t stream) {
   if (tiles128(a.dk, a.dv)) {
-    const int smem = (2 * 128 * 132 + 128 * 32) * (int)sizeof(float);
+    const int smem = (2 * 128 * 132 + 2 * 128 * 40) * (int)sizeof(float);  // M double buffer, carried tile parts
     cudaError_t err = cudaFuncSetAttribute(affine_scan128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     affine_scan128_kernel<<<dim3(a.H, a.dv / 32), 256, smem, stream>>>(a);
@@ -381,7 +382,7 @@ __global__ void __launch_bounds__(kScanThreads) compose_pieces_kernel(ComposeArg
 
 cudaError_t launch_compose_pieces(const ComposeArgs& a, cudaStream_t stream) {
   if (tiles128(a.dk, a.dv)) {
-    const int smem = (128 * 132 + 128 * 32) * (int)sizeof(float);
+    const int smem = (128 * 132 + 2 * 128 * 40) * (int)sizeof(float);  // M, carried tile parts
     cudaError_t err = cudaFuncSetAttribute(compose128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     compose128_kernel<<<dim3(a.H, 4 + a.dv / 32, a.N), 256, smem, stream>>>(a);
@@ -397,13 +398,17 @@ cudaError_t launch_compose_pieces(const ComposeArgs& a, cudaStream_t stream) {
 }
 
 // ------------------------------------------------------------------------------------------
-// dk = 128 forms of the scan and of the composition: 128 x 32 tiles, M staged row-major in
-// shared memory by 16-byte asynchronous copies (double-buffered along the scan), thread t owning
-// rows t/8 + 32 i (i < 4) and columns 4 (t % 8) .. + 3 (sixteen accumulators; each M element
-// read from shared memory feeds four of them, each float4 of the carried tile sixteen).
+// dk = 128 forms of the scan and of the composition: 128 x 32 tiles.  M is staged row-major in
+// shared memory by 16-byte asynchronous copies (double-buffered along the scan).  The tile
+// product runs on the tensor cores as tf32 mma.sync (m16n8k8) with the three-term split
+// a b = a_hi b_hi + a_hi b_lo + a_lo b_hi (a_hi = a rounded to tf32, a_lo = the remainder, also
+// rounded; the dropped a_lo b_lo is below fp32 rounding), so the products keep fp32 accuracy.
+// Thread ownership is the MMA accumulator fragment: warp w owns rows 16 w + g and 16 w + g + 8
+// (g = lane / 4), columns 8 n + 2 t and + 1 (t = lane % 4, n < 4) -- sixteen values.
 // ------------------------------------------------------------------------------------------
 constexpr int kT = 32;          // tile columns
-constexpr int kLdM = 132;       // padded row of the staged M: 16-byte rows, conflict-free column reads
+constexpr int kLdM = 132;       // padded row of the staged M: 16-byte rows, conflict-free fragment reads
+constexpr int kLdC = 40;        // padded row of the carried tile's two parts: conflict-free fragment reads
 constexpr int kTileThreads = 256;
 
 __device__ __forceinline__ void cp_async16_g2s(float* dst, const float* src) {
@@ -423,50 +428,93 @@ __device__ __forceinline__ void stage_m(float* Ms, const float* Mg) {
   cp_async_commit_group();
 }
 
-// acc[i][u] = sum_l Ms[rows_i][l] cur[l][c0 + u]
-__device__ __forceinline__ void tile_product(const float* Ms, const float* cur, float acc[4][4]) {
-  const int rb = threadIdx.x >> 3, c0 = (threadIdx.x & 7) * 4;
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+  uint32_t u;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(u) : "f"(x));
+  return u;
+}
+
+// the carried 128 x 32 tile X, as its tf32 high part (chi) and rounded remainder (clo), from this
+// thread's fragment x[n][c]
+__device__ __forceinline__ void put_carried(float* chi, float* clo, const float (&x)[4][4]) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int n = 0; n < 4; ++n)
 #pragma unroll
-    for (int u = 0; u < 4; ++u) acc[i][u] = 0.f;
-  // four columns of M per step: one 16-byte load per row (conflict-free with the 132-float
-  // padding), four 16-byte loads of the carried tile, 64 fused multiply-adds
-#pragma unroll 2
-  for (int l = 0; l < 128; l += 4) {
-    float4 mr[4];
+    for (int hh = 0; hh < 2; ++hh) {
+      const int r = 16 * w + g + 8 * hh, c = 8 * n + 2 * t;
+      const float a = x[n][2 * hh], b = x[n][2 * hh + 1];
+      const float ah = __uint_as_float(tf32_rna(a)), bh = __uint_as_float(tf32_rna(b));
+      *reinterpret_cast<float2*>(chi + r * kLdC + c) = make_float2(ah, bh);
+      *reinterpret_cast<float2*>(clo + r * kLdC + c) =
+          make_float2(__uint_as_float(tf32_rna(a - ah)), __uint_as_float(tf32_rna(b - bh)));
+    }
+}
+
+// acc = Ms (128 x 128, row-major, stride kLdM) times X (128 x 32, held as chi + clo)
+__device__ __forceinline__ void tile_product_tc(const float* Ms, const float* chi, const float* clo,
+                                                float (&acc)[4][4]) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) mr[i] = *reinterpret_cast<const float4*>(Ms + (rb + 32 * i) * kLdM + l);
+  for (int n = 0; n < 4; ++n)
 #pragma unroll
-    for (int dl = 0; dl < 4; ++dl) {
-      const float4 b = *reinterpret_cast<const float4*>(cur + (l + dl) * kT + c0);
+    for (int u = 0; u < 4; ++u) acc[n][u] = 0.f;
+  const float* a0p = Ms + (16 * w + g) * kLdM;
+  const float* a1p = a0p + 8 * kLdM;
+#pragma unroll 4
+  for (int k0 = 0; k0 < 128; k0 += 8) {
+    const float av[4] = {a0p[k0 + t], a1p[k0 + t], a0p[k0 + t + 4], a1p[k0 + t + 4]};
+    uint32_t ah[4], al[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float m = dl == 0 ? mr[i].x : dl == 1 ? mr[i].y : dl == 2 ? mr[i].z : mr[i].w;
-        acc[i][0] = fmaf(m, b.x, acc[i][0]);
-        acc[i][1] = fmaf(m, b.y, acc[i][1]);
-        acc[i][2] = fmaf(m, b.z, acc[i][2]);
-        acc[i][3] = fmaf(m, b.w, acc[i][3]);
-      }
+    for (int i = 0; i < 4; ++i) {
+      ah[i] = tf32_rna(av[i]);
+      al[i] = tf32_rna(av[i] - __uint_as_float(ah[i]));
+    }
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      const int c = 8 * n + g;
+      const uint32_t bh0 = __float_as_uint(chi[(k0 + t) * kLdC + c]), bh1 = __float_as_uint(chi[(k0 + t + 4) * kLdC + c]);
+      const uint32_t bl0 = __float_as_uint(clo[(k0 + t) * kLdC + c]), bl1 = __float_as_uint(clo[(k0 + t + 4) * kLdC + c]);
+      sm100::mma1688_tf32(acc[n], al[0], al[1], al[2], al[3], bh0, bh1);
+      sm100::mma1688_tf32(acc[n], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+      sm100::mma1688_tf32(acc[n], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
     }
   }
 }
 
-// four consecutive columns j0 + c0 .. + 3 of row r of a state block in either layout
-__device__ __forceinline__ float4 load_state4(const float* blk, int r, int j, int dv, int v_first) {
-  if (!v_first) return *reinterpret_cast<const float4*>(blk + (size_t)r * dv + j);
-  return make_float4(blk[(size_t)j * 128 + r], blk[(size_t)(j + 1) * 128 + r], blk[(size_t)(j + 2) * 128 + r],
-                     blk[(size_t)(j + 3) * 128 + r]);
+// two consecutive columns j, j + 1 of row r of a state block in either layout
+__device__ __forceinline__ float2 load_state2(const float* blk, int r, int j, int dv, int v_first) {
+  if (!v_first) return *reinterpret_cast<const float2*>(blk + (size_t)r * dv + j);
+  return make_float2(blk[(size_t)j * 128 + r], blk[(size_t)(j + 1) * 128 + r]);
 }
-__device__ __forceinline__ void store_state4(float* blk, int r, int j, int dv, int v_first, float4 x) {
+__device__ __forceinline__ void store_state2(float* blk, int r, int j, int dv, int v_first, float2 x) {
   if (!v_first) {
-    *reinterpret_cast<float4*>(blk + (size_t)r * dv + j) = x;
+    *reinterpret_cast<float2*>(blk + (size_t)r * dv + j) = x;
   } else {
     blk[(size_t)j * 128 + r] = x.x;
     blk[(size_t)(j + 1) * 128 + r] = x.y;
-    blk[(size_t)(j + 2) * 128 + r] = x.z;
-    blk[(size_t)(j + 3) * 128 + r] = x.w;
   }
+}
+// this thread's fragment of columns j0 .. j0 + 31 of a state block
+__device__ __forceinline__ void load_frag(float (&x)[4][4], const float* blk, int j0, int dv, int v_first) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int n = 0; n < 4; ++n)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const float2 v = load_state2(blk, 16 * w + g + 8 * hh, j0 + 8 * n + 2 * t, dv, v_first);
+      x[n][2 * hh] = v.x;
+      x[n][2 * hh + 1] = v.y;
+    }
+}
+__device__ __forceinline__ void store_frag(float* blk, const float (&x)[4][4], int j0, int dv, int v_first) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int n = 0; n < 4; ++n)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+      store_state2(blk, 16 * w + g + 8 * hh, j0 + 8 * n + 2 * t, dv, v_first,
+                   make_float2(x[n][2 * hh], x[n][2 * hh + 1]));
 }
 
 // the exclusive scan (as affine_scan_kernel) for dk = 128: one block per (head, 32 columns)
@@ -474,25 +522,20 @@ __global__ void __launch_bounds__(kTileThreads, 1) affine_scan128_kernel(ScanArg
   extern __shared__ __align__(16) float smf[];
   float* Ms0 = smf;
   float* Ms1 = Ms0 + 128 * kLdM;
-  float* cur = Ms1 + 128 * kLdM;  // [128][kT]
+  float* chi = Ms1 + 128 * kLdM;  // [128][kLdC] the carried tile, tf32 high part
+  float* clo = chi + 128 * kLdC;  // and remainder
   const int h = blockIdx.x, j0 = blockIdx.y * kT, H = a.H, dv = a.dv, vf = a.v_first;
   const size_t st = (size_t)128 * dv;
-  const int rb = threadIdx.x >> 3, c0 = (threadIdx.x & 7) * 4;
   if (a.N > 0) stage_m(Ms0, a.M + (size_t)h * 128 * 128);
-  float4 x[4];  // this thread's part of the carried state
-#pragma unroll
-  for (int i = 0; i < 4; ++i) x[i] = load_state4(a.initial + (size_t)h * st, rb + 32 * i, j0 + c0, dv, vf);
+  float x[4][4];  // this thread's part of the carried state
+  load_frag(x, a.initial + (size_t)h * st, j0, dv, vf);
   for (int s = 0; s < a.N; ++s) {
     float* Ms = (s & 1) ? Ms1 : Ms0;
     const size_t blk = ((size_t)s * H + h) * st;
-    float4 u[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = rb + 32 * i;
-      *reinterpret_cast<float4*>(cur + r * kT + c0) = x[i];
-      if (a.incoming) store_state4(a.incoming + blk, r, j0 + c0, dv, vf, x[i]);
-      u[i] = load_state4(a.U + blk, r, j0 + c0, dv, vf);
-    }
+    float u[4][4];
+    put_carried(chi, clo, x);
+    if (a.incoming) store_frag(a.incoming + blk, x, j0, dv, vf);
+    load_frag(u, a.U + blk, j0, dv, vf);
     if (s + 1 < a.N) {
       stage_m((s & 1) ? Ms0 : Ms1, a.M + ((size_t)(s + 1) * H + h) * 128 * 128);
       cp_async_wait_groups<1>();
@@ -501,17 +544,15 @@ __global__ void __launch_bounds__(kTileThreads, 1) affine_scan128_kernel(ScanArg
     }
     __syncthreads();  // M_s staged, the carried tile complete
     float acc[4][4];
-    tile_product(Ms, cur, acc);
+    tile_product_tc(Ms, chi, clo, acc);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      x[i] = make_float4(acc[i][0] + u[i].x, acc[i][1] + u[i].y, acc[i][2] + u[i].z, acc[i][3] + u[i].w);
-      if (a.outgoing) store_state4(a.outgoing + blk, rb + 32 * i, j0 + c0, dv, vf, x[i]);
-    }
-    __syncthreads();  // every read of cur and of M_s is done
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) x[n][c] = acc[n][c] + u[n][c];
+    if (a.outgoing) store_frag(a.outgoing + blk, x, j0, dv, vf);
+    __syncthreads();  // every read of the carried tile and of M_s is done
   }
-  if (a.final_state)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) store_state4(a.final_state + (size_t)h * st, rb + 32 * i, j0 + c0, dv, vf, x[i]);
+  if (a.final_state) store_frag(a.final_state + (size_t)h * st, x, j0, dv, vf);
 }
 
 // the composition (as compose_pieces_kernel) for dk = 128: one block per (head, 32 columns of
@@ -519,52 +560,53 @@ __global__ void __launch_bounds__(kTileThreads, 1) affine_scan128_kernel(ScanArg
 __global__ void __launch_bounds__(kTileThreads, 2) compose128_kernel(ComposeArgs a) {
   extern __shared__ __align__(16) float smf[];
   float* Ms = smf;
-  float* cur = Ms + 128 * kLdM;
+  float* chi = Ms + 128 * kLdM;
+  float* clo = chi + 128 * kLdC;
   const int h = blockIdx.x, seg = blockIdx.z, H = a.H, dv = a.dv, vf = a.v_first, k = a.k;
   const int nbm = 128 / kT;
   const bool is_m = (int)blockIdx.y < nbm;
   const int j0 = (is_m ? (int)blockIdx.y : (int)blockIdx.y - nbm) * kT;
   const size_t st = (size_t)128 * dv;
-  const int rb = threadIdx.x >> 3, c0 = (threadIdx.x & 7) * 4;
   const size_t first = (size_t)seg * k;
-  float4 x[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = rb + 32 * i;
-    x[i] = is_m ? *reinterpret_cast<const float4*>(a.M + (first * H + h) * 128 * 128 + (size_t)r * 128 + j0 + c0)
-                : load_state4(a.U + (first * H + h) * st, r, j0 + c0, dv, vf);
-  }
+  float x[4][4];
+  if (is_m)
+    load_frag(x, a.M + (first * H + h) * 128 * 128, j0, 128, 0);  // M is row-major [128][128]
+  else
+    load_frag(x, a.U + (first * H + h) * st, j0, dv, vf);
   for (int p = 1; p < k; ++p) {
     const size_t piece = first + p;
     stage_m(Ms, a.M + (piece * H + h) * 128 * 128);
-    float4 u[4];
+    float u[4][4];
+    put_carried(chi, clo, x);
+    if (is_m) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = rb + 32 * i;
-      *reinterpret_cast<float4*>(cur + r * kT + c0) = x[i];
-      u[i] = is_m ? make_float4(0.f, 0.f, 0.f, 0.f) : load_state4(a.U + (piece * H + h) * st, r, j0 + c0, dv, vf);
+      for (int n = 0; n < 4; ++n)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) u[n][c] = 0.f;
+    } else {
+      load_frag(u, a.U + (piece * H + h) * st, j0, dv, vf);
     }
     cp_async_wait_groups<0>();
     __syncthreads();
     float acc[4][4];
-    tile_product(Ms, cur, acc);
+    tile_product_tc(Ms, chi, clo, acc);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      x[i] = make_float4(acc[i][0] + u[i].x, acc[i][1] + u[i].y, acc[i][2] + u[i].z, acc[i][3] + u[i].w);
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) x[n][c] = acc[n][c] + u[n][c];
     __syncthreads();
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = rb + 32 * i, j = j0 + c0;
-    const size_t ob = ((size_t)seg * H + h) * st;
-    if (is_m) {
-      *reinterpret_cast<float4*>(a.M_out + ((size_t)seg * H + h) * 128 * 128 + (size_t)r * 128 + j) = x[i];
-    } else {
-      store_state4(a.U_out + ob, r, j, dv, vf, x[i]);
-      store_state4(a.incoming + ob, r, j, dv, vf, load_state4(a.inc + (first * H + h) * st, r, j, dv, vf));
-      const float* nxt = seg + 1 < a.N ? a.inc + ((size_t)(seg + 1) * k * H + h) * st : a.final_state + (size_t)h * st;
-      store_state4(a.outgoing + ob, r, j, dv, vf, load_state4(nxt, r, j, dv, vf));
-    }
+  const size_t ob = ((size_t)seg * H + h) * st;
+  if (is_m) {
+    store_frag(a.M_out + ((size_t)seg * H + h) * 128 * 128, x, j0, 128, 0);
+  } else {
+    store_frag(a.U_out + ob, x, j0, dv, vf);
+    float y[4][4];
+    load_frag(y, a.inc + (first * H + h) * st, j0, dv, vf);
+    store_frag(a.incoming + ob, y, j0, dv, vf);
+    const float* nxt = seg + 1 < a.N ? a.inc + ((size_t)(seg + 1) * k * H + h) * st : a.final_state + (size_t)h * st;
+    load_frag(y, nxt, j0, dv, vf);
+    store_frag(a.outgoing + ob, y, j0, dv, vf);
   }
 }
 
@@ -680,29 +722,24 @@ __global__ void __launch_bounds__(kTileThreads, 1) pool_scan128_kernel(PoolScanA
   extern __shared__ __align__(16) float smf[];
   float* Ms0 = smf;
   float* Ms1 = Ms0 + 128 * kLdM;
-  float* cur = Ms1 + 128 * kLdM;
+  float* chi = Ms1 + 128 * kLdM;
+  float* clo = chi + 128 * kLdC;
   const int h = blockIdx.x, j0 = blockIdx.y * kT, b = blockIdx.z, H = a.H, dv = a.dv, vf = a.v_first;
   const size_t st = (size_t)128 * dv;
-  const int rb = threadIdx.x >> 3, c0 = (threadIdx.x & 7) * 4;
   const int p0 = a.seq_first[b], p1 = a.seq_first[b + 1];
   const int32_t slot = a.slots ? a.slots[b] : b;
   float* blk = a.pool + ((size_t)slot * H + h) * st;
   if (p1 > p0) stage_m(Ms0, a.M + ((size_t)p0 * H + h) * 128 * 128);
-  float4 x[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) x[i] = load_state4(blk, rb + 32 * i, j0 + c0, dv, vf);
+  float x[4][4];
+  load_frag(x, blk, j0, dv, vf);
   for (int p = p0; p < p1; ++p) {
     const int s = p - p0;
     float* Ms = (s & 1) ? Ms1 : Ms0;
     const size_t pb = ((size_t)p * H + h) * st;
-    float4 u[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = rb + 32 * i;
-      *reinterpret_cast<float4*>(cur + r * kT + c0) = x[i];
-      store_state4(a.incoming + pb, r, j0 + c0, dv, vf, x[i]);
-      u[i] = load_state4(a.U + pb, r, j0 + c0, dv, vf);
-    }
+    float u[4][4];
+    put_carried(chi, clo, x);
+    store_frag(a.incoming + pb, x, j0, dv, vf);
+    load_frag(u, a.U + pb, j0, dv, vf);
     if (p + 1 < p1) {
       stage_m((s & 1) ? Ms0 : Ms1, a.M + ((size_t)(p + 1) * H + h) * 128 * 128);
       cp_async_wait_groups<1>();
@@ -711,18 +748,18 @@ __global__ void __launch_bounds__(kTileThreads, 1) pool_scan128_kernel(PoolScanA
     }
     __syncthreads();
     float acc[4][4];
-    tile_product(Ms, cur, acc);
+    tile_product_tc(Ms, chi, clo, acc);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      x[i] = make_float4(acc[i][0] + u[i].x, acc[i][1] + u[i].y, acc[i][2] + u[i].z, acc[i][3] + u[i].w);
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) x[n][c] = acc[n][c] + u[n][c];
     __syncthreads();
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) store_state4(blk, rb + 32 * i, j0 + c0, dv, vf, x[i]);
+  store_frag(blk, x, j0, dv, vf);
 }
 
 cudaError_t launch_pool_scan(const PoolScanArgs& a, cudaStream_t stream) {
-  const int smem = (2 * 128 * kLdM + 128 * kT) * (int)sizeof(float);
+  const int smem = (2 * 128 * kLdM + 2 * 128 * kLdC) * (int)sizeof(float);
   cudaError_t err = cudaFuncSetAttribute(pool_scan128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   if (a.batch == 0) return cudaSuccess;
