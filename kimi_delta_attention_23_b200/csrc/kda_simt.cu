@@ -529,13 +529,19 @@ __global__ void __launch_bounds__(kTileThreads, 1) affine_scan128_kernel(ScanArg
   if (a.N > 0) stage_m(Ms0, a.M + (size_t)h * 128 * 128);
   float x[4][4];  // this thread's part of the carried state
   load_frag(x, a.initial + (size_t)h * st, j0, dv, vf);
+  float un[4][4];  // the next step's contribution, loaded one step ahead
+  if (a.N > 0) load_frag(un, a.U + (size_t)h * st, j0, dv, vf);
   for (int s = 0; s < a.N; ++s) {
     float* Ms = (s & 1) ? Ms1 : Ms0;
     const size_t blk = ((size_t)s * H + h) * st;
     float u[4][4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) u[n][c] = un[n][c];
+    if (s + 1 < a.N) load_frag(un, a.U + ((size_t)(s + 1) * H + h) * st, j0, dv, vf);
     put_carried(chi, clo, x);
     if (a.incoming) store_frag(a.incoming + blk, x, j0, dv, vf);
-    load_frag(u, a.U + blk, j0, dv, vf);
     if (s + 1 < a.N) {
       stage_m((s & 1) ? Ms0 : Ms1, a.M + ((size_t)(s + 1) * H + h) * 128 * 128);
       cp_async_wait_groups<1>();
@@ -732,14 +738,20 @@ __global__ void __launch_bounds__(kTileThreads, 1) pool_scan128_kernel(PoolScanA
   if (p1 > p0) stage_m(Ms0, a.M + ((size_t)p0 * H + h) * 128 * 128);
   float x[4][4];
   load_frag(x, blk, j0, dv, vf);
+  float un[4][4];  // the next piece's contribution, loaded one step ahead
+  if (p1 > p0) load_frag(un, a.U + ((size_t)p0 * H + h) * st, j0, dv, vf);
   for (int p = p0; p < p1; ++p) {
     const int s = p - p0;
     float* Ms = (s & 1) ? Ms1 : Ms0;
     const size_t pb = ((size_t)p * H + h) * st;
     float u[4][4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) u[n][c] = un[n][c];
+    if (p + 1 < p1) load_frag(un, a.U + ((size_t)(p + 1) * H + h) * st, j0, dv, vf);
     put_carried(chi, clo, x);
     store_frag(a.incoming + pb, x, j0, dv, vf);
-    load_frag(u, a.U + pb, j0, dv, vf);
     if (p + 1 < p1) {
       stage_m((s & 1) ? Ms0 : Ms1, a.M + ((size_t)(p + 1) * H + h) * 128 * 128);
       cp_async_wait_groups<1>();
