@@ -33,6 +33,11 @@
  *    stack as the state pool and state_indices = 0..N-1 then produces every segment's
  *    outputs in parallel; afterwards that pool holds the outgoing states.
  *
+ *  kda_context_parallel_range_summary / kda_context_parallel_range_finish
+ *    The same method across GPUs: each rank reduces its own token range of the sequence to one
+ *    affine map, the caller gathers the maps and scans them over the ranks, and each rank
+ *    finishes its range from the state entering it.
+ *
  * Conventions shared by every call
  *  - All tensor pointers are DEVICE pointers owned by the caller, row-major and densely
  *    packed in the stated shapes.  The library allocates no device memory.
@@ -311,6 +316,51 @@ KDA_API kda_status_t kda_context_parallel_piece_offsets(const int32_t *seg_offse
  * current device's SM count: query it with the device current that will run the prefill. */
 KDA_API size_t kda_context_parallel_workspace_preferred(int64_t T, int32_t num_segments,
                                                         int32_t num_v_heads, int32_t dv);
+
+/*
+ * Context parallelism across GPUs ("KDA Context Parallelism", Theory: a segment summarised as the
+ * affine map F(S) = M S + U is applied to any incoming state without replaying its tokens;
+ * Compose segments in sequence order; Incoming and outgoing states).  One long sequence is cut
+ * into consecutive token ranges, one per rank (GPU); a rank holds only its own range's tokens
+ * and cuts that range into its own segments.  Per rank, in this order:
+ *   1. kda_context_parallel_range_summary: the range built (as chunk-aligned pieces, all in
+ *      parallel, with per-token readouts kept in the workspace) and composed into ONE map of the
+ *      whole range, range_M [Hv,128,128] and range_U [Hv,<state>];
+ *   2. the caller gathers every rank's map in rank order (an all-gather; the library makes no
+ *      collective call) and runs the exclusive scan over the ranks from the sequence's initial
+ *      state (kda_segment_summarize_and_scan with KDA_SEG_SCAN_ONLY): incoming[r] is the state
+ *      entering rank r's range and the scan's final state is the sequence's final state;
+ *   3. kda_context_parallel_range_finish: from the state entering the range, the pieces'
+ *      incoming states (the exclusive scan over the pieces), the summary and the incoming and
+ *      outgoing states of each of the range's segments, and the outputs of every token.
+ * Steps 1 and 3 use the same workspace (>= kda_context_parallel_range_workspace_size bytes,
+ * 256-byte aligned), which the caller leaves untouched in between, on the same device, with the
+ * same T, num_segments, num_v_heads and layout flag.  bf16 q/k/v with dk = dv = 128 only.
+ * With one rank the three steps give what kda_context_parallel_prefill gives.
+ *
+ *   q, k, v, raw_gate, beta_logits, a_log, dt_bias   the range's tokens, as kda_chunk_fwd (T may
+ *     be 0: the map is then the identity and zero, and the token pointers may be NULL)
+ *   seg_offsets [num_segments + 1] int32 device, 0 .. T, non-decreasing (the range's segments)
+ *   range_M, range_U  fp32, written by step 1
+ *   range_incoming [Hv,<state>] fp32, read by step 3;  range_outgoing [Hv,<state>] fp32 written
+ *     by step 3 (nullable): the state leaving the range
+ *   out [T,Hv,128] out_dtype;  M [N,Hv,128,128], U / incoming / outgoing [N,Hv,<state>] fp32,
+ *     written by step 3, as kda_context_parallel_prefill's
+ * A bad offset is reported in device_status (KDA_ERR_DEVICE_CHECK) and its piece skipped.
+ */
+KDA_API size_t kda_context_parallel_range_workspace_size(int64_t T, int32_t num_segments,
+                                                         int32_t num_v_heads, int32_t dv);
+KDA_API kda_status_t kda_context_parallel_range_summary(
+    const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype, const float *raw_gate,
+    const float *beta_logits, const float *a_log, const float *dt_bias, int64_t T,
+    int32_t num_k_heads, int32_t num_v_heads, int32_t dk, int32_t dv, const int32_t *seg_offsets,
+    int32_t num_segments, float *range_M, float *range_U, uint32_t flags, float gate_lower_bound,
+    void *workspace, size_t workspace_bytes, int32_t *device_status, void *stream);
+KDA_API kda_status_t kda_context_parallel_range_finish(
+    int64_t T, int32_t num_v_heads, int32_t dk, int32_t dv, int32_t num_segments,
+    const float *range_incoming, void *out, kda_dtype_t out_dtype, float *range_outgoing, float *M,
+    float *U, float *incoming, float *outgoing, uint32_t flags, void *workspace,
+    size_t workspace_bytes, int32_t *device_status, void *stream);
 
 /* Bytes of workspace with which kda_chunk_fwd may take its split route on the current device
  * (0 when the batch has chains enough for the SMs, for dk or dv other than 128, or with

@@ -11,6 +11,10 @@ Public calls (same names as the C ABI):
   kda_context_parallel(M, U, initial)     the scan alone, returning exactly incoming_states,
                                           outgoing_states and final_state
   kda_context_parallel_prefill(...)       the context-parallel prefill of one long sequence
+  kda_context_parallel_range_summary(...) one rank's token range of a sequence as one map
+  kda_context_parallel_range_finish(...)  that range's outputs from the state entering it
+                                          (``distributed.context_parallel_prefill`` joins the
+                                          two across ranks with one all-gather)
 """
 from __future__ import annotations
 
@@ -22,7 +26,8 @@ import torch
 __all__ = ["kda_chunk_fwd", "kda_decode", "kda_segment_summarize_and_scan", "kda_context_parallel",
            "kda_context_parallel_apply", "kda_context_parallel_prefill", "kda_context_parallel_workspace_size",
            "kda_context_parallel_workspace_preferred", "kda_context_parallel_pieces",
-           "kda_context_parallel_piece_offsets", "kda_segment_compose", "kda_workspace_size",
+           "kda_context_parallel_piece_offsets", "kda_segment_compose", "kda_context_parallel_range_workspace_size",
+           "kda_context_parallel_range_summary", "kda_context_parallel_range_finish", "kda_workspace_size",
            "kda_status_string", "load_library", "KdaError", "LIB_PATH"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -84,6 +89,14 @@ def load_library():
     lib.kda_segment_compose.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, u32, vp]
     lib.kda_context_parallel_workspace_preferred.restype = sz
     lib.kda_context_parallel_workspace_preferred.argtypes = [i64, i32, i32, i32]
+    lib.kda_context_parallel_range_workspace_size.restype = sz
+    lib.kda_context_parallel_range_workspace_size.argtypes = [i64, i32, i32, i32]
+    lib.kda_context_parallel_range_summary.restype = ctypes.c_int
+    lib.kda_context_parallel_range_summary.argtypes = [vp, vp, vp, ctypes.c_int, fp, fp, fp, fp, i64, i32, i32,
+                                                       i32, i32, ip, i32, fp, fp, u32, f32, vp, sz, ip, vp]
+    lib.kda_context_parallel_range_finish.restype = ctypes.c_int
+    lib.kda_context_parallel_range_finish.argtypes = [i64, i32, i32, i32, i32, fp, vp, ctypes.c_int, fp, fp, fp,
+                                                      fp, fp, u32, vp, sz, ip, vp]
     lib.kda_workspace_size.restype = sz
     lib.kda_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32, i32, u32]
     lib.kda_status_string.restype = ctypes.c_char_p
@@ -519,4 +532,104 @@ def kda_context_parallel_prefill(q, k, v, raw_gate, beta_logits, a_log, dt_bias,
     if rc != 0:
         raise KdaError(rc, "kda_context_parallel_prefill")
     return {"out": out, "final_state": final_state, "incoming_states": incoming, "outgoing_states": outgoing,
+            "transition_matrices": M, "local_contributions": U}
+
+
+def kda_context_parallel_range_workspace_size(T, num_segments, num_v_heads, dv=128) -> int:
+    """Workspace bytes of the two per-rank calls on the current device."""
+    return int(load_library().kda_context_parallel_range_workspace_size(T, num_segments, num_v_heads, dv))
+
+
+def _token_ptr(t, T):
+    # a range without tokens passes no token pointers
+    return _ptr(t) if T > 0 else None
+
+
+def kda_context_parallel_range_summary(q, k, v, raw_gate, beta_logits, a_log, dt_bias, seg_offsets, *,
+                                       range_transition=None, range_contribution=None, workspace=None,
+                                       gate_mode="original", beta_mode="logits", state_layout="K_FIRST",
+                                       gate_lower_bound=-5.0, device_status=None, stream=None):
+    """One rank's token range (bf16 q/k/v, dk = dv = 128, cut at seg_offsets) as ONE affine map.
+
+    Returns dict(range_transition [Hv,128,128], range_contribution [Hv,<state>], workspace); the
+    workspace carries the range's readouts and pieces to kda_context_parallel_range_finish.
+    """
+    lib = load_library()
+    dev = q.device
+    _dev(q, "q", torch.bfloat16, dev)
+    T, Hk, dk = q.shape
+    _shape(_dev(k, "k", torch.bfloat16, dev), "k", (T, Hk, dk))
+    _dev(v, "v", torch.bfloat16, dev)
+    Hv, dv = v.shape[1], v.shape[2]
+    _shape(v, "v", (T, Hv, dv))
+    _shape(_dev(raw_gate, "raw_gate", torch.float32, dev), "raw_gate", (T, Hv, dk))
+    _shape(_dev(beta_logits, "beta_logits", torch.float32, dev), "beta_logits", (T, Hv))
+    _shape(_dev(a_log, "a_log", torch.float32, dev), "a_log", (Hv,))
+    _shape(_dev(dt_bias, "dt_bias", torch.float32, dev), "dt_bias", (Hv, dk))
+    _dev(seg_offsets, "seg_offsets", torch.int32, dev)
+    N = seg_offsets.numel() - 1
+    st = (dk, dv) if state_layout == "K_FIRST" else (dv, dk)
+    if range_transition is None:
+        range_transition = torch.empty((Hv, dk, dk), dtype=torch.float32, device=dev)
+    _shape(_dev(range_transition, "range_transition", torch.float32, dev), "range_transition", (Hv, dk, dk))
+    if range_contribution is None:
+        range_contribution = torch.empty((Hv, *st), dtype=torch.float32, device=dev)
+    _shape(_dev(range_contribution, "range_contribution", torch.float32, dev), "range_contribution", (Hv, *st))
+    if workspace is None:
+        with torch.cuda.device(dev):
+            need = kda_context_parallel_range_workspace_size(T, max(N, 1), Hv, dv)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _dev(workspace, "workspace", torch.uint8, dev)
+    rc = lib.kda_context_parallel_range_summary(
+        _token_ptr(q, T), _token_ptr(k, T), _token_ptr(v, T), _BF16, _token_ptr(raw_gate, T),
+        _token_ptr(beta_logits, T), _ptr(a_log), _ptr(dt_bias), T, Hk, Hv, dk, dv, _ptr(seg_offsets), N,
+        _ptr(range_transition), _ptr(range_contribution), _flags(gate_mode, beta_mode, state_layout),
+        float(gate_lower_bound), _ptr(workspace), workspace.numel(), _ptr(device_status), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_context_parallel_range_summary")
+    return {"range_transition": range_transition, "range_contribution": range_contribution, "workspace": workspace}
+
+
+def kda_context_parallel_range_finish(range_incoming, workspace, seg_offsets, tokens, out=None, *,
+                                      output_dtype=torch.bfloat16, range_outgoing=None, M=None, U=None,
+                                      incoming=None, outgoing=None, state_layout="K_FIRST", device_status=None,
+                                      stream=None):
+    """A range's outputs and per-segment states from the state entering it (range_incoming
+    [Hv,<state>] fp32) and the workspace that kda_context_parallel_range_summary filled.
+
+    Returns dict(out, range_outgoing, incoming_states, outgoing_states, transition_matrices,
+    local_contributions) for the range's own segments.
+    """
+    lib = load_library()
+    dev = range_incoming.device
+    _dev(range_incoming, "range_incoming", torch.float32, dev)
+    Hv, st = range_incoming.shape[0], tuple(range_incoming.shape[1:])
+    dk = dv = 128
+    _shape(range_incoming, "range_incoming", (Hv, dk, dv))
+    _dev(workspace, "workspace", torch.uint8, dev)
+    _dev(seg_offsets, "seg_offsets", torch.int32, dev)
+    N = seg_offsets.numel() - 1
+    T = int(tokens)
+    if out is None:
+        out = torch.empty((T, Hv, dv), dtype=output_dtype, device=dev)
+    _shape(_dev(out, "out", output_dtype, dev), "out", (T, Hv, dv))
+
+    def buf(t, name, shape):
+        if t is None:
+            return torch.empty(shape, dtype=torch.float32, device=dev)
+        _shape(_dev(t, name, torch.float32, dev), name, shape)
+        return t
+
+    range_outgoing = buf(range_outgoing, "range_outgoing", (Hv, *st))
+    M = buf(M, "M", (N, Hv, dk, dk))
+    U = buf(U, "U", (N, Hv, *st))
+    incoming = buf(incoming, "incoming", (N, Hv, *st))
+    outgoing = buf(outgoing, "outgoing", (N, Hv, *st))
+    rc = lib.kda_context_parallel_range_finish(
+        T, Hv, dk, dv, N, _ptr(range_incoming), _token_ptr(out, T), _DTYPES[output_dtype], _ptr(range_outgoing),
+        _ptr(M), _ptr(U), _ptr(incoming), _ptr(outgoing), _flags("original", "logits", state_layout),
+        _ptr(workspace), workspace.numel(), _ptr(device_status), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_context_parallel_range_finish")
+    return {"out": out, "range_outgoing": range_outgoing, "incoming_states": incoming, "outgoing_states": outgoing,
             "transition_matrices": M, "local_contributions": U}

@@ -575,6 +575,183 @@ extern "C" kda_status_t kda_context_parallel_prefill(
                                     out_dtype, flags & KDA_STATE_V_FIRST, device_status, stream);
 }
 
+// ------------------------------------------------------------------------------------------
+// Context parallelism across GPUs: each rank holds one range of consecutive segments of the
+// sequence.  The range is built as pieces (with readouts) and composed into one summary; the
+// summaries are exchanged and scanned by the caller; the range is then finished from the state
+// entering it.  The workspace carries the readouts and the pieces' summaries between the two
+// calls.
+// ------------------------------------------------------------------------------------------
+namespace {
+
+struct RangeWorkspace {
+  __nv_bfloat16_raw* o_m;  // [T][Hv][128] readout through the transition
+  __nv_bfloat16_raw* o_u;  // [T][Hv][128] readout of the contribution
+  int32_t* offs;           // [np + 1] piece boundaries
+  float* pM;               // [np][Hv][128][128]
+  float* pU;               // [np][Hv][state]
+  float* pIn;              // [np + 1][Hv][state]: slot p + 1 holds the outgoing state of piece p
+  int32_t np;
+};
+
+size_t range_workspace_bytes(int64_t T, int32_t N, int32_t Hv, int kp) {
+  return round256((size_t)2 * T * Hv * 128 * 2) + pieces_bytes(N, kp, Hv, 128, 128);
+}
+
+RangeWorkspace range_workspace(void* ws, int64_t T, int32_t N, int32_t Hv, int kp) {
+  RangeWorkspace r{};
+  uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  r.np = N * kp;
+  r.o_m = reinterpret_cast<__nv_bfloat16_raw*>(w);
+  r.o_u = r.o_m + (size_t)T * Hv * 128;
+  w += round256((size_t)2 * T * Hv * 128 * 2);
+  r.offs = reinterpret_cast<int32_t*>(w);
+  w += round256((size_t)(r.np + 1) * sizeof(int32_t));
+  r.pM = reinterpret_cast<float*>(w);
+  r.pU = r.pM + (size_t)r.np * Hv * 128 * 128;
+  r.pIn = r.pU + (size_t)r.np * Hv * 128 * 128;
+  return r;
+}
+
+bool range_workspace_ok(const void* ws, size_t bytes, int64_t T, int32_t N, int32_t Hv, int kp) {
+  return ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0 && bytes >= range_workspace_bytes(T, N, Hv, kp);
+}
+
+}  // namespace
+
+extern "C" size_t kda_context_parallel_range_workspace_size(int64_t T, int32_t num_segments, int32_t num_v_heads,
+                                                            int32_t dv) {
+  if (T < 0 || num_segments < 1 || num_v_heads <= 0 || dv != 128) return 0;
+  return range_workspace_bytes(T, num_segments, num_v_heads, choose_pieces(T, num_segments, num_v_heads));
+}
+
+extern "C" kda_status_t kda_context_parallel_range_summary(
+    const void* q, const void* k, const void* v, kda_dtype_t qkv_dtype, const float* raw_gate,
+    const float* beta_logits, const float* a_log, const float* dt_bias, int64_t T, int32_t num_k_heads,
+    int32_t num_v_heads, int32_t dk, int32_t dv, const int32_t* seg_offsets, int32_t num_segments,
+    float* range_M, float* range_U, uint32_t flags, float gate_lower_bound, void* workspace,
+    size_t workspace_bytes, int32_t* device_status, void* stream) {
+  if (num_segments < 1 || T < 0 || num_k_heads <= 0 || num_v_heads <= 0 || dk <= 0 || dv <= 0)
+    return KDA_ERR_INVALID_ARG;
+  if (num_v_heads % num_k_heads != 0) return KDA_ERR_INVALID_ARG;
+  if ((flags & ~kKnownFlags) != 0 || (flags & (KDA_SEG_SCAN_ONLY | KDA_FORCE_SIMT))) return KDA_ERR_INVALID_ARG;
+  if (T > 0 && (!q || !k || !v || !raw_gate || !beta_logits)) return KDA_ERR_INVALID_ARG;
+  if (!a_log || !dt_bias || !seg_offsets || !range_M || !range_U) return KDA_ERR_INVALID_ARG;
+  if (!dtype_ok(qkv_dtype)) return KDA_ERR_UNSUPPORTED;
+  if (qkv_dtype != KDA_BF16 || dk != 128 || dv != 128 || !kda::fused_available()) return KDA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(raw_gate) || !aligned16(dt_bias) ||
+      !aligned16(range_M) || !aligned16(range_U))
+    return KDA_ERR_INVALID_ARG;
+  const int kp = choose_pieces(T, num_segments, num_v_heads);
+  if (!range_workspace_ok(workspace, workspace_bytes, T, num_segments, num_v_heads, kp)) return KDA_ERR_WORKSPACE;
+  const RangeWorkspace L = range_workspace(workspace, T, num_segments, num_v_heads, kp);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (kda::launch_split_offsets(seg_offsets, num_segments, kp, L.offs, s) != cudaSuccess) return KDA_ERR_CUDA;
+  // the pieces in parallel: transition, contribution and both readouts in one launch
+  kda::FusedArgs f{};
+  f.q = q;
+  f.k = k;
+  f.v = v;
+  f.raw_gate = raw_gate;
+  f.beta = beta_logits;
+  f.a_log = a_log;
+  f.dt_bias = dt_bias;
+  f.cu = L.offs;
+  f.batch = L.np;
+  f.total_tokens = T;
+  f.Hk = num_k_heads;
+  f.Hv = num_v_heads;
+  f.max_slots = L.np;
+  f.out = L.o_m;
+  f.out2 = L.o_u;
+  f.out_bf16 = 1;
+  f.flags = flags;
+  f.lb = gate_lower_bound;
+  f.status = device_status;
+  f.build = 1;
+  f.state_out = L.pM;
+  f.state_out2 = L.pU;
+  f.v_first = (flags & KDA_STATE_V_FIRST) ? 1 : 0;
+  if (kda::launch_fused_chunk(f, s) != cudaSuccess) return KDA_ERR_CUDA;
+  // the whole range as one map: the pieces composed in order
+  kda::ComposeArgs ca{};
+  ca.M = L.pM;
+  ca.U = L.pU;
+  ca.inc = nullptr;
+  ca.N = 1;
+  ca.k = L.np;
+  ca.H = num_v_heads;
+  ca.dk = 128;
+  ca.dv = 128;
+  ca.v_first = f.v_first;
+  ca.M_out = range_M;
+  ca.U_out = range_U;
+  return kda::launch_compose_pieces(ca, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" kda_status_t kda_context_parallel_range_finish(
+    int64_t T, int32_t num_v_heads, int32_t dk, int32_t dv, int32_t num_segments, const float* range_incoming,
+    void* out, kda_dtype_t out_dtype, float* range_outgoing, float* M, float* U, float* incoming, float* outgoing,
+    uint32_t flags, void* workspace, size_t workspace_bytes, int32_t* device_status, void* stream) {
+  if (num_segments < 1 || T < 0 || num_v_heads <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+  if ((flags & ~kKnownFlags) != 0) return KDA_ERR_INVALID_ARG;
+  if (!range_incoming || !M || !U || !incoming || !outgoing || (T > 0 && !out)) return KDA_ERR_INVALID_ARG;
+  if (!dtype_ok(out_dtype)) return KDA_ERR_UNSUPPORTED;
+  if (dk != 128 || dv != 128) return KDA_ERR_UNSUPPORTED;
+  if (!aligned16(out)) return KDA_ERR_INVALID_ARG;
+  const int kp = choose_pieces(T, num_segments, num_v_heads);
+  if (!range_workspace_ok(workspace, workspace_bytes, T, num_segments, num_v_heads, kp)) return KDA_ERR_WORKSPACE;
+  const RangeWorkspace L = range_workspace(workspace, T, num_segments, num_v_heads, kp);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int v_first = (flags & KDA_STATE_V_FIRST) ? 1 : 0;
+  const size_t blk = (size_t)num_v_heads * 128 * 128;
+  // the incoming state of every piece, from the state entering the range
+  kda::ScanArgs sa{};
+  sa.M = L.pM;
+  sa.U = L.pU;
+  sa.initial = range_incoming;
+  sa.N = L.np;
+  sa.H = num_v_heads;
+  sa.dk = 128;
+  sa.dv = 128;
+  sa.v_first = v_first;
+  sa.incoming = L.pIn;
+  sa.outgoing = L.pIn + blk;
+  sa.final_state = range_outgoing;
+  if (kda::launch_affine_scan(sa, s) != cudaSuccess) return KDA_ERR_CUDA;
+  // each segment's summary and states from its pieces'
+  kda::ComposeArgs ca{};
+  ca.M = L.pM;
+  ca.U = L.pU;
+  ca.inc = L.pIn;
+  ca.final_state = L.pIn + (size_t)L.np * blk;
+  ca.N = num_segments;
+  ca.k = kp;
+  ca.H = num_v_heads;
+  ca.dk = 128;
+  ca.dv = 128;
+  ca.v_first = v_first;
+  ca.M_out = M;
+  ca.U_out = U;
+  ca.incoming = incoming;
+  ca.outgoing = outgoing;
+  if (kda::launch_compose_pieces(ca, s) != cudaSuccess) return KDA_ERR_CUDA;
+  // the outputs: every piece's readouts with its incoming state
+  kda::ApplyArgs ap{};
+  ap.seg_offsets = L.offs;
+  ap.num_segments = L.np;
+  ap.total_tokens = T;
+  ap.Hv = num_v_heads;
+  ap.incoming = L.pIn;
+  ap.v_first = v_first;
+  ap.o_m = L.o_m;
+  ap.o_u = L.o_u;
+  ap.out = out;
+  ap.out_bf16 = out_dtype == KDA_BF16;
+  ap.status = device_status;
+  return kda::launch_cp_apply(ap, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 extern "C" size_t kda_workspace_size(int64_t total_tokens, int32_t batch, int32_t num_k_heads,
                                      int32_t num_v_heads, int32_t dk, int32_t dv, int32_t num_segments,
                                      uint32_t flags) {

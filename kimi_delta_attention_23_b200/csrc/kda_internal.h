@@ -134,7 +134,8 @@ struct PoolScanArgs {
 struct ComposeArgs {
   const float* M;            // [N*k][H][dk][dk] the pieces' transitions (row-major)
   const float* U;            // [N*k][H][state] the pieces' contributions
-  const float* inc;          // [N*k][H][state] the pieces' incoming states
+  const float* inc;          // [N*k][H][state] the pieces' incoming states, or NULL (then
+                             // final_state, incoming and outgoing are unused)
   const float* final_state;  // [H][state]
   int32_t N, k, H, dk, dv, v_first;
   float* M_out;              // [N][H][dk][dk]

@@ -316,7 +316,8 @@ cudaError_t launch_split_offsets(const int32_t* offs, int32_t N, int32_t k, int3
 // One block per (segment, head, 16-column tile): tiles of M_i (dk columns) carry the product of
 // the pieces' transitions from I; tiles of U_i (dv columns) carry the pieces' affine maps from
 // 0.  The U tiles also copy the segment's incoming state (its first piece's) and outgoing state
-// (the next segment's incoming state, or the final state).
+// (the next segment's incoming state, or the final state), unless the pieces' incoming states
+// are not given (inc == NULL: summaries only).
 __global__ void __launch_bounds__(kScanThreads) compose_pieces_kernel(ComposeArgs a) {
   extern __shared__ float sm[];
   const int h = blockIdx.x, seg = blockIdx.z, tid = threadIdx.x;
@@ -373,6 +374,7 @@ __global__ void __launch_bounds__(kScanThreads) compose_pieces_kernel(ComposeArg
     } else {
       const size_t o = state_off(i, j0 + jj, dk, dv, a.v_first);
       a.U_out[((size_t)seg * H + h) * st + o] = cur[e];
+      if (!a.inc) continue;
       a.incoming[((size_t)seg * H + h) * st + o] = a.inc[((size_t)seg * k * H + h) * st + o];
       a.outgoing[((size_t)seg * H + h) * st + o] =
           seg + 1 < a.N ? a.inc[((size_t)(seg + 1) * k * H + h) * st + o] : a.final_state[(size_t)h * st + o];
@@ -607,6 +609,7 @@ __global__ void __launch_bounds__(kTileThreads, 2) compose128_kernel(ComposeArgs
     store_frag(a.M_out + ((size_t)seg * H + h) * 128 * 128, x, j0, 128, 0);
   } else {
     store_frag(a.U_out + ob, x, j0, dv, vf);
+    if (!a.inc) return;
     float y[4][4];
     load_frag(y, a.inc + (first * H + h) * st, j0, dv, vf);
     store_frag(a.incoming + ob, y, j0, dv, vf);
