@@ -1291,6 +1291,11 @@ bool encode_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint3
 
 }  // namespace
 
+bool encode_token_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t esize, int64_t tokens,
+                       int heads, uint32_t box_x, CUtensorMapSwizzle swz) {
+  return encode_rows(m, base, dt, esize, tokens, heads, box_x, swz);
+}
+
 cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream) {
   cudaError_t err = cudaFuncSetAttribute(fused_chunk_kernel<false, true>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);

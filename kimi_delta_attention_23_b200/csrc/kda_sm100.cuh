@@ -83,6 +83,8 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src_smem
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // the shared-memory sources of every committed store have been read (the tiles may be rewritten)
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// the shared-memory sources of every committed store but the newest group have been read
+__device__ __forceinline__ void bulk_wait_read_prev() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // every committed store has completed
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
