@@ -323,8 +323,9 @@ class Step:
                 self.ws = torch.empty(max(kda.kda_context_parallel_workspace_preferred(T, N, Hv, dv), 1),
                                       dtype=torch.uint8, device=dev)
             else:
-                self.rm = torch.empty((T, Hv, dv), dtype=torch.bfloat16, device=dev)
-                self.ru = torch.empty((T, Hv, dv), dtype=torch.bfloat16, device=dev)
+                # head-major readouts, as the prefill entry keeps them in its workspace
+                self.rm = torch.empty((Hv, T, dv), dtype=torch.bfloat16, device=dev)
+                self.ru = torch.empty((Hv, T, dv), dtype=torch.bfloat16, device=dev)
                 if self.pieces > 1:
                     self.poffs = torch.empty(P + 1, dtype=torch.int32, device=dev)
                     self.pM = torch.empty((P, Hv, dk, dk), device=dev)
@@ -372,7 +373,8 @@ class Step:
             kda.kda_segment_summarize_and_scan(w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias,
                                                self.poffs, self.init, M=self.pM, U=self.pU, incoming=self.pIn[:-1],
                                                outgoing=self.pIn[1:], final_state=self.fin, q=w.q,
-                                               readout_m=self.rm, readout_u=self.ru, **self.kw())
+                                               readout_m=self.rm, readout_u=self.ru, readout_layout="head_major",
+                                               **self.kw())
             if ev:
                 ev[1].record(self.stream)
             kda.kda_segment_compose(self.pM, self.pU, self.pIn, self.fin, self.pieces, M=self.M, U=self.U,
@@ -381,19 +383,19 @@ class Step:
             if ev:
                 ev[2].record(self.stream)
             kda.kda_context_parallel_apply(self.rm, self.ru, self.pIn[:-1], self.poffs, self.out,
-                                           state_layout=w.state_layout, device_status=self.status,
-                                           stream=self.stream)
+                                           readout_layout="head_major", state_layout=w.state_layout,
+                                           device_status=self.status, stream=self.stream)
         elif self.cp:
             kda.kda_segment_summarize_and_scan(w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias,
                                                w.seg_offsets, self.init, M=self.M, U=self.U, incoming=self.inc,
                                                outgoing=self.outg, final_state=self.fin, q=w.q, readout_m=self.rm,
-                                               readout_u=self.ru, **self.kw())
+                                               readout_u=self.ru, readout_layout="head_major", **self.kw())
             if ev:
                 ev[1].record(self.stream)
                 ev[2].record(self.stream)
             kda.kda_context_parallel_apply(self.rm, self.ru, self.inc, w.seg_offsets, self.out,
-                                           state_layout=w.state_layout, device_status=self.status,
-                                           stream=self.stream)
+                                           readout_layout="head_major", state_layout=w.state_layout,
+                                           device_status=self.status, stream=self.stream)
         elif self.decode:
             if ev:
                 ev[1].record(self.stream)

@@ -91,7 +91,9 @@ enum {
   KDA_STATE_V_FIRST = 1u << 2, /* state_layout="V_FIRST": a slot stores S^T as [dv][dk]; else [dk][dv] */
   KDA_FUSED = 1u << 3,         /* use_computebound: accepted; the bf16 path is always the fused kernel */
   KDA_SEG_SCAN_ONLY = 1u << 4, /* segment call: M and U are inputs, only the scan runs           */
-  KDA_FORCE_SIMT = 1u << 5     /* run the fp32 CUDA-core chunk kernel even for bf16 inputs       */
+  KDA_FORCE_SIMT = 1u << 5,    /* run the fp32 CUDA-core chunk kernel even for bf16 inputs       */
+  KDA_READOUT_HEAD_MAJOR = 1u << 6 /* readout_m / readout_u stored [Hv, T, 128] instead of
+                                      [T, Hv, 128] (calls that write or read readouts only)      */
 };
 
 /*
@@ -189,7 +191,8 @@ KDA_API kda_status_t kda_decode(const void *q, const void *k, const void *v, kda
  *   q, readout_m, readout_u  optional (all three or none; bf16 k/v with dk = dv = 128 only):
  *   q [T, Hk, 128] bf16; the build then also writes, per token, the readout through the
  *   transition readout_m[t] = q_t^T M_{<=t} and of the contribution readout_u[t] = q_t^T U_{<=t}
- *   ([T, Hv, 128] bf16 each), the inputs of kda_context_parallel_apply.
+ *   ([T, Hv, 128] bf16 each; [Hv, T, 128] with KDA_READOUT_HEAD_MAJOR, which makes every
+ *   head's rows contiguous for the apply), the inputs of kda_context_parallel_apply.
  */
 KDA_API kda_status_t kda_segment_summarize_and_scan(
     const void *k, const void *v, kda_dtype_t kv_dtype, const float *raw_gate,
@@ -207,7 +210,8 @@ KDA_API kda_status_t kda_segment_summarize_and_scan(
  * M_{<=t} S_in + U_{<=t}, so out_t = readout_m[t] . S_in + readout_u[t] with
  * readout_m[t] = q_t^T M_{<=t} and readout_u[t] = q_t^T U_{<=t}.
  *
- *   readout_m, readout_u [T, Hv, 128] bf16 (from kda_segment_summarize_and_scan)
+ *   readout_m, readout_u [T, Hv, 128] bf16 (from kda_segment_summarize_and_scan), or
+ *     [Hv, T, 128] with KDA_READOUT_HEAD_MAJOR
  *   incoming [N, Hv, <state>] fp32 (flags: KDA_STATE_V_FIRST for the transposed layout)
  *   out [T, Hv, 128] out_dtype
  * dv must be 128; bad segment offsets are reported in device_status and that segment skipped.

@@ -40,6 +40,7 @@ STATE_V_FIRST = 1 << 2
 FUSED = 1 << 3
 SEG_SCAN_ONLY = 1 << 4
 FORCE_SIMT = 1 << 5
+READOUT_HEAD_MAJOR = 1 << 6
 
 _F32, _BF16 = 0, 1
 _DTYPES = {torch.float32: _F32, torch.bfloat16: _BF16}
@@ -131,6 +132,16 @@ def _flags(gate_mode, beta_mode, state_layout, use_computebound=False, force_sim
     f |= FORCE_SIMT if force_simt else 0
     f |= SEG_SCAN_ONLY if scan_only else 0
     return f
+
+
+def _readout_flags(readout_layout):
+    if readout_layout not in ("token_major", "head_major"):
+        raise ValueError(f"readout_layout must be 'token_major' or 'head_major', got {readout_layout!r}")
+    return READOUT_HEAD_MAJOR if readout_layout == "head_major" else 0
+
+
+def _readout_shape(T, Hv, dv, readout_layout):
+    return (Hv, T, dv) if readout_layout == "head_major" else (T, Hv, dv)
 
 
 def _ptr(t):
@@ -278,16 +289,17 @@ def kda_decode(q, k, v, raw_gate, beta_logits, a_log, dt_bias, state_pool, state
 
 def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, seg_offsets, initial_state,
                                    *, M=None, U=None, incoming=None, outgoing=None, final_state=None,
-                                   q=None, readout_m=None, readout_u=None, scan_only=False, gate_mode="original",
-                                   beta_mode="logits", state_layout="K_FIRST", gate_lower_bound=-5.0,
-                                   device_status=None, stream=None):
+                                   q=None, readout_m=None, readout_u=None, readout_layout="token_major",
+                                   scan_only=False, gate_mode="original", beta_mode="logits", state_layout="K_FIRST",
+                                   gate_lower_bound=-5.0, device_status=None, stream=None):
     """Segment summaries (M_i, U_i) of one sequence and the exclusive scan over them.
 
     Returns dict(incoming_states, outgoing_states, final_state, transition_matrices,
     local_contributions[, readout_m, readout_u]); the segment axis leads every stack.  With
     ``scan_only`` the given M and U are inputs and are not written.  With ``q`` (bf16, 128-wide
     heads) the build also returns each token's readouts through the transition and of the
-    contribution, the inputs of ``kda_context_parallel_apply``.
+    contribution, the inputs of ``kda_context_parallel_apply``: [T, Hv, 128] each, or [Hv, T, 128]
+    with ``readout_layout="head_major"`` (every head's rows contiguous; the apply reads them faster).
     """
     lib = load_library()
     dev = initial_state.device
@@ -330,13 +342,16 @@ def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, 
     final_state = buf(final_state, "final_state", (Hv, *st))
     if q is not None:
         _shape(_dev(q, "q", torch.bfloat16, dev), "q", (T, Hk, dk))
+        rshape = _readout_shape(T, Hv, dv, readout_layout)
         if readout_m is None:
-            readout_m = torch.empty((T, Hv, dv), dtype=torch.bfloat16, device=dev)
+            readout_m = torch.empty(rshape, dtype=torch.bfloat16, device=dev)
         if readout_u is None:
-            readout_u = torch.empty((T, Hv, dv), dtype=torch.bfloat16, device=dev)
-        _shape(_dev(readout_m, "readout_m", torch.bfloat16, dev), "readout_m", (T, Hv, dv))
-        _shape(_dev(readout_u, "readout_u", torch.bfloat16, dev), "readout_u", (T, Hv, dv))
+            readout_u = torch.empty(rshape, dtype=torch.bfloat16, device=dev)
+        _shape(_dev(readout_m, "readout_m", torch.bfloat16, dev), "readout_m", rshape)
+        _shape(_dev(readout_u, "readout_u", torch.bfloat16, dev), "readout_u", rshape)
     flags = _flags(gate_mode, beta_mode, state_layout, scan_only=scan_only)
+    if q is not None:
+        flags |= _readout_flags(readout_layout)
     rc = lib.kda_segment_summarize_and_scan(
         _ptr(k) if not scan_only else None, _ptr(v) if not scan_only else None, kv_dtype,
         _ptr(raw_gate) if not scan_only else None, _ptr(beta_logits) if not scan_only else None,
@@ -354,13 +369,18 @@ def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, 
 
 
 def kda_context_parallel_apply(readout_m, readout_u, incoming, seg_offsets, out=None, *, output_dtype=torch.bfloat16,
-                               state_layout="K_FIRST", device_status=None, stream=None):
-    """out_t = readout_m[t] . S_in(segment of t) + readout_u[t] for every token."""
+                               readout_layout="token_major", state_layout="K_FIRST", device_status=None, stream=None):
+    """out_t = readout_m[t] . S_in(segment of t) + readout_u[t] for every token (readouts [T, Hv, 128],
+    or [Hv, T, 128] with ``readout_layout="head_major"``; out [T, Hv, 128] either way)."""
     lib = load_library()
     dev = incoming.device
     _dev(readout_m, "readout_m", torch.bfloat16, dev)
-    T, Hv, dv = readout_m.shape
-    _shape(_dev(readout_u, "readout_u", torch.bfloat16, dev), "readout_u", (T, Hv, dv))
+    rflags = _readout_flags(readout_layout)
+    if readout_layout == "head_major":
+        Hv, T, dv = readout_m.shape
+    else:
+        T, Hv, dv = readout_m.shape
+    _shape(_dev(readout_u, "readout_u", torch.bfloat16, dev), "readout_u", _readout_shape(T, Hv, dv, readout_layout))
     _dev(incoming, "incoming", torch.float32, dev)
     _dev(seg_offsets, "seg_offsets", torch.int32, dev)
     N = seg_offsets.numel() - 1
@@ -368,8 +388,8 @@ def kda_context_parallel_apply(readout_m, readout_u, incoming, seg_offsets, out=
         out = torch.empty((T, Hv, dv), dtype=output_dtype, device=dev)
     _shape(_dev(out, "out", None, dev), "out", (T, Hv, dv))
     rc = lib.kda_context_parallel_apply(_ptr(readout_m), _ptr(readout_u), _ptr(incoming), _ptr(seg_offsets), N, T,
-                                        Hv, dv, _ptr(out), _DTYPES[out.dtype], _flags("original", "logits",
-                                                                                      state_layout),
+                                        Hv, dv, _ptr(out), _DTYPES[out.dtype],
+                                        _flags("original", "logits", state_layout) | rflags,
                                         _ptr(device_status), _stream(stream, dev))
     if rc != 0:
         raise KdaError(rc, "kda_context_parallel_apply")

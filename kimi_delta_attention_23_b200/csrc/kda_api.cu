@@ -17,7 +17,7 @@ bool fused_available();
 namespace {
 
 constexpr uint32_t kKnownFlags = KDA_GATE_SAFE | KDA_BETA_PROB | KDA_STATE_V_FIRST | KDA_FUSED |
-                                 KDA_SEG_SCAN_ONLY | KDA_FORCE_SIMT;
+                                 KDA_SEG_SCAN_ONLY | KDA_FORCE_SIMT | KDA_READOUT_HEAD_MAJOR;
 
 bool dtype_ok(kda_dtype_t t) { return t == KDA_F32 || t == KDA_BF16; }
 
@@ -249,6 +249,7 @@ extern "C" kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* 
   bf.out = o_m;
   bf.out2 = o_u;
   bf.out_bf16 = 1;
+  bf.readout_hm = 1;  // the readouts are this call's own: head-major, contiguous per head
   bf.gate_run_if = 0;
   if (kda::launch_fused_chunk(bf, s) != cudaSuccess) return KDA_ERR_CUDA;
   kda::PoolScanArgs ps{};
@@ -276,6 +277,7 @@ extern "C" kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* 
   ap.out = out;
   ap.out_bf16 = out_dtype == KDA_BF16;
   ap.status = device_status;
+  ap.readout_hm = 1;
   ap.skip_flag = fallback;
   return kda::launch_cp_apply(ap, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
@@ -371,6 +373,7 @@ extern "C" kda_status_t kda_segment_summarize_and_scan(
       f.out = readout_m;
       f.out2 = readout_u;
       f.out_bf16 = 1;
+      f.readout_hm = (flags & KDA_READOUT_HEAD_MAJOR) ? 1 : 0;
       f.flags = flags;
       f.lb = gate_lower_bound;
       f.status = device_status;
@@ -517,6 +520,7 @@ extern "C" kda_status_t kda_context_parallel_apply(const void* readout_m, const 
   ap.out = out;
   ap.out_bf16 = out_dtype == KDA_BF16;
   ap.status = device_status;
+  ap.readout_hm = (flags & KDA_READOUT_HEAD_MAJOR) ? 1 : 0;
   return kda::launch_cp_apply(ap, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -555,24 +559,26 @@ extern "C" kda_status_t kda_context_parallel_prefill(
     if (st != KDA_OK) return st;
     st = kda_segment_summarize_and_scan(
         k, v, qkv_dtype, raw_gate, beta_logits, a_log, dt_bias, T, num_k_heads, num_v_heads, dk, dv, sub, np,
-        initial_state, pM, pU, pIn, pIn + blk, final_state, q, o_m, o_u, flags, gate_lower_bound, nullptr, 0,
-        device_status, stream);
+        initial_state, pM, pU, pIn, pIn + blk, final_state, q, o_m, o_u, flags | KDA_READOUT_HEAD_MAJOR,
+        gate_lower_bound, nullptr, 0, device_status, stream);
     if (st != KDA_OK) return st;
     st = kda_segment_compose(pM, pU, pIn, final_state, num_segments, kp, num_v_heads, dk, dv, M, U, incoming,
                              outgoing, flags & KDA_STATE_V_FIRST, stream);
     if (st != KDA_OK) return st;
     return kda_context_parallel_apply(o_m, o_u, pIn, sub, np, T, num_v_heads, dv, out, out_dtype,
-                                      flags & KDA_STATE_V_FIRST, device_status, stream);
+                                      (flags & KDA_STATE_V_FIRST) | KDA_READOUT_HEAD_MAJOR, device_status, stream);
   }
   // every segment in parallel (M_i, U_i and both readouts), then the exclusive scan
   kda_status_t st = kda_segment_summarize_and_scan(k, v, qkv_dtype, raw_gate, beta_logits, a_log, dt_bias, T,
                                                    num_k_heads, num_v_heads, dk, dv, seg_offsets, num_segments,
                                                    initial_state, M, U, incoming, outgoing, final_state, q, o_m,
-                                                   o_u, flags, gate_lower_bound, nullptr, 0, device_status, stream);
+                                                   o_u, flags | KDA_READOUT_HEAD_MAJOR, gate_lower_bound, nullptr, 0,
+                                                   device_status, stream);
   if (st != KDA_OK) return st;
   // the incoming state's share added to the readouts
   return kda_context_parallel_apply(o_m, o_u, incoming, seg_offsets, num_segments, T, num_v_heads, dv, out,
-                                    out_dtype, flags & KDA_STATE_V_FIRST, device_status, stream);
+                                    out_dtype, (flags & KDA_STATE_V_FIRST) | KDA_READOUT_HEAD_MAJOR, device_status,
+                                    stream);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -665,6 +671,7 @@ extern "C" kda_status_t kda_context_parallel_range_summary(
   f.out = L.o_m;
   f.out2 = L.o_u;
   f.out_bf16 = 1;
+  f.readout_hm = 1;
   f.flags = flags;
   f.lb = gate_lower_bound;
   f.status = device_status;
@@ -746,6 +753,7 @@ extern "C" kda_status_t kda_context_parallel_range_finish(
   ap.v_first = v_first;
   ap.o_m = L.o_m;
   ap.o_u = L.o_u;
+  ap.readout_hm = 1;
   ap.out = out;
   ap.out_bf16 = out_dtype == KDA_BF16;
   ap.status = device_status;

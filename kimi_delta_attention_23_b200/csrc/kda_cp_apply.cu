@@ -23,10 +23,10 @@
 
 namespace kda {
 
-// tensor map of a token-major [tokens][heads][128] tensor (kda_fused.cu): box = box_x channels x
-// 1 head x 64 tokens
+// tensor map of a [tokens][heads][128] tensor (kda_fused.cu): box = box_x channels x 1 head x 64
+// tokens; head_major: a [heads][tokens][128] tensor, coordinates (channel, token, head)
 bool encode_token_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t esize, int64_t tokens,
-                       int heads, uint32_t box_x, CUtensorMapSwizzle swz);
+                       int heads, uint32_t box_x, CUtensorMapSwizzle swz, bool head_major);
 
 namespace {
 
@@ -155,8 +155,9 @@ __global__ void __launch_bounds__(kThreads, 1) cp_apply_kernel(ApplyArgs a, cons
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int ch = q >> 1, rh = q & 1;
-      tma_load_3d(dst + ch * 16384 + rh * 8192, &tm.om, 64 * ch, p.h, t0 + 64 * rh, bar);
-      tma_load_3d(dst + kTileBytes + ch * 16384 + rh * 8192, &tm.ou, 64 * ch, p.h, t0 + 64 * rh, bar);
+      const int y = a.readout_hm ? t0 + 64 * rh : p.h, z = a.readout_hm ? p.h : t0 + 64 * rh;
+      tma_load_3d(dst + ch * 16384 + rh * 8192, &tm.om, 64 * ch, y, z, bar);
+      tma_load_3d(dst + kTileBytes + ch * 16384 + rh * 8192, &tm.ou, 64 * ch, y, z, bar);
     }
   };
   auto fail = [&]() {
@@ -342,11 +343,11 @@ cudaError_t launch_cp_apply(const ApplyArgs& a, cudaStream_t stream) {
   memset(&tm, 0, sizeof(tm));
   const bool ok =
       encode_token_rows(&tm.om, a.o_m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.total_tokens, a.Hv, 64,
-                        CU_TENSOR_MAP_SWIZZLE_128B) &&
+                        CU_TENSOR_MAP_SWIZZLE_128B, a.readout_hm != 0) &&
       encode_token_rows(&tm.ou, a.o_u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.total_tokens, a.Hv, 64,
-                        CU_TENSOR_MAP_SWIZZLE_128B) &&
+                        CU_TENSOR_MAP_SWIZZLE_128B, a.readout_hm != 0) &&
       (!a.out_bf16 || encode_token_rows(&tm.out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.total_tokens, a.Hv,
-                                        64, CU_TENSOR_MAP_SWIZZLE_128B));
+                                        64, CU_TENSOR_MAP_SWIZZLE_128B, false));
   if (!ok) return cudaErrorInvalidValue;
   int dev = 0, sms = 0;
   if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;

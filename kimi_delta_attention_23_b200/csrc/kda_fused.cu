@@ -1198,8 +1198,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         // full chunks leave through two tensor stores (sources read before (1) of the next chunk)
         if (L == C) {
           if (tid == kPfThread) {
-            tma_store_3d(&tm.out, sbase + OFF_KQ, 0, h, (int)c0);
-            tma_store_3d(&tm.out2, sbase + OFF_KQ + 16384, 0, h, (int)c0);
+            const int y = a.readout_hm ? (int)c0 : h, z = a.readout_hm ? h : (int)c0;
+            tma_store_3d(&tm.out, sbase + OFF_KQ, 0, y, z);
+            tma_store_3d(&tm.out2, sbase + OFF_KQ + 16384, 0, y, z);
             bulk_commit();
           }
         } else {
@@ -1207,7 +1208,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           const int st = e >> 10, row = (e >> 4) & 63, cc = e & 15;
           if (row < L)
             *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(st ? a.out2 : a.out) +
-                                      ((size_t)(c0 + row) * a.Hv + h) * D + cc * 8) =
+                                      (a.readout_hm ? (size_t)h * a.total_tokens + c0 + row
+                                                    : (size_t)(c0 + row) * a.Hv + h) * D + cc * 8) =
                 *reinterpret_cast<const uint4*>(sm + OFF_KQ + st * 16384 + row * 256 + cc * 16);
         }
         }
@@ -1277,13 +1279,18 @@ EncodeTiledFn encode_fn() {
 }
 
 // [tokens][heads][128] row-major; box = box_x channels x 1 head x 64 tokens
+// head_major: [heads][tokens][128] instead, coordinates (channel, token, head), box = box_x
+// channels x 64 tokens x 1 head
 bool encode_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t esize, int64_t tokens,
-                 int heads, uint32_t box_x = D, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
+                 int heads, uint32_t box_x = D, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE,
+                 bool head_major = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)tokens};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * esize, (cuuint64_t)heads * D * esize};
-  const cuuint32_t box[3] = {box_x, 1u, (cuuint32_t)C};
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)(head_major ? tokens : heads),
+                              (cuuint64_t)(head_major ? heads : tokens)};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * esize,
+                                 (cuuint64_t)(head_major ? tokens : heads) * D * esize};
+  const cuuint32_t box[3] = {box_x, head_major ? (cuuint32_t)C : 1u, head_major ? 1u : (cuuint32_t)C};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -1292,8 +1299,8 @@ bool encode_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint3
 }  // namespace
 
 bool encode_token_rows(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint32_t esize, int64_t tokens,
-                       int heads, uint32_t box_x, CUtensorMapSwizzle swz) {
-  return encode_rows(m, base, dt, esize, tokens, heads, box_x, swz);
+                       int heads, uint32_t box_x, CUtensorMapSwizzle swz, bool head_major) {
+  return encode_rows(m, base, dt, esize, tokens, heads, box_x, swz, head_major);
 }
 
 cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream) {
@@ -1318,8 +1325,10 @@ cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream) {
                               CU_TENSOR_MAP_SWIZZLE_128B);
   // bf16 outputs (the prefill output, or both readouts of the build) leave through tensor stores
   const bool out_ok = rows == 0 || !a.out || !a.out_bf16 ||
-                      (encode_rows(&tm.out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv) &&
-                       (!a.out2 || encode_rows(&tm.out2, a.out2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv)));
+                      (encode_rows(&tm.out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv, D,
+                                   CU_TENSOR_MAP_SWIZZLE_NONE, a.build && a.readout_hm) &&
+                       (!a.out2 || encode_rows(&tm.out2, a.out2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv, D,
+                                               CU_TENSOR_MAP_SWIZZLE_NONE, a.build && a.readout_hm)));
   if (!ok || !out_ok) return cudaErrorInvalidValue;
   dim3 grid(a.Hv, a.batch);
   if (a.build && a.out)

@@ -73,6 +73,7 @@ struct FusedArgs {
   int32_t values_zero;      // 1: all values are zero (transition build)
   void* out;                // [T,Hv,128] or NULL (no readout); with build: readout of the transition
   void* out2;               // build only: readout of the contribution [T,Hv,128] bf16 (or NULL)
+  int32_t readout_hm;       // build only: both readouts stored [Hv][T][128] instead
   int32_t out_bf16;
   uint32_t flags;
   float lb;
@@ -92,6 +93,7 @@ struct ApplyArgs {
   int32_t v_first;
   const void* o_m;             // bf16 [T][Hv][128] readout through the transition
   const void* o_u;             // bf16 [T][Hv][128] readout of the contribution
+  int32_t readout_hm;          // both readouts stored [Hv][T][128] instead
   void* out;                   // [T][Hv][128]
   int32_t out_bf16;
   int32_t* status;

@@ -250,3 +250,30 @@ def test_split_prefill_matches_oracle_and_unsplit(layout):
         assert rel_l2(res["incoming_states"], scan["incoming_states"]) < 1e-2
         assert rel_l2(res["outgoing_states"], scan["outgoing_states"]) < 1e-2
     assert rel_l2(split["out"], whole["out"].double().cpu().numpy()) < 1e-2
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_head_major_readouts_equal_token_major(out_dtype):
+    """KDA_READOUT_HEAD_MAJOR stores the same readouts as [Hv, T, 128]: bit for bit the
+    token-major ones transposed, and the apply gives the same outputs from either layout
+    (ragged segments: partial chunks in the build, partial tiles in the apply)."""
+    w = W.random_inputs([1500], 2, 4, 128, 128, seed=31, state_std=0.1)
+    wd = w.to("cuda")
+    offs = torch.tensor([0, 130, 131, 700, 1500], dtype=torch.int32, device="cuda")
+    init = wd.state_pool[0].contiguous()
+    res = {}
+    for layout in ("token_major", "head_major"):
+        r = kda.kda_segment_summarize_and_scan(wd.k, wd.v, wd.raw_gate, wd.beta_logits, wd.a_log, wd.dt_bias, offs,
+                                               init, q=wd.q, readout_layout=layout)
+        out = kda.kda_context_parallel_apply(r["readout_m"], r["readout_u"], r["incoming_states"], offs,
+                                             output_dtype=out_dtype, readout_layout=layout)
+        res[layout] = (r, out)
+    torch.cuda.synchronize()
+    (rt, ot), (rh, oh) = res["token_major"], res["head_major"]
+    assert rh["readout_m"].shape == (4, 1500, 128)
+    assert torch.equal(rh["readout_m"], rt["readout_m"].transpose(0, 1))
+    assert torch.equal(rh["readout_u"], rt["readout_u"].transpose(0, 1))
+    assert torch.equal(oh, ot)
+    o_ref, _ = oracle.kda_forward(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens,
+                                  w.state_pool, w.state_indices)
+    assert rel_l2(oh, o_ref) < 1e-2
