@@ -13,6 +13,11 @@ Other workloads (``--workload``) time one kda_chunk_fwd call over the whole batc
 state pool carries over from step to step (each step resumes from the previous final states,
 as a split prefill would), so the timed work never includes a pool restore.
 
+Besides the contract's keys the line carries ``roofline`` (the dominant launch's algorithmic
+bytes over its device time, against the measured HBM bandwidth), ``step_roofline`` (the whole
+step's algorithmic bytes and FLOPs: GB/s, TFLOP/s, and the fraction of the roofline taken as
+the slower of bytes at HBM bandwidth and FLOPs at the dense bf16 peak) and ``breakdown_ms``.
+
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload (the
 oracle is the only reference implementation there is).  Under torchrun every rank runs its
 own replica of the workload (weak scaling, no data-path collective); timings are device
@@ -85,6 +90,25 @@ def apply_bytes(w, N, dv=128):
     th = w.total_tokens * w.num_v_heads
     ob = 2 if w.output_dtype == torch.bfloat16 else 4
     return th * (2 * dv * 2 + dv * ob) + N * w.num_v_heads * dv * dv * 4
+
+
+def step_roofline(w, ms_step, segments, pk, dk=128, dv=128):
+    """The whole step against the roofline as the slower of its algorithmic bytes at the HBM
+    bandwidth and its algorithmic FLOPs at the dense bf16 tensor peak.  Bytes: the straight
+    prefill's (q, k, v, gate, beta, outputs, the state read and written per chain), plus, for the
+    context-parallel step, twice the segments' M, U and incoming tensors."""
+    if segments:
+        nbytes = chunk_fwd_bytes(w, 1, dk, dv) + 2 * segments * w.num_v_heads * 3 * dk * dv * 4
+    else:
+        nbytes = chunk_fwd_bytes(w, w.batch, dk, dv)
+    flops = chunk_fwd_flops(w, dk=dk, dv=dv)
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9) * 1e3
+    t_tensor = flops / (pk["bf16_tflops"] * 1e12) * 1e3
+    return {"bound": "hbm" if t_hbm >= t_tensor else "tensor", "algorithmic_bytes": nbytes,
+            "algorithmic_flops": flops, "gbs": nbytes / (ms_step / 1e3) / 1e9,
+            "tflops": flops / (ms_step / 1e3) / 1e12, "roofline_ms": max(t_hbm, t_tensor),
+            "hbm_ms": t_hbm, "tensor_ms": t_tensor, "frac": max(t_hbm, t_tensor) / ms_step,
+            "peak_source": pk["source"]}
 
 
 def chunk_fwd_flops(w, C=64, dk=128, dv=128):
@@ -503,6 +527,8 @@ def run_ours(args):
                             decode_bytes(w) if step.decode else chunk_fwd_bytes(w, w.batch)) / 1e9)},
             "breakdown_ms": breakdown,
             "roofline": roof, "gpu_launches": step.launches() * args.steps, "clocks": clocks.summary()}
+    if not step.decode:
+        line["step_roofline"] = step_roofline(w, ms_step, step.N if step.cp else 0, pk)
     if e2e is not None:
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
