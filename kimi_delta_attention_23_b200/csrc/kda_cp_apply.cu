@@ -10,9 +10,9 @@
 // Per 128-token tile of one (segment, head) pair the product O_M (128 x 128) . S_in (128 x 128)
 // runs on tcgen05 into a TMEM accumulator; both readout tiles arrive by tensor copies through a
 // three-stage ring, so two tiles' loads are in flight while one is finished.  All eight warps
-// work in step: one thread issues the next tile's MMA (into the other of two accumulators)
-// before the current tile's epilogue, which adds O_U and writes the bf16 result over the O_U
-// tile in place; a full tile leaves through tensor stores, a partial last tile of a segment
+// work in step: after a tile's epilogue (which adds O_U and writes the bf16 result over the O_U
+// tile in place) one thread issues the copies two tiles ahead and the next tile's MMA, into the
+// other of two accumulators; a full tile leaves through tensor stores, a partial last tile of a segment
 // through row stores (rows past the segment belong to the next one).
 #include <cuda.h>
 #include <string.h>
@@ -227,14 +227,6 @@ __global__ void __launch_bounds__(kThreads, 1) cp_apply_kernel(ApplyArgs a, cons
     const bool has_next = i + 1 < count;
     const TilePos nxt = has_next ? advance(cur) : cur;
     const bool same_pair = has_next && nxt.seg == cur.seg && nxt.h == cur.h;
-    // the next tile's product runs under this tile's epilogue when it reads the same state
-    if (tid == 0 && same_pair) {
-      const int s1 = (int)((i + 1) % kStages);
-      if (mbar_wait_bounded(bar_full + 8 * s1, (uint32_t)(((i + 1) / kStages) & 1), kWaitLimitNs))
-        issue_mma(s1, acc ^ 1);
-      else
-        fail();
-    }
     const bool ok = mbar_wait_bounded(bar_acc + 8 * acc, (uint32_t)((i >> 1) & 1), kWaitLimitNs) &&
                     mbar_wait_bounded(bar_full + 8 * s, (uint32_t)((i / kStages) & 1), kWaitLimitNs);
     if (!ok) fail();
@@ -297,17 +289,10 @@ __global__ void __launch_bounds__(kThreads, 1) cp_apply_kernel(ApplyArgs a, cons
     }
     if (has_next && !same_pair) {
       // a new pair: its state replaces the B operand (this tile's product, its last reader, is
-      // complete), then its first product
+      // complete)
       stage_state(nxt);
       tc_fence_before();
       __syncthreads();
-      if (tid == 0) {
-        const int s1 = (int)((i + 1) % kStages);
-        if (mbar_wait_bounded(bar_full + 8 * s1, (uint32_t)(((i + 1) / kStages) & 1), kWaitLimitNs))
-          issue_mma(s1, acc ^ 1);
-        else
-          fail();
-      }
     }
     // tile i + 2 goes to the stage of tile i - 1, whose stores (the group before this tile's)
     // have read it by now
@@ -317,6 +302,16 @@ __global__ void __launch_bounds__(kThreads, 1) cp_apply_kernel(ApplyArgs a, cons
         issue_loads(lpos, (int)((i + 2) % kStages));
       }
       if (i + 3 < count) lpos = advance(lpos);
+    }
+    // the next tile's product, into the other accumulator (its last reader, the epilogue of tile
+    // i - 1, is done): its copies were issued one epilogue ago, so they have had this tile's
+    // epilogue to land
+    if (tid == 0 && has_next) {
+      const int s1 = (int)((i + 1) % kStages);
+      if (mbar_wait_bounded(bar_full + 8 * s1, (uint32_t)(((i + 1) / kStages) & 1), kWaitLimitNs))
+        issue_mma(s1, acc ^ 1);
+      else
+        fail();
     }
     cur = nxt;
   }
