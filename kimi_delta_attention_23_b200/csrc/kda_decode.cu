@@ -17,6 +17,8 @@
 // (up to 64 elements each) between the read and the write.  The loads of the block are issued
 // before the gate is evaluated, so the per-channel vectors are computed under their latency.
 //
+// Thread mapping for dk = dv = 128 (kVec): the same split, with lane l taking the four
+// consecutive elements 4l .. 4l + 3 of each stored row, so every state access is 16 bytes.
 // Thread mapping (any 1 <= dk, dv <= 128):
 //   K_FIRST ([dk][dv] row-major): warp w takes rows i = w + 8m, lane l takes columns
 //     j = l + 32c; a warp load is 32 consecutive floats of one row.  Column sums over i
@@ -38,7 +40,7 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-template <bool kVFirst>
+template <bool kVFirst, bool kVec>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeArgs a) {
   __shared__ float sAlpha[128], sK[128], sQ[128], sV[128], sDelta[128];
   __shared__ float sRed[2][kDecWarps][128];
@@ -56,15 +58,25 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeArgs
   }
   float* blk = a.pool + ((size_t)slot * a.Hv + h) * (size_t)dk * dv;
 
-  // ---- issue the loads of this thread's state elements first
+  // ---- issue the loads of this thread's state elements first.  Element c of stored row
+  // r = warp + 8m is at stored column col(c) = 4 lane + c (kVec) or lane + 32 c.
+  auto col = [&](int c) { return kVec ? 4 * lane + c : lane + 32 * c; };
   float s[16][4];
 #pragma unroll
   for (int m = 0; m < 16; ++m) {
+    if constexpr (kVec) {
+      const float4 v4 = *reinterpret_cast<const float4*>(blk + (size_t)(warp + 8 * m) * 128 + 4 * lane);
+      s[m][0] = v4.x;
+      s[m][1] = v4.y;
+      s[m][2] = v4.z;
+      s[m][3] = v4.w;
+    } else {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int i = kVFirst ? lane + 32 * c : warp + 8 * m;  // key channel (row of S)
-      const int j = kVFirst ? warp + 8 * m : lane + 32 * c;  // value column
-      s[m][c] = (i < dk && j < dv) ? blk[kVFirst ? (size_t)j * dk + i : (size_t)i * dv + j] : 0.f;
+      for (int c = 0; c < 4; ++c) {
+        const int i = kVFirst ? col(c) : warp + 8 * m;  // key channel (row of S)
+        const int j = kVFirst ? warp + 8 * m : col(c);  // value column
+        s[m][c] = (i < dk && j < dv) ? blk[kVFirst ? (size_t)j * dk + i : (size_t)i * dv + j] : 0.f;
+      }
     }
   }
 
@@ -114,7 +126,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeArgs
     float al[4], kc[4], qc[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const int i = lane + 32 * c;
+      const int i = col(c);
       al[c] = sAlpha[i & 127];
       kc[c] = sK[i & 127];
       qc[c] = sQ[i & 127];
@@ -134,10 +146,16 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeArgs
       if (j < dv) {
         const float delta = beta * (sV[j] - pk);
         if (lane == 0) store_out(out, out_row + j, fmaf(qk, delta, pq), a.out_bf16);
+        if constexpr (kVec) {
+          *reinterpret_cast<float4*>(blk + (size_t)j * 128 + 4 * lane) =
+              make_float4(fmaf(kc[0], delta, s[m][0]), fmaf(kc[1], delta, s[m][1]), fmaf(kc[2], delta, s[m][2]),
+                          fmaf(kc[3], delta, s[m][3]));
+        } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int i = lane + 32 * c;
-          if (i < dk) blk[(size_t)j * dk + i] = fmaf(kc[c], delta, s[m][c]);
+          for (int c = 0; c < 4; ++c) {
+            const int i = col(c);
+            if (i < dk) blk[(size_t)j * dk + i] = fmaf(kc[c], delta, s[m][c]);
+          }
         }
       }
     }
@@ -156,8 +174,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeArgs
     }
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      sRed[0][warp][lane + 32 * c] = pk[c];
-      sRed[1][warp][lane + 32 * c] = pq[c];
+      sRed[0][warp][col(c)] = pk[c];
+      sRed[1][warp][col(c)] = pq[c];
     }
     __syncthreads();
     if (tid < dv) {
@@ -174,16 +192,22 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeArgs
     __syncthreads();
     float dl[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) dl[c] = sDelta[(lane + 32 * c) & 127];
+    for (int c = 0; c < 4; ++c) dl[c] = sDelta[col(c) & 127];
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
       const int i = warp + 8 * m;
       if (i < dk) {
         const float kv = sK[i];
+        if constexpr (kVec) {
+          *reinterpret_cast<float4*>(blk + (size_t)i * 128 + 4 * lane) =
+              make_float4(fmaf(kv, dl[0], s[m][0]), fmaf(kv, dl[1], s[m][1]), fmaf(kv, dl[2], s[m][2]),
+                          fmaf(kv, dl[3], s[m][3]));
+        } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int j = lane + 32 * c;
-          if (j < dv) blk[(size_t)i * dv + j] = fmaf(kv, dl[c], s[m][c]);
+          for (int c = 0; c < 4; ++c) {
+            const int j = col(c);
+            if (j < dv) blk[(size_t)i * dv + j] = fmaf(kv, dl[c], s[m][c]);
+          }
         }
       }
     }
@@ -195,10 +219,19 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeArgs
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const int64_t blocks = (int64_t)a.batch * a.Hv;
   if (blocks == 0) return cudaSuccess;
-  if (a.v_first)
-    decode_kernel<true><<<(unsigned)blocks, kDecThreads, 0, stream>>>(a);
-  else
-    decode_kernel<false><<<(unsigned)blocks, kDecThreads, 0, stream>>>(a);
+  // 16-byte state accesses when every stored row is 128 floats and the pool is 16-byte aligned
+  const bool vec = a.dk == 128 && a.dv == 128 && (reinterpret_cast<uintptr_t>(a.pool) & 15u) == 0;
+  if (a.v_first) {
+    if (vec)
+      decode_kernel<true, true><<<(unsigned)blocks, kDecThreads, 0, stream>>>(a);
+    else
+      decode_kernel<true, false><<<(unsigned)blocks, kDecThreads, 0, stream>>>(a);
+  } else {
+    if (vec)
+      decode_kernel<false, true><<<(unsigned)blocks, kDecThreads, 0, stream>>>(a);
+    else
+      decode_kernel<false, false><<<(unsigned)blocks, kDecThreads, 0, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 
