@@ -33,6 +33,10 @@
  *    stack as the state pool and state_indices = 0..N-1 then produces every segment's
  *    outputs in parallel; afterwards that pool holds the outgoing states.
  *
+ *  kda_prefill_host_pipelined
+ *    kda_chunk_fwd's result for one sequence held in host memory, its copies over the host link
+ *    pipelined with the kernels in segments.
+ *
  *  kda_context_parallel_range_summary / kda_context_parallel_range_finish
  *    The same method across GPUs: each rank reduces its own token range of the sequence to one
  *    affine map, the caller gathers the maps and scans them over the ranks, and each rank
@@ -365,6 +369,38 @@ KDA_API kda_status_t kda_context_parallel_range_finish(
     const float *range_incoming, void *out, kda_dtype_t out_dtype, float *range_outgoing, float *M,
     float *U, float *incoming, float *outgoing, uint32_t flags, void *workspace,
     size_t workspace_bytes, int32_t *device_status, void *stream);
+
+/*
+ * kda_prefill_host_pipelined -- the prefill of ONE sequence whose inputs and outputs are in
+ * host memory (pinned, for the copies to overlap), as kda_chunk_fwd computes it
+ * ("max.nn.state_space.kda_chunk": the recurrence over 64-token chunks, the state carried from
+ * chunk to chunk), with the copies over the host link pipelined in segments of
+ * segment_tokens tokens (a multiple of 64): segment i's inputs are copied in while segment
+ * i - 1 runs and earlier segments' outputs are copied out, both directions at once.  Segment
+ * boundaries fall on chunk boundaries, so the outputs and the final state equal
+ * kda_chunk_fwd's on the whole sequence bit for bit.
+ *
+ *   q, k [T, Hk, 128], v [T, Hv, 128] bf16; raw_gate [T, Hv, 128], beta_logits [T, Hv],
+ *   a_log [Hv], dt_bias [Hv, 128] fp32; initial_state [Hv, <state>] fp32   HOST, read
+ *   out [T, Hv, 128] out_dtype; final_state [Hv, <state>] fp32              HOST, written
+ *   workspace: DEVICE, >= kda_prefill_host_workspace_size(...) bytes, 256-byte aligned: the
+ *     staged sequence (inputs, outputs, state); its contents on return are unspecified
+ *   flags: gate / beta modes and KDA_STATE_V_FIRST; device_status (device, nullable) as for
+ *     kda_chunk_fwd
+ * Asynchronous on `stream`: the kernels run there and the stream completes after the last
+ * copy out; read the host outputs after synchronising it.  The copies run on two helper
+ * streams the library creates on a device's first call and keeps (with four events); calls are
+ * serialised while they enqueue.  bf16 q/k/v with dk = dv = 128 only; else KDA_ERR_UNSUPPORTED.
+ */
+KDA_API size_t kda_prefill_host_workspace_size(int64_t T, int32_t num_k_heads, int32_t num_v_heads,
+                                               kda_dtype_t out_dtype, int64_t segment_tokens);
+KDA_API kda_status_t kda_prefill_host_pipelined(
+    const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype, const float *raw_gate,
+    const float *beta_logits, const float *a_log, const float *dt_bias, int64_t T,
+    int32_t num_k_heads, int32_t num_v_heads, int32_t dk, int32_t dv, const float *initial_state,
+    void *out, kda_dtype_t out_dtype, float *final_state, int64_t segment_tokens, uint32_t flags,
+    float gate_lower_bound, void *workspace, size_t workspace_bytes, int32_t *device_status,
+    void *stream);
 
 /* Bytes of workspace with which kda_chunk_fwd may take its split route on the current device
  * (0 when the batch has chains enough for the SMs, for dk or dv other than 128, or with

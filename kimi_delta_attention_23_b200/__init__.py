@@ -11,6 +11,8 @@ Public calls (same names as the C ABI):
   kda_context_parallel(M, U, initial)     the scan alone, returning exactly incoming_states,
                                           outgoing_states and final_state
   kda_context_parallel_prefill(...)       the context-parallel prefill of one long sequence
+  kda_prefill_host_pipelined(...)         kda_chunk_fwd on one sequence in pinned host memory, the
+                                          copies pipelined with the kernels in segments
   kda_context_parallel_range_summary(...) one rank's token range of a sequence as one map
   kda_context_parallel_range_finish(...)  that range's outputs from the state entering it
                                           (``distributed.context_parallel_prefill`` joins the
@@ -27,7 +29,8 @@ __all__ = ["kda_chunk_fwd", "kda_decode", "kda_segment_summarize_and_scan", "kda
            "kda_context_parallel_apply", "kda_context_parallel_prefill", "kda_context_parallel_workspace_size",
            "kda_context_parallel_workspace_preferred", "kda_context_parallel_pieces",
            "kda_context_parallel_piece_offsets", "kda_segment_compose", "kda_context_parallel_range_workspace_size",
-           "kda_context_parallel_range_summary", "kda_context_parallel_range_finish", "kda_workspace_size",
+           "kda_context_parallel_range_summary", "kda_context_parallel_range_finish", "kda_prefill_host_pipelined",
+           "kda_prefill_host_workspace_size", "kda_workspace_size",
            "kda_status_string", "load_library", "KdaError", "LIB_PATH"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -98,6 +101,11 @@ def load_library():
     lib.kda_context_parallel_range_finish.restype = ctypes.c_int
     lib.kda_context_parallel_range_finish.argtypes = [i64, i32, i32, i32, i32, fp, vp, ctypes.c_int, fp, fp, fp,
                                                       fp, fp, u32, vp, sz, ip, vp]
+    lib.kda_prefill_host_workspace_size.restype = sz
+    lib.kda_prefill_host_workspace_size.argtypes = [i64, i32, i32, ctypes.c_int, i64]
+    lib.kda_prefill_host_pipelined.restype = ctypes.c_int
+    lib.kda_prefill_host_pipelined.argtypes = [vp, vp, vp, ctypes.c_int, fp, fp, fp, fp, i64, i32, i32, i32, i32, fp,
+                                               vp, ctypes.c_int, fp, i64, u32, f32, vp, sz, ip, vp]
     lib.kda_workspace_size.restype = sz
     lib.kda_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32, i32, u32]
     lib.kda_status_string.restype = ctypes.c_char_p
@@ -653,3 +661,73 @@ def kda_context_parallel_range_finish(range_incoming, workspace, seg_offsets, to
         raise KdaError(rc, "kda_context_parallel_range_finish")
     return {"out": out, "range_outgoing": range_outgoing, "incoming_states": incoming, "outgoing_states": outgoing,
             "transition_matrices": M, "local_contributions": U}
+
+
+def kda_prefill_host_workspace_size(T, num_k_heads, num_v_heads, output_dtype=torch.bfloat16,
+                                    segment_tokens=8192) -> int:
+    return int(load_library().kda_prefill_host_workspace_size(T, num_k_heads, num_v_heads, _DTYPES[output_dtype],
+                                                              segment_tokens))
+
+
+def _host(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host (CPU) tensor, got {t.device}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() and not t.is_pinned():  # (an empty tensor has no storage to pin)
+        raise ValueError(f"{name} must be in pinned host memory (tensor.pin_memory()) for the copies to overlap")
+    return t
+
+
+def kda_prefill_host_pipelined(q, k, v, raw_gate, beta_logits, a_log, dt_bias, initial_state, out=None, *,
+                               final_state=None, segment_tokens=8192, workspace=None, output_dtype=None,
+                               gate_mode="original", beta_mode="logits", state_layout="K_FIRST",
+                               gate_lower_bound=-5.0, device_status=None, stream=None, device=None):
+    """kda_chunk_fwd's prefill of ONE sequence held in pinned host memory (bf16 q/k/v,
+    dk = dv = 128), the copies pipelined with the kernels in segments of ``segment_tokens``.
+
+    Every tensor argument is a pinned CPU tensor (``workspace`` and ``device_status`` excepted:
+    device).  Returns dict(out, final_state), host tensors that are complete once ``stream``
+    (default: the device's current stream) has been synchronised.
+    """
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _host(q, "q", torch.bfloat16)
+    T, Hk, dk = q.shape
+    _shape(_host(k, "k", torch.bfloat16), "k", (T, Hk, dk))
+    _host(v, "v", torch.bfloat16)
+    Hv, dv = v.shape[1], v.shape[2]
+    _shape(v, "v", (T, Hv, dv))
+    _shape(_host(raw_gate, "raw_gate", torch.float32), "raw_gate", (T, Hv, dk))
+    _shape(_host(beta_logits, "beta_logits", torch.float32), "beta_logits", (T, Hv))
+    _shape(_host(a_log, "a_log", torch.float32), "a_log", (Hv,))
+    _shape(_host(dt_bias, "dt_bias", torch.float32), "dt_bias", (Hv, dk))
+    st = (dk, dv) if state_layout == "K_FIRST" else (dv, dk)
+    _shape(_host(initial_state, "initial_state", torch.float32), "initial_state", (Hv, *st))
+    if output_dtype is None:
+        output_dtype = v.dtype if out is None else out.dtype
+    if out is None:
+        out = torch.empty((T, Hv, dv), dtype=output_dtype, pin_memory=True)
+    _shape(_host(out, "out", output_dtype), "out", (T, Hv, dv))
+    if final_state is None:
+        final_state = torch.empty((Hv, *st), dtype=torch.float32, pin_memory=True)
+    _shape(_host(final_state, "final_state", torch.float32), "final_state", (Hv, *st))
+    with torch.cuda.device(dev):
+        if workspace is None:
+            need = kda_prefill_host_workspace_size(T, Hk, Hv, output_dtype, segment_tokens)
+            if need == 0:
+                raise ValueError("segment_tokens must be a positive multiple of 64")
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        _dev(workspace, "workspace", torch.uint8, dev)
+        rc = lib.kda_prefill_host_pipelined(
+            _ptr(q), _ptr(k), _ptr(v), _BF16, _ptr(raw_gate), _ptr(beta_logits), _ptr(a_log), _ptr(dt_bias), T,
+            Hk, Hv, dk, dv, _ptr(initial_state), _ptr(out), _DTYPES[output_dtype], _ptr(final_state),
+            int(segment_tokens), _flags(gate_mode, beta_mode, state_layout), float(gate_lower_bound),
+            _ptr(workspace), workspace.numel(), _ptr(device_status), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_prefill_host_pipelined")
+    return {"out": out, "final_state": final_state}

@@ -174,3 +174,22 @@ def test_decode_host_checks(lib, over, code):
 
 def test_decode_empty_batch_is_a_no_op(lib):
     assert _decode(lib, batch=0, q=0, k=0, v=0, raw=0, beta=0, out=0) == 0
+
+
+def test_host_pipelined_prefill_host_checks(lib):
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
+
+    def call(segment=1024, qkv=1, final=16, flags=0, ws=256, ws_bytes=16, out_dtype=1):
+        return lib.kda_prefill_host_pipelined(p(16), p(16), p(16), qkv, p(16), p(16), p(16), p(16), 4096, 2, 2, 128,
+                                              128, p(16), p(16), out_dtype, p(final), segment, flags, -5.0, p(ws),
+                                              ws_bytes, None, None)
+    assert call(segment=100) == 1          # not a multiple of 64
+    assert call(segment=0) == 1
+    assert call(final=0) == 1              # null final state
+    assert call(flags=1 << 4) == 1         # a segment-call flag
+    assert call(qkv=0) == 2                # fp32 q/k/v bind no kernel here
+    assert call() == 3                     # workspace too small
+    need = kda.kda_prefill_host_workspace_size(4096, 2, 2, segment_tokens=1024)
+    assert need >= 4096 * 2 * 128 * (2 + 2) + 4096 * 2 * 128 * (2 + 4 + 2)
+    assert call(ws=256 + 8, ws_bytes=need) == 3  # workspace not 256-byte aligned
+    assert kda.kda_prefill_host_workspace_size(4096, 2, 2, segment_tokens=100) == 0
