@@ -42,11 +42,24 @@ __device__ __forceinline__ float warp_sum(float x) {
 
 template <bool kVFirst, bool kVec>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeArgs a) {
-  __shared__ float sAlpha[128], sK[128], sQ[128], sV[128], sDelta[128];
-  __shared__ float sRed[2][kDecWarps][128];
+  __shared__ __align__(16) float sAlpha[128], sK[128], sQ[128], sV[128], sDelta[128];
+  __shared__ __align__(16) float sRed[2][kDecWarps][128];
   __shared__ float sBeta, sQK;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // four consecutive floats at 4 lane (kVec): one 16-byte access, no bank conflict
+  auto get4 = [&](const float* arr, float (&o)[4]) {
+    if constexpr (kVec) {
+      const float4 v4 = *reinterpret_cast<const float4*>(arr + 4 * lane);
+      o[0] = v4.x;
+      o[1] = v4.y;
+      o[2] = v4.z;
+      o[3] = v4.w;
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) o[c] = arr[(lane + 32 * c) & 127];
+    }
+  };
   const int64_t bh = blockIdx.x;
   const int h = (int)(bh % a.Hv);
   const int64_t b = bh / a.Hv;
@@ -124,13 +137,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeArgs
 
   if constexpr (kVFirst) {
     float al[4], kc[4], qc[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int i = col(c);
-      al[c] = sAlpha[i & 127];
-      kc[c] = sK[i & 127];
-      qc[c] = sQ[i & 127];
-    }
+    get4(sAlpha, al);
+    get4(sK, kc);
+    get4(sQ, qc);
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
       float pk = 0.f, pq = 0.f;
@@ -172,10 +181,15 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeArgs
         pq[c] = fmaf(qv, s[m][c], pq[c]);
       }
     }
+    if constexpr (kVec) {
+      *reinterpret_cast<float4*>(&sRed[0][warp][4 * lane]) = make_float4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<float4*>(&sRed[1][warp][4 * lane]) = make_float4(pq[0], pq[1], pq[2], pq[3]);
+    } else {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      sRed[0][warp][col(c)] = pk[c];
-      sRed[1][warp][col(c)] = pq[c];
+      for (int c = 0; c < 4; ++c) {
+        sRed[0][warp][col(c)] = pk[c];
+        sRed[1][warp][col(c)] = pq[c];
+      }
     }
     __syncthreads();
     if (tid < dv) {
@@ -191,8 +205,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const DecodeArgs
     }
     __syncthreads();
     float dl[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) dl[c] = sDelta[col(c) & 127];
+    get4(sDelta, dl);
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
       const int i = warp + 8 * m;
