@@ -543,8 +543,8 @@ def measure_e2e(w, args, stream, pg):
     """The step end to end through the public API from pinned host buffers: every input copied in,
     the step, the output rows and the final state copied out, all inside the timed region.  A
     single long bf16 sequence goes through kda_prefill_host_pipelined (the call for a sequence held
-    in host memory: copies in and out pipelined with the kernels, segments of the workload's
-    segment length); other workloads copy in, call kda_chunk_fwd, and copy out."""
+    in host memory: copies in and out pipelined with the kernels in 2048-token segments); other
+    workloads copy in, call kda_chunk_fwd, and copy out."""
     dev = w.q.device
     if w.seg_offsets is not None and w.q.dtype == torch.bfloat16:
         return measure_e2e_host_pipelined(w, args, stream, pg)
@@ -592,7 +592,9 @@ def measure_e2e_host_pipelined(w, args, stream, pg):
     import kimi_delta_attention_23_b200 as kda
     dev = w.q.device
     T, Hk, Hv = w.total_tokens, w.k.shape[1], w.num_v_heads
-    seg = max(64, (int(w.seg_offsets[1].item()) // 64) * 64)
+    # pipeline granularity: 2048-token segments (8192: 104.1 ms, 4096: 102.8, 2048: 101.8, 1024:
+    # 103.3 on the 131072-token, 32-head sequence; the copies in bound it near 100 ms)
+    seg = min(2048, max(64, -(-T // 64) * 64))
     host = {n: getattr(w, n).cpu().contiguous().pin_memory()
             for n in ("q", "k", "v", "raw_gate", "beta_logits", "a_log", "dt_bias")}
     host["initial_state"] = w.state_pool[0].cpu().contiguous().pin_memory()
