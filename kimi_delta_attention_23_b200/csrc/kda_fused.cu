@@ -149,7 +149,33 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   const uint32_t raw_addr = smem_addr(smem_raw);
   uint8_t* sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int h = blockIdx.x, b = blockIdx.y;
+  const int h = blockIdx.x;
+  int b = blockIdx.y;
+  if constexpr (!kBuild) {
+    // longest sequences first: blocks start in the order of blockIdx.y, and a batch's time is
+    // bound by when its longest chains start, so block row y takes the sequence of rank y in
+    // decreasing length (ties by index) -- for batches of at most kThreads sequences; the
+    // lengths go through the score scratch, which no chunk has touched yet
+    if (a.batch > 1 && a.batch <= kThreads) {
+      int* s_len = reinterpret_cast<int*>(sm + OFF_A);
+      volatile int* s_pick = reinterpret_cast<volatile int*>(sm + OFF_A + 4 * kThreads);
+      for (int s = tid; s < a.batch; s += kThreads) s_len[s] = a.cu[s + 1] - a.cu[s];
+      if (tid == 0) *s_pick = b;
+      __syncthreads();
+      if (tid < a.batch) {
+        const int ls = s_len[tid];
+        int rank = 0;
+        for (int s2 = 0; s2 < a.batch; ++s2) {
+          const int l2 = s_len[s2];
+          rank += (l2 > ls || (l2 == ls && s2 < tid)) ? 1 : 0;
+        }
+        if (rank == (int)blockIdx.y) *s_pick = tid;
+      }
+      __syncthreads();
+      b = *s_pick;
+      __syncthreads();  // every read of the scratch and of the pick is done
+    }
+  }
   const int kh = h / (a.Hv / a.Hk);
   const bool safe = a.flags & KDA_GATE_SAFE, prob = a.flags & KDA_BETA_PROB;
 
