@@ -216,3 +216,25 @@ def test_decreasing_offsets_are_reported():
                       wd.state_pool.clone(), wd.state_indices, device_status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 5
+
+
+# ------------------------------------------------------------------------------------------
+# batch order: the prefill hands block rows to sequences longest first for batches of at most
+# 256 sequences (index order above that); either way every sequence is computed once
+# ------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("lengths_kind", ["over_256", "exactly_256_equal", "many_ties"])
+def test_batch_order_covers_every_sequence_once(lengths_kind):
+    g = torch.Generator().manual_seed(41)
+    if lengths_kind == "over_256":
+        lengths = torch.randint(0, 200, (300,), generator=g).tolist()
+    elif lengths_kind == "exactly_256_equal":
+        lengths = [70] * 256
+    else:
+        lengths = [int(x) for x in torch.randint(0, 3, (40,), generator=g) * 64 + 5]
+    B = len(lengths)
+    slots = B + 7
+    idx = torch.randperm(slots, generator=g)[:B].to(torch.int32)
+    w = W.random_inputs(lengths, 1, 2, 128, 128, seed=B, state_std=0.2, max_slots=slots, state_indices=idx)
+    out, pool = gpu_forward(w)
+    check(w, out, pool, 1e-2)
