@@ -265,16 +265,12 @@ __global__ void __launch_bounds__(kScanThreads) affine_scan_kernel(ScanArgs a) {
 }
 
 bool tiles128(int dk, int dv);
-__global__ void affine_scan128_kernel(ScanArgs a);
+cudaError_t launch_affine_scan128(const ScanArgs& a, cudaStream_t stream);
 __global__ void compose128_kernel(ComposeArgs a);
 
 cudaError_t launch_affine_scan(const ScanArgs& a, cudaStream_t stream) {
   if (tiles128(a.dk, a.dv)) {
-    const int smem = (2 * 128 * 132 + 2 * 128 * 40) * (int)sizeof(float);  // M double buffer, carried tile parts
-    cudaError_t err = cudaFuncSetAttribute(affine_scan128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (err != cudaSuccess) return err;
-    affine_scan128_kernel<<<dim3(a.H, a.dv / 32), 256, smem, stream>>>(a);
-    return cudaGetLastError();
+    return launch_affine_scan128(a, stream);
   }
   const size_t smem = ((size_t)a.dk * (a.dk + 1) + 2 * (size_t)a.dk * kScanCols) * sizeof(float);
   cudaError_t err = cudaFuncSetAttribute(affine_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -436,12 +432,13 @@ __device__ __forceinline__ uint32_t tf32_rna(float x) {
   return u;
 }
 
-// the carried 128 x 32 tile X, as its tf32 high part (chi) and rounded remainder (clo), from this
-// thread's fragment x[n][c]
-__device__ __forceinline__ void put_carried(float* chi, float* clo, const float (&x)[4][4]) {
+// the carried 128 x 8 NT tile X (NT 8-column MMA tiles), as its tf32 high part (chi) and
+// rounded remainder (clo), from this thread's fragment x[n][c]
+template <int NT>
+__device__ __forceinline__ void put_carried(float* chi, float* clo, const float (&x)[NT][4]) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int n = 0; n < 4; ++n)
+  for (int n = 0; n < NT; ++n)
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       const int r = 16 * w + g + 8 * hh, c = 8 * n + 2 * t;
@@ -453,12 +450,13 @@ __device__ __forceinline__ void put_carried(float* chi, float* clo, const float 
     }
 }
 
-// acc = Ms (128 x 128, row-major, stride kLdM) times X (128 x 32, held as chi + clo)
+// acc = Ms (128 x 128, row-major, stride kLdM) times X (128 x 8 NT, held as chi + clo)
+template <int NT>
 __device__ __forceinline__ void tile_product_tc(const float* Ms, const float* chi, const float* clo,
-                                                float (&acc)[4][4]) {
+                                                float (&acc)[NT][4]) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int n = 0; n < 4; ++n)
+  for (int n = 0; n < NT; ++n)
 #pragma unroll
     for (int u = 0; u < 4; ++u) acc[n][u] = 0.f;
   const float* a0p = Ms + (16 * w + g) * kLdM;
@@ -473,7 +471,7 @@ __device__ __forceinline__ void tile_product_tc(const float* Ms, const float* ch
       al[i] = tf32_rna(av[i] - __uint_as_float(ah[i]));
     }
 #pragma unroll
-    for (int n = 0; n < 4; ++n) {
+    for (int n = 0; n < NT; ++n) {
       const int c = 8 * n + g;
       const uint32_t bh0 = __float_as_uint(chi[(k0 + t) * kLdC + c]), bh1 = __float_as_uint(chi[(k0 + t + 4) * kLdC + c]);
       const uint32_t bl0 = __float_as_uint(clo[(k0 + t) * kLdC + c]), bl1 = __float_as_uint(clo[(k0 + t + 4) * kLdC + c]);
@@ -497,11 +495,12 @@ __device__ __forceinline__ void store_state2(float* blk, int r, int j, int dv, i
     blk[(size_t)(j + 1) * 128 + r] = x.y;
   }
 }
-// this thread's fragment of columns j0 .. j0 + 31 of a state block
-__device__ __forceinline__ void load_frag(float (&x)[4][4], const float* blk, int j0, int dv, int v_first) {
+// this thread's fragment of columns j0 .. j0 + 8 NT - 1 of a state block
+template <int NT>
+__device__ __forceinline__ void load_frag(float (&x)[NT][4], const float* blk, int j0, int dv, int v_first) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int n = 0; n < 4; ++n)
+  for (int n = 0; n < NT; ++n)
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       const float2 v = load_state2(blk, 16 * w + g + 8 * hh, j0 + 8 * n + 2 * t, dv, v_first);
@@ -509,36 +508,38 @@ __device__ __forceinline__ void load_frag(float (&x)[4][4], const float* blk, in
       x[n][2 * hh + 1] = v.y;
     }
 }
-__device__ __forceinline__ void store_frag(float* blk, const float (&x)[4][4], int j0, int dv, int v_first) {
+template <int NT>
+__device__ __forceinline__ void store_frag(float* blk, const float (&x)[NT][4], int j0, int dv, int v_first) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int n = 0; n < 4; ++n)
+  for (int n = 0; n < NT; ++n)
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh)
       store_state2(blk, 16 * w + g + 8 * hh, j0 + 8 * n + 2 * t, dv, v_first,
                    make_float2(x[n][2 * hh], x[n][2 * hh + 1]));
 }
 
-// the exclusive scan (as affine_scan_kernel) for dk = 128: one block per (head, 32 columns)
+// the exclusive scan (as affine_scan_kernel) for dk = 128: one block per (head, 8 NT columns)
+template <int NT>
 __global__ void __launch_bounds__(kTileThreads, 1) affine_scan128_kernel(ScanArgs a) {
   extern __shared__ __align__(16) float smf[];
   float* Ms0 = smf;
   float* Ms1 = Ms0 + 128 * kLdM;
   float* chi = Ms1 + 128 * kLdM;  // [128][kLdC] the carried tile, tf32 high part
   float* clo = chi + 128 * kLdC;  // and remainder
-  const int h = blockIdx.x, j0 = blockIdx.y * kT, H = a.H, dv = a.dv, vf = a.v_first;
+  const int h = blockIdx.x, j0 = blockIdx.y * 8 * NT, H = a.H, dv = a.dv, vf = a.v_first;
   const size_t st = (size_t)128 * dv;
   if (a.N > 0) stage_m(Ms0, a.M + (size_t)h * 128 * 128);
-  float x[4][4];  // this thread's part of the carried state
+  float x[NT][4];  // this thread's part of the carried state
   load_frag(x, a.initial + (size_t)h * st, j0, dv, vf);
-  float un[4][4];  // the next step's contribution, loaded one step ahead
+  float un[NT][4];  // the next step's contribution, loaded one step ahead
   if (a.N > 0) load_frag(un, a.U + (size_t)h * st, j0, dv, vf);
   for (int s = 0; s < a.N; ++s) {
     float* Ms = (s & 1) ? Ms1 : Ms0;
     const size_t blk = ((size_t)s * H + h) * st;
-    float u[4][4];
+    float u[NT][4];
 #pragma unroll
-    for (int n = 0; n < 4; ++n)
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int c = 0; c < 4; ++c) u[n][c] = un[n][c];
     if (s + 1 < a.N) load_frag(un, a.U + ((size_t)(s + 1) * H + h) * st, j0, dv, vf);
@@ -551,10 +552,10 @@ __global__ void __launch_bounds__(kTileThreads, 1) affine_scan128_kernel(ScanArg
       cp_async_wait_groups<0>();
     }
     __syncthreads();  // M_s staged, the carried tile complete
-    float acc[4][4];
+    float acc[NT][4];
     tile_product_tc(Ms, chi, clo, acc);
 #pragma unroll
-    for (int n = 0; n < 4; ++n)
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int c = 0; c < 4; ++c) x[n][c] = acc[n][c] + u[n][c];
     if (a.outgoing) store_frag(a.outgoing + blk, x, j0, dv, vf);
@@ -620,6 +621,29 @@ __global__ void __launch_bounds__(kTileThreads, 2) compose128_kernel(ComposeArgs
 }
 
 bool tiles128(int dk, int dv) { return dk == 128 && dv % kT == 0 && dv <= 128; }
+
+// whether 16-column tiles (twice the blocks of 32-column ones) still fit the SMs in one wave
+bool narrow_tiles(int64_t blocks32) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                 cudaSuccess)
+    return false;
+  return 2 * blocks32 <= sms;
+}
+
+cudaError_t launch_affine_scan128(const ScanArgs& a, cudaStream_t stream) {
+  const int smem = (2 * 128 * kLdM + 2 * 128 * kLdC) * (int)sizeof(float);  // M double buffer, carried tile parts
+  if (narrow_tiles((int64_t)a.H * (a.dv / 32))) {
+    cudaError_t err = cudaFuncSetAttribute(affine_scan128_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    affine_scan128_kernel<2><<<dim3(a.H, a.dv / 16), kTileThreads, smem, stream>>>(a);
+  } else {
+    cudaError_t err = cudaFuncSetAttribute(affine_scan128_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    affine_scan128_kernel<4><<<dim3(a.H, a.dv / kT), kTileThreads, smem, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
 
 // ------------------------------------------------------------------------------------------
 // A varlen batch as pieces: every sequence cut into chunk-aligned pieces of at most piece_len
@@ -726,6 +750,7 @@ cudaError_t launch_plan_pieces(const PlanArgs& a, cudaStream_t stream) {
 
 // one block per (head, 32 columns, sequence): the sequence's pieces applied in order to its
 // pool state, each piece's incoming state recorded, the final state written back
+template <int NT>
 __global__ void __launch_bounds__(kTileThreads, 1) pool_scan128_kernel(PoolScanArgs a) {
   if (*a.fallback) return;
   extern __shared__ __align__(16) float smf[];
@@ -733,23 +758,23 @@ __global__ void __launch_bounds__(kTileThreads, 1) pool_scan128_kernel(PoolScanA
   float* Ms1 = Ms0 + 128 * kLdM;
   float* chi = Ms1 + 128 * kLdM;
   float* clo = chi + 128 * kLdC;
-  const int h = blockIdx.x, j0 = blockIdx.y * kT, b = blockIdx.z, H = a.H, dv = a.dv, vf = a.v_first;
+  const int h = blockIdx.x, j0 = blockIdx.y * 8 * NT, b = blockIdx.z, H = a.H, dv = a.dv, vf = a.v_first;
   const size_t st = (size_t)128 * dv;
   const int p0 = a.seq_first[b], p1 = a.seq_first[b + 1];
   const int32_t slot = a.slots ? a.slots[b] : b;
   float* blk = a.pool + ((size_t)slot * H + h) * st;
   if (p1 > p0) stage_m(Ms0, a.M + ((size_t)p0 * H + h) * 128 * 128);
-  float x[4][4];
+  float x[NT][4];
   load_frag(x, blk, j0, dv, vf);
-  float un[4][4];  // the next piece's contribution, loaded one step ahead
+  float un[NT][4];  // the next piece's contribution, loaded one step ahead
   if (p1 > p0) load_frag(un, a.U + ((size_t)p0 * H + h) * st, j0, dv, vf);
   for (int p = p0; p < p1; ++p) {
     const int s = p - p0;
     float* Ms = (s & 1) ? Ms1 : Ms0;
     const size_t pb = ((size_t)p * H + h) * st;
-    float u[4][4];
+    float u[NT][4];
 #pragma unroll
-    for (int n = 0; n < 4; ++n)
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int c = 0; c < 4; ++c) u[n][c] = un[n][c];
     if (p + 1 < p1) load_frag(un, a.U + ((size_t)(p + 1) * H + h) * st, j0, dv, vf);
@@ -762,10 +787,10 @@ __global__ void __launch_bounds__(kTileThreads, 1) pool_scan128_kernel(PoolScanA
       cp_async_wait_groups<0>();
     }
     __syncthreads();
-    float acc[4][4];
+    float acc[NT][4];
     tile_product_tc(Ms, chi, clo, acc);
 #pragma unroll
-    for (int n = 0; n < 4; ++n)
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int c = 0; c < 4; ++c) x[n][c] = acc[n][c] + u[n][c];
     __syncthreads();
@@ -775,10 +800,18 @@ __global__ void __launch_bounds__(kTileThreads, 1) pool_scan128_kernel(PoolScanA
 
 cudaError_t launch_pool_scan(const PoolScanArgs& a, cudaStream_t stream) {
   const int smem = (2 * 128 * kLdM + 2 * 128 * kLdC) * (int)sizeof(float);
-  cudaError_t err = cudaFuncSetAttribute(pool_scan128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (err != cudaSuccess) return err;
   if (a.batch == 0) return cudaSuccess;
-  pool_scan128_kernel<<<dim3(a.H, a.dv / kT, a.batch), kTileThreads, smem, stream>>>(a);
+  // the scan is bound per SM by its tile products: with blocks to spare for the SMs, 16-column
+  // tiles spread the same products over twice the blocks
+  if (narrow_tiles((int64_t)a.H * (a.dv / 32) * a.batch)) {
+    cudaError_t err = cudaFuncSetAttribute(pool_scan128_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    pool_scan128_kernel<2><<<dim3(a.H, a.dv / 16, a.batch), kTileThreads, smem, stream>>>(a);
+  } else {
+    cudaError_t err = cudaFuncSetAttribute(pool_scan128_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    pool_scan128_kernel<4><<<dim3(a.H, a.dv / kT, a.batch), kTileThreads, smem, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 
