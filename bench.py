@@ -92,7 +92,7 @@ def apply_bytes(w, N, dv=128):
     return th * (2 * dv * 2 + dv * ob) + N * w.num_v_heads * dv * dv * 4
 
 
-def step_roofline(w, ms_step, segments, pk, dk=128, dv=128):
+def step_roofline(w, ms_step, segments, pk, dk=128, dv=128, sm_mhz=None):
     """The whole step against the roofline as the slower of its algorithmic bytes at the HBM
     bandwidth and its algorithmic FLOPs at the dense bf16 tensor peak.  Bytes: the straight
     prefill's (q, k, v, gate, beta, outputs, the state read and written per chain), plus, for the
@@ -104,11 +104,19 @@ def step_roofline(w, ms_step, segments, pk, dk=128, dv=128):
     flops = chunk_fwd_flops(w, dk=dk, dv=dv)
     t_hbm = nbytes / (pk["hbm_gbs"] * 1e9) * 1e3
     t_tensor = flops / (pk["bf16_tflops"] * 1e12) * 1e3
-    return {"bound": "hbm" if t_hbm >= t_tensor else "tensor", "algorithmic_bytes": nbytes,
-            "algorithmic_flops": flops, "gbs": nbytes / (ms_step / 1e3) / 1e9,
-            "tflops": flops / (ms_step / 1e3) / 1e12, "roofline_ms": max(t_hbm, t_tensor),
-            "hbm_ms": t_hbm, "tensor_ms": t_tensor, "frac": max(t_hbm, t_tensor) / ms_step,
-            "peak_source": pk["source"]}
+    res = {"bound": "hbm" if t_hbm >= t_tensor else "tensor", "algorithmic_bytes": nbytes,
+           "algorithmic_flops": flops, "gbs": nbytes / (ms_step / 1e3) / 1e9,
+           "tflops": flops / (ms_step / 1e3) / 1e12, "roofline_ms": max(t_hbm, t_tensor),
+           "hbm_ms": t_hbm, "tensor_ms": t_tensor, "frac": max(t_hbm, t_tensor) / ms_step,
+           "peak_source": pk["source"]}
+    # beside it, not part of it: the special-function floor of the gates, three transcendental
+    # operations per token, head and key channel (softplus's exp and log, the decay's exp) at 16
+    # per clock per SM
+    if sm_mhz and torch.cuda.is_available():
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        sfu_ops = 3.0 * w.total_tokens * w.num_v_heads * dk
+        res["sfu_ms"] = sfu_ops / (16.0 * sms * sm_mhz * 1e6) * 1e3
+    return res
 
 
 def chunk_fwd_flops(w, C=64, dk=128, dv=128):
@@ -528,7 +536,8 @@ def run_ours(args):
             "breakdown_ms": breakdown,
             "roofline": roof, "gpu_launches": step.launches() * args.steps, "clocks": clocks.summary()}
     if not step.decode:
-        line["step_roofline"] = step_roofline(w, ms_step, step.N if step.cp else 0, pk)
+        line["step_roofline"] = step_roofline(w, ms_step, step.N if step.cp else 0, pk,
+                                              sm_mhz=line["clocks"].get("sm_mhz") or line["clocks"].get("sm_max_mhz"))
     if e2e is not None:
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
