@@ -30,7 +30,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 

@@ -10,7 +10,6 @@ the recurrence.  All arithmetic is float64 on inputs widened exactly from bf16/f
 from __future__ import annotations
 
 import ctypes
-import os
 
 import numpy as np
 

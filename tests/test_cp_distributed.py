@@ -3,7 +3,6 @@ sequence, exchange their range maps through ``distributed.exchange_summaries`` (
 all-gather); the three per-rank steps run on the fp64 oracle here (there is no GPU), so these
 tests pin the cut into ranges, the exchange order and which incoming state each rank takes
 against the oracle's straight token-by-token pass over the whole sequence."""
-import os
 import socket
 
 import numpy as np
