@@ -9,8 +9,9 @@ state, cut into 16 segments of 8192) a step is the context-parallel prefill:
      gives incoming / outgoing / final states;
   2. kda_context_parallel_apply: every output row from its readouts and its segment's incoming
      state.
-Other workloads (``--workload``) time one kda_chunk_fwd call over the whole batch; their
-state pool carries over from step to step (each step resumes from the previous final states,
+Other workloads (``--workload``), and the default one with ``--straight`` (the straight pass
+over the whole sequence), time one kda_chunk_fwd call over the whole batch; their state pool
+carries over from step to step (each step resumes from the previous final states,
 as a split prefill would), so the timed work never includes a pool restore.
 
 Besides the contract's keys the line carries ``roofline`` (the dominant launch's algorithmic
@@ -325,11 +326,12 @@ def run_reference(args):
 class Step:
     """One pass of the hot path on device-resident inputs; records per-call CUDA events."""
 
-    def __init__(self, w, stream, public=False):
+    def __init__(self, w, stream, public=False, straight=False):
         import kimi_delta_attention_23_b200 as kda
         self.kda, self.w, self.stream, self.public = kda, w, stream, public
         dev = w.q.device
-        self.cp = w.seg_offsets is not None
+        # straight: a segmented workload run as one kda_chunk_fwd call over the whole sequence
+        self.cp = w.seg_offsets is not None and not straight
         self.decode = bool(w.notes.get("decode"))
         T, Hv, dv, dk = w.total_tokens, w.num_v_heads, w.dv, w.dk
         self.out = torch.empty((T, Hv, dv), dtype=w.output_dtype, device=dev)
@@ -458,7 +460,7 @@ def run_ours(args):
     kbuild.build()
     w = W.make(args.workload, device=dev, seed=rank_seed(args.workload, rank))
     stream = torch.cuda.current_stream(dev)
-    step = Step(w, stream)
+    step = Step(w, stream, straight=args.straight)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -527,6 +529,7 @@ def run_ours(args):
             "config": {"workload": args.workload, "tokens": tokens, "num_v_heads": w.num_v_heads,
                        "num_k_heads": w.num_k_heads, "dk": w.dk, "dv": w.dv, "batch": w.batch,
                        "segments": step.N if step.cp else None,
+                       "pass": "context_parallel" if step.cp else ("decode" if step.decode else "straight"),
                        "pieces_per_segment": step.pieces if step.cp else None, "gate_mode": w.gate_mode,
                        "state_layout": w.state_layout, "parallelism": f"dp{world}" if world > 1 else "single",
                        "l2": "inputs larger than L2 (%.2f GB read per step), no flush" % (
@@ -662,7 +665,7 @@ def profile_launches(args):
     from kimi_delta_attention_23_b200 import build as kbuild
     kbuild.build()
     w = W.make(args.workload, device="cuda")
-    if w.seg_offsets is not None:
+    if w.seg_offsets is not None and not args.straight:
         step = Step(w, torch.cuda.current_stream())
         for _ in range(args.profile_launches):
             step()
@@ -695,6 +698,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=W.WORKLOADS, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--straight", action="store_true",
+                    help="segmented workloads: time one kda_chunk_fwd call over the whole sequence instead of "
+                         "the context-parallel step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
