@@ -542,7 +542,6 @@ extern "C" kda_status_t kda_context_parallel_prefill(
     return KDA_ERR_WORKSPACE;
   __nv_bfloat16_raw* o_m = reinterpret_cast<__nv_bfloat16_raw*>(workspace);
   __nv_bfloat16_raw* o_u = o_m + (size_t)T * num_v_heads * dv;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int kp = choose_pieces(T, num_segments, num_v_heads);
   if (kp > 1 && workspace_bytes >= round256(need) + pieces_bytes(num_segments, kp, num_v_heads, dk, dv)) {
     // more chains than segments: every segment is built as kp chunk-aligned pieces, the scan
