@@ -57,7 +57,7 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far beyond any legitim
 // 128-byte swizzle layout (see sw_off)
 constexpr int OFF_S = 0;                    // prefill: bf16 output staging (the bf16 state lives in TMEM)
 constexpr int OFF_KQ = OFF_S + 32768;       // [K o Gamma ; Q o Gamma]   128 rows x 128 K (then output staging)
-constexpr int OFF_KPT = OFF_KQ + 32768;     // K'^T       128 rows x 64 K
+constexpr int OFF_KPT = OFF_KQ + 32768;     // K'         64 rows x 128, the MN-major B operand K'^T
 constexpr int OFF_X = OFF_KPT + 16384;      // X^T, then Delta^T   128 rows x 64 K
 constexpr int OFF_V = OFF_X + 16384;        // V as the MN-major A operand V^T (two 64-column halves, 8 KB
                                             // apart, 128B-swizzled by the tensor copy)
@@ -549,7 +549,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     // is one of them, possibly scaled once more: K o Gamma = kp o pre, K o pi = kp (o prevb in an
     // upper half), K o kappa = ks (o nextb in a lower half), K' = ks o suf, the 8-level halves
     // kp / qp (upper) and ks (lower).
-    float kpv[8][4];  // K' values of my 8 rows x 4 channels (packed pairwise below)
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int row = warp * 8 + r;
@@ -582,26 +581,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
             pack4(ks[0] * nextb[0], ks[1] * nextb[1], ks[2] * nextb[2], ks[3] * nextb[3]);
         *reinterpret_cast<uint2*>(sm + OFF_KK8 + sw_off(r32, ch, 32)) = ks_b;
       }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) kpv[r][c] = ks[c] * suf[c];
-    }
-    // K'^T: channel rows, token columns; pairs of consecutive tokens pack into one word
-    uint32_t kpt[4][4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-#pragma unroll
-      for (int m = 0; m < 4; ++m) kpt[c][m] = pack_bf16(kpv[2 * m][c], kpv[2 * m + 1][c]);
-    // the four stores rotate over the channels by lane so that each store instruction spreads
-    // its 32 rows over all eight 16-byte bank groups
-#pragma unroll
-    for (int cs = 0; cs < 4; ++cs) {
-      const int c = (cs + (lane >> 1)) & 3;
-      uint4 val;
-      val.x = c == 0 ? kpt[0][0] : c == 1 ? kpt[1][0] : c == 2 ? kpt[2][0] : kpt[3][0];
-      val.y = c == 0 ? kpt[0][1] : c == 1 ? kpt[1][1] : c == 2 ? kpt[2][1] : kpt[3][1];
-      val.z = c == 0 ? kpt[0][2] : c == 1 ? kpt[1][2] : c == 2 ? kpt[2][2] : kpt[3][2];
-      val.w = c == 0 ? kpt[0][3] : c == 1 ? kpt[1][3] : c == 2 ? kpt[2][3] : kpt[3][3];
-      *reinterpret_cast<uint4*>(sm + OFF_KPT + sw_off(ch + c, warp * 8, 128)) = val;
+      // K' = K o (decay to the chunk end), token rows like the other tiles: the update reads it
+      // as the MN-major B operand K'^T
+      *reinterpret_cast<uint2*>(sm + OFF_KPT + sw_off(row, ch, 64)) =
+          pack4(ks[0] * suf[0], ks[1] * suf[1], ks[2] * suf[2], ks[3] * suf[3]);
     }
 
     fence_async_smem();  // the operand tiles are read by the tensor cores
@@ -964,8 +947,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmS, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128(sbase + OFF_KPT + kk * 32),
-                 idesc_bf16_f32(128), 1);
+        mma_bf16(tmS, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128_mn(sbase + OFF_KPT + kk * 2048, 8192),
+                 idesc_bf16_f32(128, false, true), 1);
       mma_commit(bar4);
     }
     // the next chunk's gates run on the CUDA cores while these products are on the tensor cores
@@ -1160,7 +1143,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16(u ? tmSu : tmS, desc_sw128(sbase + (u ? OFF_X : OFF_XM) + kk * 32),
-                   desc_sw128(sbase + OFF_KPT + kk * 32), idesc_bf16_f32(128), 1);
+                   desc_sw128_mn(sbase + OFF_KPT + kk * 2048, 8192), idesc_bf16_f32(128, false, true), 1);
         mma_commit(bar4);
       }
       // the next chunk's gates run on the CUDA cores while these products are on the tensor cores
