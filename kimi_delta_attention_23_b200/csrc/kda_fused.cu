@@ -71,7 +71,7 @@ constexpr int OFF_QPI8 = OFF_KPI8 + 8192;
 constexpr int OFF_KK8 = OFF_QPI8 + 8192;    // 32 x 128: lower-half columns to the half end
 constexpr int OFF_A = OFF_KK8 + 8192;       // fp32 [64][68] key scores
 constexpr int OFF_TAU = OFF_A + 17408;      // fp32 [8][128] decay product of each 8-row block
-constexpr int OFF_MP = OFF_TAU + 4096;      // fp32 [6][128] decay between 16-blocks of a pair
+constexpr int OFF_MP = OFF_TAU + 4096;      // bf16x2 [6][64] decay between 16-blocks of a pair
 constexpr int OFF_BETA = OFF_MP + 3072;     // fp32 [64]
 constexpr int OFF_GC = OFF_BETA + 256;      // fp32 [128] Gamma of the last row
 constexpr int OFF_BAR = OFF_GC + 512;       // mbarriers (+0..+39, +48, +56), TMEM base (+40), abort flag (+44)
@@ -114,9 +114,11 @@ __device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
   return make_uint2(pack_bf16(a, b), pack_bf16(c, d));
 }
 
-__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t x, float s0, float s1) {
-  float2 f = unpack_bf16(x);
-  return pack_bf16(f.x * s0, f.y * s1);
+// two bf16 products in one instruction (each rounded to nearest)
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t x, uint32_t y) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(x), "r"(y));
+  return d;
 }
 
 // slot -> (row, column) of the 8x8 diagonal-block scores: slots 0..27 are A (row > column),
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + OFF_BAR + 44);
   float* sA = reinterpret_cast<float*>(sm + OFF_A);
   float* sTau = reinterpret_cast<float*>(sm + OFF_TAU);
-  float* sMp = reinterpret_cast<float*>(sm + OFF_MP);
+  uint32_t* sMp = reinterpret_cast<uint32_t*>(sm + OFF_MP);
   float* sBeta = reinterpret_cast<float*>(sm + OFF_BETA);
   float* sGC = reinterpret_cast<float*>(sm + OFF_GC);
 
@@ -535,14 +537,15 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         t16a[c] = tv[2 * D] * tv[3 * D];  // 16-block 1
         t16b[c] = tv[4 * D] * tv[5 * D];  // 16-block 2
       }
-      const float4 one = make_float4(1.f, 1.f, 1.f, 1.f);
-      *reinterpret_cast<float4*>(sMp + 0 * D + ch) = one;
-      *reinterpret_cast<float4*>(sMp + 1 * D + ch) = make_float4(t16a[0], t16a[1], t16a[2], t16a[3]);
-      *reinterpret_cast<float4*>(sMp + 2 * D + ch) = one;
-      *reinterpret_cast<float4*>(sMp + 3 * D + ch) =
-          make_float4(t16a[0] * t16b[0], t16a[1] * t16b[1], t16a[2] * t16b[2], t16a[3] * t16b[3]);
-      *reinterpret_cast<float4*>(sMp + 4 * D + ch) = make_float4(t16b[0], t16b[1], t16b[2], t16b[3]);
-      *reinterpret_cast<float4*>(sMp + 5 * D + ch) = one;
+      // bf16 pairs of channels (the scale of a bf16 operand pair in the score products)
+      const uint2 one = pack4(1.f, 1.f, 1.f, 1.f);
+      uint2* mp2 = reinterpret_cast<uint2*>(sMp + ch / 2);
+      mp2[0 * 32] = one;
+      mp2[1 * 32] = pack4(t16a[0], t16a[1], t16a[2], t16a[3]);
+      mp2[2 * 32] = one;
+      mp2[3 * 32] = pack4(t16a[0] * t16b[0], t16a[1] * t16b[1], t16a[2] * t16b[2], t16a[3] * t16b[3]);
+      mp2[4 * 32] = pack4(t16b[0], t16b[1], t16b[2], t16b[3]);
+      mp2[5 * 32] = one;
     }
     // operand tiles.  The block-local products are formed once per row -- kp = k o p8 (prefix
     // from the block start), qp = q o p8, ks = k o s8 (suffix to the block end) -- and every tile
@@ -619,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         // pairs (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
         const int pa = warp < 1 ? 1 : (warp < 3 ? 2 : 3), pb = warp - pa * (pa - 1) / 2;
         float accA[2][4] = {}, accP[2][4] = {};
-        const float* mp = sMp + warp * D;
+        const uint32_t* mp = sMp + warp * (D / 2);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           uint32_t ak0, ak1, ak2, ak3, aq0, aq1, aq2, aq3, b00, b01, b10, b11;
@@ -629,12 +632,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           const int br = 16 * pb + (m >> 1) * 8 + (lane & 7), bkc = 2 * kk + (m & 1);
           ldsm_x4(sbase + OFF_KC + sw_off(br, bkc * 8, 64), b00, b01, b10, b11);
           if (pa - pb > 1) {  // adjacent 16-blocks have nothing between them
-            const int k0 = 16 * kk + 2 * t;
-            const float m0 = mp[k0], m1 = mp[k0 + 1], m2 = mp[k0 + 8], m3 = mp[k0 + 9];
-            b00 = scale_bf16x2(b00, m0, m1);
-            b10 = scale_bf16x2(b10, m0, m1);
-            b01 = scale_bf16x2(b01, m2, m3);
-            b11 = scale_bf16x2(b11, m2, m3);
+            // channels 16 kk + 2 t, + 1 and 16 kk + 2 t + 8, + 9
+            const uint32_t m01 = mp[8 * kk + t], m89 = mp[8 * kk + t + 4];
+            b00 = mul_bf16x2(b00, m01);
+            b10 = mul_bf16x2(b10, m01);
+            b01 = mul_bf16x2(b01, m89);
+            b11 = mul_bf16x2(b11, m89);
           }
           mma16816(accA[0], ak0, ak1, ak2, ak3, b00, b01);
           mma16816(accA[1], ak0, ak1, ak2, ak3, b10, b11);
