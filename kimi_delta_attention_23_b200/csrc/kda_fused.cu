@@ -114,6 +114,19 @@ __device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
   return make_uint2(pack_bf16(a, b), pack_bf16(c, d));
 }
 
+// two fp32 products in one instruction (each rounded to nearest, as two multiplies would be)
+__device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ uint2 pack4(float2 lo, float2 hi) {
+  return make_uint2(pack_bf16(lo.x, lo.y), pack_bf16(hi.x, hi.y));
+}
+
 // two bf16 products in one instruction (each rounded to nearest)
 __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t x, uint32_t y) {
   uint32_t d;
@@ -552,42 +565,52 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     // is one of them, possibly scaled once more: K o Gamma = kp o pre, K o pi = kp (o prevb in an
     // upper half), K o kappa = ks (o nextb in a lower half), K' = ks o suf, the 8-level halves
     // kp / qp (upper) and ks (lower).
+    // (channel pairs multiplied two at a time)
+    const float2 pre01 = make_float2(pre[0], pre[1]), pre23 = make_float2(pre[2], pre[3]);
+    const float2 suf01 = make_float2(suf[0], suf[1]), suf23 = make_float2(suf[2], suf[3]);
+    const float2 pb01 = make_float2(prevb[0], prevb[1]), pb23 = make_float2(prevb[2], prevb[3]);
+    const float2 nb01 = make_float2(nextb[0], nextb[1]), nb23 = make_float2(nextb[2], nextb[3]);
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int row = warp * 8 + r;
-      const float kp[4] = {kf[r][0] * p8[r][0], kf[r][1] * p8[r][1], kf[r][2] * p8[r][2], kf[r][3] * p8[r][3]};
-      const float qp[4] = {qf[r][0] * p8[r][0], qf[r][1] * p8[r][1], qf[r][2] * p8[r][2], qf[r][3] * p8[r][3]};
-      const float ks[4] = {kf[r][0] * s8[r][0], kf[r][1] * s8[r][1], kf[r][2] * s8[r][2], kf[r][3] * s8[r][3]};
+      const float2 p01 = make_float2(p8[r][0], p8[r][1]), p23 = make_float2(p8[r][2], p8[r][3]);
+      const float2 s01 = make_float2(s8[r][0], s8[r][1]), s23 = make_float2(s8[r][2], s8[r][3]);
+      const float2 k01 = make_float2(kf[r][0], kf[r][1]), k23 = make_float2(kf[r][2], kf[r][3]);
+      const float2 kp01 = mul_f32x2(k01, p01), kp23 = mul_f32x2(k23, p23);
+      const float2 ks01 = mul_f32x2(k01, s01), ks23 = mul_f32x2(k23, s23);
+      float2 qp01 = make_float2(0.f, 0.f), qp23 = qp01;
+      if constexpr (kRead) {
+        qp01 = mul_f32x2(make_float2(qf[r][0], qf[r][1]), p01);
+        qp23 = mul_f32x2(make_float2(qf[r][2], qf[r][3]), p23);
+      }
       *reinterpret_cast<uint2*>(sm + OFF_KQ + sw_off(row, ch, 128)) =
-          pack4(kp[0] * pre[0], kp[1] * pre[1], kp[2] * pre[2], kp[3] * pre[3]);
+          pack4(mul_f32x2(kp01, pre01), mul_f32x2(kp23, pre23));
       if constexpr (kRead)
         *reinterpret_cast<uint2*>(sm + OFF_KQ + sw_off(64 + row, ch, 128)) =
-            pack4(qp[0] * pre[0], qp[1] * pre[1], qp[2] * pre[2], qp[3] * pre[3]);
+            pack4(mul_f32x2(qp01, pre01), mul_f32x2(qp23, pre23));
       const int r32 = b16 * 8 + r;
       if (upper) {
-        const uint2 kp_b = pack4(kp[0], kp[1], kp[2], kp[3]);
         *reinterpret_cast<uint2*>(sm + OFF_KPI + sw_off(row, ch, 64)) =
-            pack4(kp[0] * prevb[0], kp[1] * prevb[1], kp[2] * prevb[2], kp[3] * prevb[3]);
-        *reinterpret_cast<uint2*>(sm + OFF_KPI8 + sw_off(r32, ch, 32)) = kp_b;
+            pack4(mul_f32x2(kp01, pb01), mul_f32x2(kp23, pb23));
+        *reinterpret_cast<uint2*>(sm + OFF_KPI8 + sw_off(r32, ch, 32)) = pack4(kp01, kp23);
         if constexpr (kRead) {
           *reinterpret_cast<uint2*>(sm + OFF_QPI + sw_off(row, ch, 64)) =
-              pack4(qp[0] * prevb[0], qp[1] * prevb[1], qp[2] * prevb[2], qp[3] * prevb[3]);
-          *reinterpret_cast<uint2*>(sm + OFF_QPI8 + sw_off(r32, ch, 32)) = pack4(qp[0], qp[1], qp[2], qp[3]);
+              pack4(mul_f32x2(qp01, pb01), mul_f32x2(qp23, pb23));
+          *reinterpret_cast<uint2*>(sm + OFF_QPI8 + sw_off(r32, ch, 32)) = pack4(qp01, qp23);
         }
-        *reinterpret_cast<uint2*>(sm + OFF_KC + sw_off(row, ch, 64)) = pack4(ks[0], ks[1], ks[2], ks[3]);
+        *reinterpret_cast<uint2*>(sm + OFF_KC + sw_off(row, ch, 64)) = pack4(ks01, ks23);
       } else {
-        const uint2 ks_b = pack4(ks[0], ks[1], ks[2], ks[3]);
-        *reinterpret_cast<uint2*>(sm + OFF_KPI + sw_off(row, ch, 64)) = pack4(kp[0], kp[1], kp[2], kp[3]);
+        *reinterpret_cast<uint2*>(sm + OFF_KPI + sw_off(row, ch, 64)) = pack4(kp01, kp23);
         if constexpr (kRead)
-          *reinterpret_cast<uint2*>(sm + OFF_QPI + sw_off(row, ch, 64)) = pack4(qp[0], qp[1], qp[2], qp[3]);
+          *reinterpret_cast<uint2*>(sm + OFF_QPI + sw_off(row, ch, 64)) = pack4(qp01, qp23);
         *reinterpret_cast<uint2*>(sm + OFF_KC + sw_off(row, ch, 64)) =
-            pack4(ks[0] * nextb[0], ks[1] * nextb[1], ks[2] * nextb[2], ks[3] * nextb[3]);
-        *reinterpret_cast<uint2*>(sm + OFF_KK8 + sw_off(r32, ch, 32)) = ks_b;
+            pack4(mul_f32x2(ks01, nb01), mul_f32x2(ks23, nb23));
+        *reinterpret_cast<uint2*>(sm + OFF_KK8 + sw_off(r32, ch, 32)) = pack4(ks01, ks23);
       }
       // K' = K o (decay to the chunk end), token rows like the other tiles: the update reads it
       // as the MN-major B operand K'^T
       *reinterpret_cast<uint2*>(sm + OFF_KPT + sw_off(row, ch, 64)) =
-          pack4(ks[0] * suf[0], ks[1] * suf[1], ks[2] * suf[2], ks[3] * suf[3]);
+          pack4(mul_f32x2(ks01, suf01), mul_f32x2(ks23, suf23));
     }
 
     fence_async_smem();  // the operand tiles are read by the tensor cores
