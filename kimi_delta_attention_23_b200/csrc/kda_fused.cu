@@ -123,6 +123,27 @@ __device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
 }
+__device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+// a . b over four channels held as two pairs (pairwise: (a0 b0 + a2 b2) + (a1 b1 + a3 b3))
+__device__ __forceinline__ float dot4(float2 a01, float2 a23, float2 b01, float2 b23) {
+  const float2 t = fma_f32x2(a23, b23, mul_f32x2(a01, b01));
+  return t.x + t.y;
+}
 __device__ __forceinline__ uint2 pack4(float2 lo, float2 hi) {
   return make_uint2(pack_bf16(lo.x, lo.y), pack_bf16(hi.x, hi.y));
 }
@@ -354,16 +375,32 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       float o[4] = {1.f, 1.f, 1.f, 1.f};
       if (row < Ln) {
         const float4 raw = *cell;
-        const float xs[4] = {raw.x + dtb.x, raw.y + dtb.y, raw.z + dtb.z, raw.w + dtb.w};
+        // softplus(x) in log2 units, log2(1 + 2^(x log2 e)), then alpha = exp(-exp(a_log)
+        // softplus(x)) = 2^(-c sp2); the limits come out right on both sides (x large: the power
+        // overflows to inf and alpha = 0; x very negative: it flushes to 0 and alpha = 1).  In the
+        // build the plain arithmetic runs on channel pairs (the special functions one value at
+        // a time); the prefill keeps one value at a time, which measured faster there.  The
+        // roundings are the same either way.
+        if constexpr (kBuild) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const float x = xs[c];
-          // softplus(x) in log2 units, log2(1 + 2^(x log2 e)), then alpha = exp(-exp(a_log)
-          // softplus(x)) = 2^(-c sp2); the limits come out right on both sides (x large: the power
-          // overflows to inf and alpha = 0; x very negative: it flushes to 0 and alpha = 1)
-          const float sp2 = fast_lg2(1.f + fast_ex2(x * kLog2e));
-          const float al_c = fast_ex2(-cexp * sp2);
-          o[c] = safe ? fmaxf(al_c, alpha_floor) : al_c;
+          for (int c = 0; c < 4; c += 2) {
+            const float2 x = add_f32x2(c ? make_float2(raw.z, raw.w) : make_float2(raw.x, raw.y),
+                                       c ? make_float2(dtb.z, dtb.w) : make_float2(dtb.x, dtb.y));
+            const float2 xl = mul_f32x2(x, make_float2(kLog2e, kLog2e));
+            const float2 e = add_f32x2(make_float2(1.f, 1.f), make_float2(fast_ex2(xl.x), fast_ex2(xl.y)));
+            const float2 y = mul_f32x2(make_float2(-cexp, -cexp), make_float2(fast_lg2(e.x), fast_lg2(e.y)));
+            const float a0 = fast_ex2(y.x), a1 = fast_ex2(y.y);
+            o[c] = safe ? fmaxf(a0, alpha_floor) : a0;
+            o[c + 1] = safe ? fmaxf(a1, alpha_floor) : a1;
+          }
+        } else {
+          const float xs[4] = {raw.x + dtb.x, raw.y + dtb.y, raw.z + dtb.z, raw.w + dtb.w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float sp2 = fast_lg2(1.f + fast_ex2(xs[c] * kLog2e));
+            const float al_c = fast_ex2(-cexp * sp2);
+            o[c] = safe ? fmaxf(al_c, alpha_floor) : al_c;
+          }
         }
       }
       *cell = make_float4(o[0], o[1], o[2], o[3]);
@@ -428,12 +465,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       for (int i = 28; i < 32; ++i) acc[i] = 0.f;
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        float w[4] = {kf[s][0], kf[s][1], kf[s][2], kf[s][3]};
+        float2 w01 = make_float2(kf[s][0], kf[s][1]), w23 = make_float2(kf[s][2], kf[s][3]);
 #pragma unroll
         for (int r = s + 1; r < 8; ++r) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) w[c] *= al[r][c];
-          acc[r * (r - 1) / 2 + s] = kf[r][0] * w[0] + kf[r][1] * w[1] + kf[r][2] * w[2] + kf[r][3] * w[3];
+          w01 = mul_f32x2(w01, make_float2(al[r][0], al[r][1]));
+          w23 = mul_f32x2(w23, make_float2(al[r][2], al[r][3]));
+          acc[r * (r - 1) / 2 + s] =
+              dot4(make_float2(kf[r][0], kf[r][1]), make_float2(kf[r][2], kf[r][3]), w01, w23);
         }
       }
 #pragma unroll
@@ -454,14 +492,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       float acc[64];
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        float w[4] = {kf[s][0], kf[s][1], kf[s][2], kf[s][3]};
-        acc[28 + s * (s + 1) / 2 + s] = qf[s][0] * w[0] + qf[s][1] * w[1] + qf[s][2] * w[2] + qf[s][3] * w[3];
+        float2 w01 = make_float2(kf[s][0], kf[s][1]), w23 = make_float2(kf[s][2], kf[s][3]);
+        acc[28 + s * (s + 1) / 2 + s] =
+            dot4(make_float2(qf[s][0], qf[s][1]), make_float2(qf[s][2], qf[s][3]), w01, w23);
 #pragma unroll
         for (int r = s + 1; r < 8; ++r) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) w[c] *= al[r][c];
-          acc[r * (r - 1) / 2 + s] = kf[r][0] * w[0] + kf[r][1] * w[1] + kf[r][2] * w[2] + kf[r][3] * w[3];
-          acc[28 + r * (r + 1) / 2 + s] = qf[r][0] * w[0] + qf[r][1] * w[1] + qf[r][2] * w[2] + qf[r][3] * w[3];
+          w01 = mul_f32x2(w01, make_float2(al[r][0], al[r][1]));
+          w23 = mul_f32x2(w23, make_float2(al[r][2], al[r][3]));
+          acc[r * (r - 1) / 2 + s] =
+              dot4(make_float2(kf[r][0], kf[r][1]), make_float2(kf[r][2], kf[r][3]), w01, w23);
+          acc[28 + r * (r + 1) / 2 + s] =
+              dot4(make_float2(qf[r][0], qf[r][1]), make_float2(qf[r][2], qf[r][3]), w01, w23);
         }
       }
 #pragma unroll
@@ -490,18 +531,20 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     // in-block products: p8 inclusive prefix from the block start, s8 exclusive suffix
     float p8[8][4], s8[8][4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float acc = 1.f;
+    for (int c = 0; c < 4; c += 2) {
+      float2 acc = make_float2(1.f, 1.f);
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        acc *= al[r][c];
-        p8[r][c] = acc;
+        acc = mul_f32x2(acc, make_float2(al[r][c], al[r][c + 1]));
+        p8[r][c] = acc.x;
+        p8[r][c + 1] = acc.y;
       }
-      acc = 1.f;
+      acc = make_float2(1.f, 1.f);
 #pragma unroll
       for (int r = 7; r >= 0; --r) {
-        s8[r][c] = acc;
-        acc *= al[r][c];
+        s8[r][c] = acc.x;
+        s8[r][c + 1] = acc.y;
+        acc = mul_f32x2(acc, make_float2(al[r][c], al[r][c + 1]));
       }
     }
     *reinterpret_cast<float4*>(sTau + warp * D + ch) = make_float4(p8[7][0], p8[7][1], p8[7][2], p8[7][3]);
