@@ -671,12 +671,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(128), kk > 0);
         }
       } else {
-        // D1_M = S_M^T (K o Gamma)^T and D1_U = S_U^T (K o Gamma)^T   (N = 64 each, K = 128)
+        // D1_M = -S_M^T (K o Gamma)^T and D1_U = -S_U^T (K o Gamma)^T   (N = 64 each, K = 128; the
+        // instruction negates K o Gamma, so the epilogue stores Y^T as it comes)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
-          mma_bf16_ts(tmD1u, tmSbu + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idesc_bf16_f32(64), kk > 0);
+          constexpr uint32_t idn = idesc_bf16_f32(64, false, false, true);
+          mma_bf16_ts(tmD1, tmSb + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idn, kk > 0);
+          mma_bf16_ts(tmD1u, tmSbu + 8 * kk, desc_sw128(sbase + OFF_KQ + koff), idn, kk > 0);
         }
       }
       mma_commit(bar0);
@@ -821,8 +823,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       if (warp >= 4) {
         // warps 4..7 have no part in the first doubling level: they run the state side's first
         // epilogue (the first product was issued after (2)); warp -> TMEM lane quadrant warp % 4,
-        // all 64 columns.  Y^T[j][r] = -D1[j][r] = -((K o Gamma) S0)^T into the X tile(s); V
-        // enters in the next product
+        // all 64 columns.  Y^T[j][r] = -((K o Gamma) S0)^T into the X tile(s) (in the build the
+        // products computed it negated; the prefill's one N = 128 product negates here); V enters
+        // in the next product
         if (!mbar_wait_bounded(bar0, phase, kWaitLimitNs)) {
           *s_abort = 1;
           report(a.status, KDA_ERR_DEVICE_TIMEOUT);
@@ -837,8 +840,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
 #pragma unroll
             for (int r0 = 0; r0 < 64; r0 += 8)
               *reinterpret_cast<uint4*>(sm + xoff + sw_off(ej, r0, 128)) =
-                  make_uint4(pack_bf16(-d[r0], -d[r0 + 1]), pack_bf16(-d[r0 + 2], -d[r0 + 3]),
-                             pack_bf16(-d[r0 + 4], -d[r0 + 5]), pack_bf16(-d[r0 + 6], -d[r0 + 7]));
+                  kBuild ? make_uint4(pack_bf16(d[r0], d[r0 + 1]), pack_bf16(d[r0 + 2], d[r0 + 3]),
+                                      pack_bf16(d[r0 + 4], d[r0 + 5]), pack_bf16(d[r0 + 6], d[r0 + 7]))
+                         : make_uint4(pack_bf16(-d[r0], -d[r0 + 1]), pack_bf16(-d[r0 + 2], -d[r0 + 3]),
+                                      pack_bf16(-d[r0 + 4], -d[r0 + 5]), pack_bf16(-d[r0 + 6], -d[r0 + 7]));
           }
         }
         fence_async_smem();

@@ -135,10 +135,12 @@ __device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t saddr, uint32_t mn_st
 }
 
 // Instruction descriptor: kind::f16 with bf16 A and B, fp32 accumulator, M = 128, N = n
-// (multiple of 16, 16..256); A and B K-major, or MN-major with a_mn_major / b_mn_major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t n, bool a_mn_major = false, bool b_mn_major = false) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
-         ((n >> 3) << 17) | ((128u >> 4) << 24);
+// (multiple of 16, 16..256); A and B K-major, or MN-major with a_mn_major / b_mn_major; B
+// negated with b_negate (D = A (-B)^T).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t n, bool a_mn_major = false, bool b_mn_major = false,
+                                                     bool b_negate = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_negate ? 1u : 0u) << 14) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((b_mn_major ? 1u : 0u) << 16) | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
