@@ -109,6 +109,14 @@ def test_binding_refuses_cpu_tensors():
                           torch.zeros(1, dtype=torch.int32))
 
 
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    # no fallback of any kind: without the built library the binding refuses to load
+    monkeypatch.setattr(kda, "LIB_PATH", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(kda, "_lib", None)
+    with pytest.raises(ImportError, match="not built"):
+        kda.load_library()
+
+
 def test_context_parallel_host_checks(lib):
     p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
     # apply: null pointers, dv != 128
