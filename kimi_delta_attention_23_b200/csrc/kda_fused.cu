@@ -22,12 +22,12 @@
 //   * k-side (all 8 warps): gates, in-chunk decay products, operand tiles; scores A and P --
 //     8x8 diagonal blocks on CUDA cores (a product recursion along the rows), the rest with
 //     mma.sync on operands scaled by a reference point that sits between rows and columns
-//     (both factors <= 1); the blocked triangular inverse T on CUDA cores.
+//     (both factors <= 1); the blocked triangular inverse T (CUDA cores, then tf32 mma.sync).
 //   * state side: the four products that touch S run on tcgen05 with the state transposed
 //     (dv = 128 rows = the 128 TMEM lanes): D1 = S^T [K o Gamma; Q o Gamma]^T, D2 = X^T T^T,
 //     D1o += Delta^T P^T, S^T += Delta^T K'.  S^T stays in TMEM in fp32 across chunks; a bf16
 //     copy, also in TMEM, is the A operand of the next chunk's first product.  All eight warps
-//     run the epilogues (two per TMEM lane quadrant); thread 128 issues the MMAs.
+//     run the epilogues (two per TMEM lane quadrant); four threads issue the MMAs (below).
 #include <cuda.h>
 #include <string.h>
 
