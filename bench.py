@@ -74,15 +74,22 @@ def decode_bytes(w):
 
 
 def segment_build_bytes(w, N, dk=128, dv=128):
-    """Segment build with readouts (q, k, v, gate, beta in; both bf16 readouts, M and U out) plus
-    the scan (M, U, initial in; incoming, outgoing, final out)."""
+    """The method's own bytes of the segment build plus the scan over N pieces: q, k, v, gate and
+    beta in (the straight pass's reads), M and U out; the scan reads M and U and writes the
+    incoming and outgoing states.  The per-token readouts the build also writes are this
+    design's intermediate (the apply reads them back), not the method's, and are counted apart
+    (``segment_build_intermediate_bytes``)."""
     th = w.total_tokens * w.num_v_heads
     group = w.num_v_heads // w.num_k_heads
     reads = th * ((2 * dk * 2) / group + dv * 2 + dk * 4 + 4)
-    readouts = th * 2 * dv * 2
     summaries = N * w.num_v_heads * (dk * dk + dk * dv) * 4
     scan = summaries + N * w.num_v_heads * dk * dv * 4 * 2
-    return reads + readouts + summaries + scan
+    return reads + summaries + scan
+
+
+def segment_build_intermediate_bytes(w, dv=128):
+    """The build's two bf16 readouts per token-head (written here, read back by the apply)."""
+    return w.total_tokens * w.num_v_heads * 2 * dv * 2
 
 
 def apply_bytes(w, N, dv=128):
@@ -523,6 +530,9 @@ def run_ours(args):
             "frac": achieved / pk["hbm_gbs"], "traffic": recorded_traffic(dom),
             "algorithmic_bytes_per_launch": bytes_dom, "ms_per_launch": ms_dom,
             "peak_source": pk["source"]}
+    if step.cp:
+        # the readouts: written by this launch and read back by the apply; not the method's bytes
+        roof["intermediate_bytes_per_launch"] = segment_build_intermediate_bytes(w)
     line = {"metric": DECODE_METRIC if step.decode else METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.q.dtype == torch.bfloat16 else "f32", "data": "synthetic",
@@ -542,12 +552,58 @@ def run_ours(args):
                                               sm_mhz=line["clocks"].get("sm_mhz") or line["clocks"].get("sm_max_mhz"))
     if e2e is not None:
         line["e2e"] = e2e
+    if world == 1 and not args.no_workloads and args.workload == DEFAULT_WORKLOAD and not args.straight:
+        # the other headline and reported workloads, timed in the same run (the same protocol:
+        # W untimed steps, K timed ones bracketed by CUDA events on the launching stream, clocks
+        # sampled during them); the straight pass reuses this workload's inputs
+        del step
+        line["workloads"] = extra_workloads(w, args, stream, pk, dev)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args)
     print(json.dumps(line), flush=True)
     if pg is not None:
         pg.destroy_process_group()
     return 0
+
+
+EXTRA_WORKLOADS = (("long_T131072_H32_cp16 --straight", None), ("varlen8_H32_vfirst", "varlen8_H32_vfirst"),
+                   ("batch64_T2048_H16_safe", "batch64_T2048_H16_safe"), ("single_T4096_H16", "single_T4096_H16"))
+
+
+def time_workload(w, args, stream, pk, straight=False):
+    """One workload's step timed like the main one: its ms per step, tokens/s and the fraction of
+    its roofline (algorithmic bytes at the measured HBM bandwidth vs FLOPs at the bf16 peak)."""
+    step = Step(w, stream, straight=straight)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {int(step.status.item())} during warm-up")
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(stream.device.index or 0) as clocks:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        stop.record(stream)
+        torch.cuda.synchronize()
+    ms = start.elapsed_time(stop) / args.steps
+    roof = step_roofline(w, ms, step.N if step.cp else 0, pk)
+    return {"ms_per_step": ms, "tokens_per_s": w.total_tokens / (ms / 1e3), "tokens": w.total_tokens,
+            "num_v_heads": w.num_v_heads, "batch": w.batch, "gate_mode": w.gate_mode,
+            "state_layout": w.state_layout, "pass": "context_parallel" if step.cp else "straight",
+            "algorithmic_bytes": roof["algorithmic_bytes"], "gbs": roof["gbs"], "frac": roof["frac"],
+            "gpu_launches": step.launches() * args.steps, "steps": args.steps, "warmup": args.warmup,
+            "clocks": clocks.summary()}
+
+
+def extra_workloads(w_main, args, stream, pk, dev):
+    res = {}
+    for label, name in EXTRA_WORKLOADS:
+        w = w_main if name is None else W.make(name, device=dev)
+        res[label] = time_workload(w, args, stream, pk, straight=name is None)
+        del w
+        torch.cuda.empty_cache()
+    return res
 
 
 def measure_e2e(w, args, stream, pg):
@@ -644,6 +700,8 @@ def measure_e2e_host_pipelined(w, args, stream, pg):
     world = pg.get_world_size() if pg is not None else 1
     return {"value": whole_job_throughput(T, world, ms / n), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n, "api": "kda_prefill_host_pipelined",
+            "path": "the plain chunk kernel over consecutive segments of the sequence, copies in and out "
+                    "overlapped with it (not the context-parallel step timed on the device)",
             "segment_tokens": seg}
 
 
@@ -703,6 +761,8 @@ def main():
                          "the context-parallel step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads timed after the default one (the 'workloads' key)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--profile-launches", type=int, default=0,

@@ -48,8 +48,9 @@
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
  *    default stream).  The returned status covers the host-side checks and the launch only.
  *  - Host-side checks are always on: null pointers, extents, Hv % Hk == 0, dtype groupings
- *    that bind no kernel, flag combinations.  A failed check returns before any launch and
- *    writes nothing.
+ *    that bind no kernel, flag combinations, and token counts within int32 (token offsets are
+ *    int32, as cu_seqlens; a larger T returns KDA_ERR_INVALID_ARG).  A failed check returns
+ *    before any launch and writes nothing.
  *  - device_status (nullable, device int32): kernels record the first device-side finding
  *    there (KDA_ERR_DEVICE_CHECK for a state slot outside [0, max_slots) or decreasing
  *    offsets -- that sequence is skipped and its slot and outputs are left untouched;
@@ -273,9 +274,12 @@ KDA_API kda_status_t kda_context_parallel_prefill(
  * return KDA_ERR_WORKSPACE and do nothing.  The call allocates nothing: no cudaMalloc, no
  * cudaFree, no allocating library routine.  The first call on a device looks up the array's
  * device address (once per device, with that device current); make that first call before any
- * stream capture.  Every call shares the one array and leaves its last contents there (nothing
- * in it needs to start at zero); calls whose work overlaps on the GPU (other streams, or other
- * host threads) race on it and must be serialised by the caller.
+ * stream capture.  The address is kept for the process and belongs to the device's primary
+ * context: a caller that destroys that context (cudaDeviceReset) and keeps using the library
+ * on the device gets a stale address.  Every call shares the one array and leaves its last
+ * contents there (nothing in it needs to start at zero); calls whose work overlaps on the GPU
+ * (other streams, or other host threads) race on it and must be serialised by the caller.
+ * T beyond INT32_MAX (token offsets are int32) returns KDA_ERR_INVALID_ARG.
  */
 KDA_API kda_status_t kda_context_parallel_prefill_static(
     const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype, const float *raw_gate,
@@ -285,7 +289,8 @@ KDA_API kda_status_t kda_context_parallel_prefill_static(
     float *final_state, float *M, float *U, float *incoming, float *outgoing, uint32_t flags,
     float gate_lower_bound, int32_t *device_status, void *stream);
 
-/* Workspace bytes kda_context_parallel_prefill needs: the two bf16 readouts, 2 * T * Hv * dv * 2. */
+/* Workspace bytes kda_context_parallel_prefill needs: the two bf16 readouts, 2 * T * Hv * dv * 2
+ * (SIZE_MAX for T beyond INT32_MAX, which no call accepts: token offsets are int32). */
 KDA_API size_t kda_context_parallel_workspace_size(int64_t T, int32_t num_v_heads, int32_t dv);
 
 /*
@@ -390,7 +395,10 @@ KDA_API kda_status_t kda_context_parallel_range_finish(
  * Asynchronous on `stream`: the kernels run there and the stream completes after the last
  * copy out; read the host outputs after synchronising it.  The copies run on two helper
  * streams the library creates on a device's first call and keeps (with four events); calls are
- * serialised while they enqueue.  bf16 q/k/v with dk = dv = 128 only; else KDA_ERR_UNSUPPORTED.
+ * serialised while they enqueue.  Those streams and events belong to the device's primary
+ * context and are kept for the process: a caller that destroys that context
+ * (cudaDeviceReset) leaves them stale, and later calls on the device fail.  bf16 q/k/v with
+ * dk = dv = 128 only; else KDA_ERR_UNSUPPORTED.
  */
 KDA_API size_t kda_prefill_host_workspace_size(int64_t T, int32_t num_k_heads, int32_t num_v_heads,
                                                kda_dtype_t out_dtype, int64_t segment_tokens);

@@ -181,6 +181,38 @@ def _stream(stream, device):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+class _Owned:
+    """Device tensors a wrapper allocates itself (results and scratch).
+
+    PyTorch's caching allocator ties a block to the stream that was current when it was
+    allocated.  The kernels run on ``stream``; when that is another stream, every such tensor is
+    marked as in use there (``record_stream``), so that its memory goes to other work only after
+    the kernels on ``stream`` are done with it -- the scratch a wrapper drops at return as much as
+    a result the caller frees later."""
+
+    def __init__(self, stream, device):
+        self.stream, self.device, self.tensors = stream, device, []
+
+    def empty(self, *shape, **kw):
+        t = torch.empty(*shape, **kw)
+        self.tensors.append(t)
+        return t
+
+    def keep(self, t, original=None):
+        # a temporary made from a caller's tensor (.contiguous() and the like); the caller's own
+        # tensor is left alone
+        if original is None or t.data_ptr() != original.data_ptr():
+            self.tensors.append(t)
+        return t
+
+    def launched(self):
+        if self.stream is None or self.stream == torch.cuda.current_stream(self.device):
+            return
+        for t in self.tensors:
+            if t.numel() and t.device.type == "cuda":
+                t.record_stream(self.stream)
+
+
 def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, state_pool, state_indices,
                   out=None, *, output_dtype=None, use_computebound=False, gate_mode="original",
                   beta_mode="logits", state_layout="K_FIRST", gate_lower_bound=-5.0, force_simt=False,
@@ -196,6 +228,7 @@ def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, st
     """
     lib = load_library()
     dev = q.device
+    own = _Owned(stream, dev)
     _dev(q, "q", device=dev)
     if q.dtype not in _DTYPES:
         raise ValueError("q/k/v must be float32 or bfloat16")
@@ -222,7 +255,7 @@ def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, st
     if output_dtype not in _DTYPES:
         raise ValueError("output_dtype must be float32 or bfloat16")
     if out is None:
-        out = torch.empty((T, Hv, dv), dtype=output_dtype, device=dev)
+        out = own.empty((T, Hv, dv), dtype=output_dtype, device=dev)
     _shape(_dev(out, "out", output_dtype, dev), "out", (T, Hv, dv))
     if device_status is not None:
         _shape(_dev(device_status, "device_status", torch.int32, dev), "device_status", (1,))
@@ -232,7 +265,7 @@ def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, st
         if q.dtype == torch.bfloat16 and not force_simt:
             with torch.cuda.device(dev):
                 need = kda_workspace_size(T, B, Hk, Hv, dk, dv, 0, flags)
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        workspace = own.empty(need, dtype=torch.uint8, device=dev)
     _dev(workspace, "workspace", torch.uint8, dev)
     rc = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], _ptr(raw_gate), _ptr(beta_logits),
                            _ptr(a_log), _ptr(dt_bias), _ptr(cu_seqlens), B, T, Hk, Hv, dk, dv,
@@ -240,6 +273,7 @@ def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, st
                            _DTYPES[output_dtype], flags, float(gate_lower_bound),
                            _ptr(workspace) if workspace.numel() else None, workspace.numel(),
                            _ptr(device_status), _stream(stream, dev))
+    own.launched()
     if rc != 0:
         raise KdaError(rc, "kda_chunk_fwd")
     return out
@@ -256,6 +290,7 @@ def kda_decode(q, k, v, raw_gate, beta_logits, a_log, dt_bias, state_pool, state
     """
     lib = load_library()
     dev = q.device
+    own = _Owned(stream, dev)
     _dev(q, "q", device=dev)
     if q.dtype not in _DTYPES:
         raise ValueError("q/k/v must be float32 or bfloat16")
@@ -281,7 +316,7 @@ def kda_decode(q, k, v, raw_gate, beta_logits, a_log, dt_bias, state_pool, state
     if output_dtype not in _DTYPES:
         raise ValueError("output_dtype must be float32 or bfloat16")
     if out is None:
-        out = torch.empty((B, Hv, dv), dtype=output_dtype, device=dev)
+        out = own.empty((B, Hv, dv), dtype=output_dtype, device=dev)
     _shape(_dev(out, "out", output_dtype, dev), "out", (B, Hv, dv))
     if device_status is not None:
         _shape(_dev(device_status, "device_status", torch.int32, dev), "device_status", (1,))
@@ -290,6 +325,7 @@ def kda_decode(q, k, v, raw_gate, beta_logits, a_log, dt_bias, state_pool, state
                         _ptr(dt_bias), B, Hk, Hv, dk, dv, _ptr(state_pool), state_pool.shape[0],
                         _ptr(state_indices), _ptr(out), _DTYPES[output_dtype], flags, float(gate_lower_bound),
                         _ptr(device_status), _stream(stream, dev))
+    own.launched()
     if rc != 0:
         raise KdaError(rc, "kda_decode")
     return out
@@ -311,6 +347,7 @@ def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, 
     """
     lib = load_library()
     dev = initial_state.device
+    own = _Owned(stream, dev)
     _dev(initial_state, "initial_state", torch.float32, dev)
     Hv = initial_state.shape[0]
     N = seg_offsets.numel() - 1
@@ -339,7 +376,7 @@ def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, 
 
     def buf(t, name, shape):
         if t is None:
-            return torch.empty(shape, dtype=torch.float32, device=dev)
+            return own.empty(shape, dtype=torch.float32, device=dev)
         _shape(_dev(t, name, torch.float32, dev), name, shape)
         return t
 
@@ -352,9 +389,9 @@ def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, 
         _shape(_dev(q, "q", torch.bfloat16, dev), "q", (T, Hk, dk))
         rshape = _readout_shape(T, Hv, dv, readout_layout)
         if readout_m is None:
-            readout_m = torch.empty(rshape, dtype=torch.bfloat16, device=dev)
+            readout_m = own.empty(rshape, dtype=torch.bfloat16, device=dev)
         if readout_u is None:
-            readout_u = torch.empty(rshape, dtype=torch.bfloat16, device=dev)
+            readout_u = own.empty(rshape, dtype=torch.bfloat16, device=dev)
         _shape(_dev(readout_m, "readout_m", torch.bfloat16, dev), "readout_m", rshape)
         _shape(_dev(readout_u, "readout_u", torch.bfloat16, dev), "readout_u", rshape)
     flags = _flags(gate_mode, beta_mode, state_layout, scan_only=scan_only)
@@ -367,6 +404,7 @@ def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, 
         _ptr(seg_offsets) if not scan_only else None, N, _ptr(initial_state), _ptr(M), _ptr(U),
         _ptr(incoming), _ptr(outgoing), _ptr(final_state), _ptr(q), _ptr(readout_m), _ptr(readout_u), flags,
         float(gate_lower_bound), None, 0, _ptr(device_status), _stream(stream, dev))
+    own.launched()
     if rc != 0:
         raise KdaError(rc, "kda_segment_summarize_and_scan")
     res = {"incoming_states": incoming, "outgoing_states": outgoing, "final_state": final_state,
@@ -382,6 +420,7 @@ def kda_context_parallel_apply(readout_m, readout_u, incoming, seg_offsets, out=
     or [Hv, T, 128] with ``readout_layout="head_major"``; out [T, Hv, 128] either way)."""
     lib = load_library()
     dev = incoming.device
+    own = _Owned(stream, dev)
     _dev(readout_m, "readout_m", torch.bfloat16, dev)
     rflags = _readout_flags(readout_layout)
     if readout_layout == "head_major":
@@ -393,12 +432,13 @@ def kda_context_parallel_apply(readout_m, readout_u, incoming, seg_offsets, out=
     _dev(seg_offsets, "seg_offsets", torch.int32, dev)
     N = seg_offsets.numel() - 1
     if out is None:
-        out = torch.empty((T, Hv, dv), dtype=output_dtype, device=dev)
+        out = own.empty((T, Hv, dv), dtype=output_dtype, device=dev)
     _shape(_dev(out, "out", None, dev), "out", (T, Hv, dv))
     rc = lib.kda_context_parallel_apply(_ptr(readout_m), _ptr(readout_u), _ptr(incoming), _ptr(seg_offsets), N, T,
                                         Hv, dv, _ptr(out), _DTYPES[out.dtype],
                                         _flags("original", "logits", state_layout) | rflags,
                                         _ptr(device_status), _stream(stream, dev))
+    own.launched()
     if rc != 0:
         raise KdaError(rc, "kda_context_parallel_apply")
     return out
@@ -422,10 +462,12 @@ def kda_context_parallel(transition_matrices, local_contributions, initial_state
         M, U, S0 = M.unsqueeze(1), U.unsqueeze(1), S0.unsqueeze(0)
     if M.shape[0] < 1:
         raise ValueError("at least one segment is required")
+    own = _Owned(stream, S0.device)
+    Mc, Uc, Sc = own.keep(M.contiguous(), M), own.keep(U.contiguous(), U), own.keep(S0.contiguous(), S0)
     res = kda_segment_summarize_and_scan(None, None, None, None, None, None,
-                                         torch.zeros(M.shape[0] + 1, dtype=torch.int32), S0.contiguous(),
-                                         M=M.contiguous(), U=U.contiguous(), scan_only=True,
-                                         state_layout=state_layout, stream=stream)
+                                         torch.zeros(M.shape[0] + 1, dtype=torch.int32), Sc,
+                                         M=Mc, U=Uc, scan_only=True, state_layout=state_layout, stream=stream)
+    own.launched()
     out = {k: res[k] for k in ("incoming_states", "outgoing_states", "final_state")}
     if squeeze:
         out = {"incoming_states": out["incoming_states"][:, 0], "outgoing_states": out["outgoing_states"][:, 0],
@@ -446,12 +488,14 @@ def kda_context_parallel_piece_offsets(seg_offsets, pieces, *, out=None, stream=
     """Chunk-aligned boundaries of ``pieces`` pieces per segment (device int32 [N*pieces + 1])."""
     lib = load_library()
     dev = seg_offsets.device
+    own = _Owned(stream, dev)
     _dev(seg_offsets, "seg_offsets", torch.int32, dev)
     N = seg_offsets.numel() - 1
     if out is None:
-        out = torch.empty(N * pieces + 1, dtype=torch.int32, device=dev)
+        out = own.empty(N * pieces + 1, dtype=torch.int32, device=dev)
     _shape(_dev(out, "out", torch.int32, dev), "out", (N * pieces + 1,))
     rc = lib.kda_context_parallel_piece_offsets(_ptr(seg_offsets), N, pieces, _ptr(out), _stream(stream, dev))
+    own.launched()
     if rc != 0:
         raise KdaError(rc, "kda_context_parallel_piece_offsets")
     return out
@@ -465,6 +509,7 @@ def kda_segment_compose(M_pieces, U_pieces, incoming_pieces, final_state, pieces
     """
     lib = load_library()
     dev = M_pieces.device
+    own = _Owned(stream, dev)
     _dev(M_pieces, "M_pieces", torch.float32, dev)
     NP, Hv, dk = M_pieces.shape[0], M_pieces.shape[1], M_pieces.shape[2]
     if NP % pieces:
@@ -480,7 +525,7 @@ def kda_segment_compose(M_pieces, U_pieces, incoming_pieces, final_state, pieces
 
     def buf(t, name, shape):
         if t is None:
-            return torch.empty(shape, dtype=torch.float32, device=dev)
+            return own.empty(shape, dtype=torch.float32, device=dev)
         _shape(_dev(t, name, torch.float32, dev), name, shape)
         return t
 
@@ -491,6 +536,7 @@ def kda_segment_compose(M_pieces, U_pieces, incoming_pieces, final_state, pieces
     rc = lib.kda_segment_compose(_ptr(M_pieces), _ptr(U_pieces), _ptr(incoming_pieces), _ptr(final_state), N,
                                  pieces, Hv, dk, dv, _ptr(M), _ptr(U), _ptr(incoming), _ptr(outgoing),
                                  _flags("original", "logits", state_layout), _stream(stream, dev))
+    own.launched()
     if rc != 0:
         raise KdaError(rc, "kda_segment_compose")
     return {"transition_matrices": M, "local_contributions": U, "incoming_states": incoming,
@@ -514,6 +560,7 @@ def kda_context_parallel_prefill(q, k, v, raw_gate, beta_logits, a_log, dt_bias,
     """
     lib = load_library()
     dev = q.device
+    own = _Owned(stream, dev)
     _dev(q, "q", torch.bfloat16, dev)
     T, Hk, dk = q.shape
     _shape(_dev(k, "k", torch.bfloat16, dev), "k", (T, Hk, dk))
@@ -531,12 +578,12 @@ def kda_context_parallel_prefill(q, k, v, raw_gate, beta_logits, a_log, dt_bias,
     if output_dtype is None:
         output_dtype = v.dtype if out is None else out.dtype
     if out is None:
-        out = torch.empty((T, Hv, dv), dtype=output_dtype, device=dev)
+        out = own.empty((T, Hv, dv), dtype=output_dtype, device=dev)
     _shape(_dev(out, "out", output_dtype, dev), "out", (T, Hv, dv))
 
     def buf(t, name, shape):
         if t is None:
-            return torch.empty(shape, dtype=torch.float32, device=dev)
+            return own.empty(shape, dtype=torch.float32, device=dev)
         _shape(_dev(t, name, torch.float32, dev), name, shape)
         return t
 
@@ -548,7 +595,7 @@ def kda_context_parallel_prefill(q, k, v, raw_gate, beta_logits, a_log, dt_bias,
     if workspace is None:
         with torch.cuda.device(dev):
             pref = kda_context_parallel_workspace_preferred(T, N, Hv, dv)
-        workspace = torch.empty(max(pref, 1), dtype=torch.uint8, device=dev)
+        workspace = own.empty(max(pref, 1), dtype=torch.uint8, device=dev)
     _dev(workspace, "workspace", torch.uint8, dev)
     flags = _flags(gate_mode, beta_mode, state_layout)
     rc = lib.kda_context_parallel_prefill(_ptr(q), _ptr(k), _ptr(v), _BF16, _ptr(raw_gate), _ptr(beta_logits),
@@ -557,6 +604,7 @@ def kda_context_parallel_prefill(q, k, v, raw_gate, beta_logits, a_log, dt_bias,
                                           _ptr(M), _ptr(U), _ptr(incoming), _ptr(outgoing), flags,
                                           float(gate_lower_bound), _ptr(workspace), workspace.numel(),
                                           _ptr(device_status), _stream(stream, dev))
+    own.launched()
     if rc != 0:
         raise KdaError(rc, "kda_context_parallel_prefill")
     return {"out": out, "final_state": final_state, "incoming_states": incoming, "outgoing_states": outgoing,
@@ -584,6 +632,7 @@ def kda_context_parallel_range_summary(q, k, v, raw_gate, beta_logits, a_log, dt
     """
     lib = load_library()
     dev = q.device
+    own = _Owned(stream, dev)
     _dev(q, "q", torch.bfloat16, dev)
     T, Hk, dk = q.shape
     _shape(_dev(k, "k", torch.bfloat16, dev), "k", (T, Hk, dk))
@@ -598,21 +647,22 @@ def kda_context_parallel_range_summary(q, k, v, raw_gate, beta_logits, a_log, dt
     N = seg_offsets.numel() - 1
     st = (dk, dv) if state_layout == "K_FIRST" else (dv, dk)
     if range_transition is None:
-        range_transition = torch.empty((Hv, dk, dk), dtype=torch.float32, device=dev)
+        range_transition = own.empty((Hv, dk, dk), dtype=torch.float32, device=dev)
     _shape(_dev(range_transition, "range_transition", torch.float32, dev), "range_transition", (Hv, dk, dk))
     if range_contribution is None:
-        range_contribution = torch.empty((Hv, *st), dtype=torch.float32, device=dev)
+        range_contribution = own.empty((Hv, *st), dtype=torch.float32, device=dev)
     _shape(_dev(range_contribution, "range_contribution", torch.float32, dev), "range_contribution", (Hv, *st))
     if workspace is None:
         with torch.cuda.device(dev):
             need = kda_context_parallel_range_workspace_size(T, max(N, 1), Hv, dv)
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        workspace = own.empty(max(need, 1), dtype=torch.uint8, device=dev)
     _dev(workspace, "workspace", torch.uint8, dev)
     rc = lib.kda_context_parallel_range_summary(
         _token_ptr(q, T), _token_ptr(k, T), _token_ptr(v, T), _BF16, _token_ptr(raw_gate, T),
         _token_ptr(beta_logits, T), _ptr(a_log), _ptr(dt_bias), T, Hk, Hv, dk, dv, _ptr(seg_offsets), N,
         _ptr(range_transition), _ptr(range_contribution), _flags(gate_mode, beta_mode, state_layout),
         float(gate_lower_bound), _ptr(workspace), workspace.numel(), _ptr(device_status), _stream(stream, dev))
+    own.launched()
     if rc != 0:
         raise KdaError(rc, "kda_context_parallel_range_summary")
     return {"range_transition": range_transition, "range_contribution": range_contribution, "workspace": workspace}
@@ -630,6 +680,7 @@ def kda_context_parallel_range_finish(range_incoming, workspace, seg_offsets, to
     """
     lib = load_library()
     dev = range_incoming.device
+    own = _Owned(stream, dev)
     _dev(range_incoming, "range_incoming", torch.float32, dev)
     Hv, st = range_incoming.shape[0], tuple(range_incoming.shape[1:])
     dk = dv = 128
@@ -639,12 +690,12 @@ def kda_context_parallel_range_finish(range_incoming, workspace, seg_offsets, to
     N = seg_offsets.numel() - 1
     T = int(tokens)
     if out is None:
-        out = torch.empty((T, Hv, dv), dtype=output_dtype, device=dev)
+        out = own.empty((T, Hv, dv), dtype=output_dtype, device=dev)
     _shape(_dev(out, "out", output_dtype, dev), "out", (T, Hv, dv))
 
     def buf(t, name, shape):
         if t is None:
-            return torch.empty(shape, dtype=torch.float32, device=dev)
+            return own.empty(shape, dtype=torch.float32, device=dev)
         _shape(_dev(t, name, torch.float32, dev), name, shape)
         return t
 
@@ -657,6 +708,7 @@ def kda_context_parallel_range_finish(range_incoming, workspace, seg_offsets, to
         T, Hv, dk, dv, N, _ptr(range_incoming), _token_ptr(out, T), _DTYPES[output_dtype], _ptr(range_outgoing),
         _ptr(M), _ptr(U), _ptr(incoming), _ptr(outgoing), _flags("original", "logits", state_layout),
         _ptr(workspace), workspace.numel(), _ptr(device_status), _stream(stream, dev))
+    own.launched()
     if rc != 0:
         raise KdaError(rc, "kda_context_parallel_range_finish")
     return {"out": out, "range_outgoing": range_outgoing, "incoming_states": incoming, "outgoing_states": outgoing,
@@ -696,6 +748,7 @@ def kda_prefill_host_pipelined(q, k, v, raw_gate, beta_logits, a_log, dt_bias, i
     """
     lib = load_library()
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    own = _Owned(stream, dev)
     _host(q, "q", torch.bfloat16)
     T, Hk, dk = q.shape
     _shape(_host(k, "k", torch.bfloat16), "k", (T, Hk, dk))
@@ -721,13 +774,14 @@ def kda_prefill_host_pipelined(q, k, v, raw_gate, beta_logits, a_log, dt_bias, i
             need = kda_prefill_host_workspace_size(T, Hk, Hv, output_dtype, segment_tokens)
             if need == 0:
                 raise ValueError("segment_tokens must be a positive multiple of 64")
-            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+            workspace = own.empty(need, dtype=torch.uint8, device=dev)
         _dev(workspace, "workspace", torch.uint8, dev)
         rc = lib.kda_prefill_host_pipelined(
             _ptr(q), _ptr(k), _ptr(v), _BF16, _ptr(raw_gate), _ptr(beta_logits), _ptr(a_log), _ptr(dt_bias), T,
             Hk, Hv, dk, dv, _ptr(initial_state), _ptr(out), _DTYPES[output_dtype], _ptr(final_state),
             int(segment_tokens), _flags(gate_mode, beta_mode, state_layout), float(gate_lower_bound),
             _ptr(workspace), workspace.numel(), _ptr(device_status), _stream(stream, dev))
+    own.launched()
     if rc != 0:
         raise KdaError(rc, "kda_prefill_host_pipelined")
     return {"out": out, "final_state": final_state}

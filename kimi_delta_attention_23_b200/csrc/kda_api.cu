@@ -113,9 +113,9 @@ extern "C" kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* 
                                       size_t workspace_bytes, int32_t* device_status, void* stream) {
   (void)workspace;
   (void)workspace_bytes;
-  if (batch < 0 || total_tokens < 0 || num_k_heads <= 0 || num_v_heads <= 0 || dk <= 0 || dv <= 0 ||
-      max_slots <= 0)
-    return KDA_ERR_INVALID_ARG;
+  if (batch < 0 || total_tokens < 0 || total_tokens > INT32_MAX || num_k_heads <= 0 || num_v_heads <= 0 ||
+      dk <= 0 || dv <= 0 || max_slots <= 0)
+    return KDA_ERR_INVALID_ARG;  // token offsets are int32, as cu_seqlens
   if (num_v_heads % num_k_heads != 0) return KDA_ERR_INVALID_ARG;
   if ((flags & ~kKnownFlags) != 0 || (flags & KDA_SEG_SCAN_ONLY)) return KDA_ERR_INVALID_ARG;
   if (!cu_seqlens || !state_pool || !state_indices) return KDA_ERR_INVALID_ARG;
@@ -343,7 +343,7 @@ extern "C" kda_status_t kda_segment_summarize_and_scan(
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int v_first = (flags & KDA_STATE_V_FIRST) ? 1 : 0;
   if (!(flags & KDA_SEG_SCAN_ONLY)) {
-    if (T < 0 || num_k_heads <= 0 || num_v_heads % num_k_heads != 0) return KDA_ERR_INVALID_ARG;
+    if (T < 0 || T > INT32_MAX || num_k_heads <= 0 || num_v_heads % num_k_heads != 0) return KDA_ERR_INVALID_ARG;
     if (!seg_offsets || !a_log || !dt_bias) return KDA_ERR_INVALID_ARG;
     if (T > 0 && (!k || !v || !raw_gate || !beta_logits)) return KDA_ERR_INVALID_ARG;
     if (!dtype_ok(kv_dtype)) return KDA_ERR_UNSUPPORTED;
@@ -443,6 +443,7 @@ extern "C" kda_status_t kda_segment_summarize_and_scan(
 
 extern "C" size_t kda_context_parallel_workspace_size(int64_t T, int32_t num_v_heads, int32_t dv) {
   if (T < 0 || num_v_heads <= 0 || dv <= 0) return 0;
+  if (T > INT32_MAX) return SIZE_MAX;  // beyond the int32 token offsets: no workspace can serve it
   return (size_t)2 * (size_t)T * (size_t)num_v_heads * (size_t)dv * 2;
 }
 
@@ -492,7 +493,7 @@ extern "C" kda_status_t kda_segment_compose(const float* M_pieces, const float* 
 extern "C" size_t kda_context_parallel_workspace_preferred(int64_t T, int32_t num_segments, int32_t num_v_heads,
                                                            int32_t dv) {
   const size_t base = kda_context_parallel_workspace_size(T, num_v_heads, dv);
-  if (base == 0 || num_segments < 1) return base;
+  if (base == 0 || base == SIZE_MAX || num_segments < 1) return base;
   const int k = choose_pieces(T, num_segments, num_v_heads);
   return k > 1 ? round256(base) + pieces_bytes(num_segments, k, num_v_heads, dv, dv) : base;
 }
@@ -502,7 +503,7 @@ extern "C" kda_status_t kda_context_parallel_apply(const void* readout_m, const 
                                                    int32_t num_segments, int64_t T, int32_t num_v_heads, int32_t dv,
                                                    void* out, kda_dtype_t out_dtype, uint32_t flags,
                                                    int32_t* device_status, void* stream) {
-  if (num_segments < 1 || T < 0 || num_v_heads <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+  if (num_segments < 1 || T < 0 || T > INT32_MAX || num_v_heads <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
   if ((flags & ~kKnownFlags) != 0) return KDA_ERR_INVALID_ARG;
   if (!readout_m || !readout_u || !incoming || !seg_offsets || !out) return KDA_ERR_INVALID_ARG;
   if (!dtype_ok(out_dtype)) return KDA_ERR_UNSUPPORTED;
@@ -531,8 +532,8 @@ extern "C" kda_status_t kda_context_parallel_prefill(
     const float* initial_state, void* out, kda_dtype_t out_dtype, float* final_state, float* M, float* U,
     float* incoming, float* outgoing, uint32_t flags, float gate_lower_bound, void* workspace,
     size_t workspace_bytes, int32_t* device_status, void* stream) {
-  if (num_segments < 1 || T < 0 || num_k_heads <= 0 || num_v_heads <= 0 || dk <= 0 || dv <= 0)
-    return KDA_ERR_INVALID_ARG;
+  if (num_segments < 1 || T < 0 || T > INT32_MAX || num_k_heads <= 0 || num_v_heads <= 0 || dk <= 0 || dv <= 0)
+    return KDA_ERR_INVALID_ARG;  // token offsets are int32
   if ((flags & ~kKnownFlags) != 0 || (flags & (KDA_SEG_SCAN_ONLY | KDA_FORCE_SIMT))) return KDA_ERR_INVALID_ARG;
   if (!q || !out) return KDA_ERR_INVALID_ARG;
   if (!dtype_ok(qkv_dtype) || !dtype_ok(out_dtype)) return KDA_ERR_UNSUPPORTED;
@@ -627,6 +628,7 @@ bool range_workspace_ok(const void* ws, size_t bytes, int64_t T, int32_t N, int3
 extern "C" size_t kda_context_parallel_range_workspace_size(int64_t T, int32_t num_segments, int32_t num_v_heads,
                                                             int32_t dv) {
   if (T < 0 || num_segments < 1 || num_v_heads <= 0 || dv != 128) return 0;
+  if (T > INT32_MAX) return SIZE_MAX;
   return range_workspace_bytes(T, num_segments, num_v_heads, choose_pieces(T, num_segments, num_v_heads));
 }
 
@@ -636,7 +638,7 @@ extern "C" kda_status_t kda_context_parallel_range_summary(
     int32_t num_v_heads, int32_t dk, int32_t dv, const int32_t* seg_offsets, int32_t num_segments,
     float* range_M, float* range_U, uint32_t flags, float gate_lower_bound, void* workspace,
     size_t workspace_bytes, int32_t* device_status, void* stream) {
-  if (num_segments < 1 || T < 0 || num_k_heads <= 0 || num_v_heads <= 0 || dk <= 0 || dv <= 0)
+  if (num_segments < 1 || T < 0 || T > INT32_MAX || num_k_heads <= 0 || num_v_heads <= 0 || dk <= 0 || dv <= 0)
     return KDA_ERR_INVALID_ARG;
   if (num_v_heads % num_k_heads != 0) return KDA_ERR_INVALID_ARG;
   if ((flags & ~kKnownFlags) != 0 || (flags & (KDA_SEG_SCAN_ONLY | KDA_FORCE_SIMT))) return KDA_ERR_INVALID_ARG;
@@ -699,7 +701,8 @@ extern "C" kda_status_t kda_context_parallel_range_finish(
     int64_t T, int32_t num_v_heads, int32_t dk, int32_t dv, int32_t num_segments, const float* range_incoming,
     void* out, kda_dtype_t out_dtype, float* range_outgoing, float* M, float* U, float* incoming, float* outgoing,
     uint32_t flags, void* workspace, size_t workspace_bytes, int32_t* device_status, void* stream) {
-  if (num_segments < 1 || T < 0 || num_v_heads <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+  if (num_segments < 1 || T < 0 || T > INT32_MAX || num_v_heads <= 0 || dk <= 0 || dv <= 0)
+    return KDA_ERR_INVALID_ARG;
   if ((flags & ~kKnownFlags) != 0) return KDA_ERR_INVALID_ARG;
   if (!range_incoming || !M || !U || !incoming || !outgoing || (T > 0 && !out)) return KDA_ERR_INVALID_ARG;
   if (!dtype_ok(out_dtype)) return KDA_ERR_UNSUPPORTED;

@@ -13,6 +13,7 @@
 // address up with cudaGetSymbolAddress, once per device, with that device current, and passes
 // the pointer to the kernels.
 #include <cuda_runtime.h>
+#include <stdint.h>
 
 #include <mutex>
 
@@ -56,6 +57,8 @@ extern "C" kda_status_t kda_context_parallel_prefill_static(
     const float* initial_state, void* out, kda_dtype_t out_dtype, float* final_state, float* M, float* U,
     float* incoming, float* outgoing, uint32_t flags, float gate_lower_bound, int32_t* device_status,
     void* stream) {
+  // token offsets are int32; checked before the size, whose product would be meaningless beyond
+  if (T < 0 || T > INT32_MAX || num_v_heads <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
   const size_t need = kda_context_parallel_workspace_size(T, num_v_heads, dv);
   if (need > kStaticScratchBytes) return KDA_ERR_WORKSPACE;  // beyond the fixed scratch: refuse
   void* scratch = nullptr;

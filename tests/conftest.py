@@ -6,10 +6,21 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+HERE = os.path.dirname(os.path.abspath(__file__))
+if HERE not in sys.path:
+    sys.path.insert(0, HERE)
 
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_terminal_summary(terminalreporter):
+    # the measured parity errors (whole tensor and worst (sequence, head) chain per label)
+    import parity
+    if parity.RECORDS:
+        for line in parity.summary_lines():
+            terminalreporter.write_line(line)
 
 
 @pytest.fixture(scope="session")

@@ -201,3 +201,24 @@ def test_host_pipelined_prefill_host_checks(lib):
     assert need >= 4096 * 2 * 128 * (2 + 2) + 4096 * 2 * 128 * (2 + 4 + 2)
     assert call(ws=256 + 8, ws_bytes=need) == 3  # workspace not 256-byte aligned
     assert kda.kda_prefill_host_workspace_size(4096, 2, 2, segment_tokens=100) == 0
+
+
+def test_token_counts_beyond_int32_are_refused(lib):
+    # token offsets are int32 (as cu_seqlens): larger counts are refused before any size arithmetic
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
+    big = (1 << 31)
+    assert _chunk(lib, T=big) == 1
+    assert _seg(lib, T=big) == 1
+    args = [p(16)] * 3 + [1] + [p(16)] * 4 + [big, 2, 2, 128, 128, p(16), 2, p(16), p(16), 1] + [p(16)] * 5 + \
+        [0, -5.0]
+    assert lib.kda_context_parallel_prefill(*args, p(256), 1 << 40, None, None) == 1
+    fn = lib.kda_context_parallel_prefill_static
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    fn.restype = ctypes.c_int
+    fn.argtypes = [vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, i64, i32, i32, i32, i32, vp, i32, vp, vp, ctypes.c_int,
+                   vp, vp, vp, vp, vp, ctypes.c_uint32, ctypes.c_float, vp, vp]
+    assert fn(*args, None, None) == 1
+    assert lib.kda_context_parallel_apply(p(16), p(16), p(16), p(16), 2, big, 2, 128, p(16), 1, 0, None, None) == 1
+    # the sizes say that no workspace can serve such a call
+    assert kda.kda_context_parallel_workspace_size(big, 32, 128) == 2 ** 64 - 1
+    assert kda.kda_context_parallel_workspace_preferred(big, 16, 32, 128) == 2 ** 64 - 1

@@ -17,6 +17,7 @@ import torch.distributed as dist
 import kda_workloads as W
 import kimi_delta_attention_23_b200 as kda
 import oracle
+import parity
 from kimi_delta_attention_23_b200 import distributed as D
 
 pytestmark = pytest.mark.gpu
@@ -86,13 +87,13 @@ def test_emulated_ranks_match_the_straight_recurrence(cuda_device, world, T, lay
     ranges, sums, scan, fins = emulate(w, world, layout)
     out = torch.cat([f["out"] for f in fins])
     o_ref, p_ref = straight(w, layout)
-    assert rel_l2(out, o_ref) < TOL
-    assert rel_l2(scan["final_state"], p_ref[0]) < TOL
+    parity.check_rows("emulated ranks: out", out, o_ref, TOL)
+    parity.check_states("emulated ranks: final", scan["final_state"], p_ref[0], TOL)
     for i, ((s, e), f) in enumerate(zip(ranges, fins)):
         assert rel_l2(f["range_outgoing"], scan["outgoing_states"][i]) < 1e-4  # the range's end, two ways
         if s > 0:
             _, p_s = straight(w, layout, upto=s)
-            assert rel_l2(scan["incoming_states"][i], p_s[0]) < TOL
+            parity.check_states("emulated ranks: incoming of a rank", scan["incoming_states"][i], p_s[0], TOL)
 
 
 def test_range_segments_match_oracle_summaries(cuda_device):
@@ -105,17 +106,17 @@ def test_range_segments_match_oracle_summaries(cuda_device):
         M, U = oracle.kda_segment_summary(cpu(w.k)[s:e], cpu(w.v)[s:e], cpu(w.raw_gate)[s:e],
                                           cpu(w.beta_logits)[s:e], cpu(w.a_log), cpu(w.dt_bias), cpu(offs))
         sc = oracle.kda_affine_scan(M, U, cpu(scan["incoming_states"][i]).double().numpy())
-        assert rel_l2(f["transition_matrices"], M) < TOL
-        assert rel_l2(f["local_contributions"], U) < TOL
-        assert rel_l2(f["incoming_states"], sc["incoming_states"]) < TOL
-        assert rel_l2(f["outgoing_states"], sc["outgoing_states"]) < TOL
+        parity.check_maps("rank segments: M", f["transition_matrices"], M, TOL)
+        parity.check_states("rank segments: U", f["local_contributions"], U, TOL)
+        parity.check_states("rank segments: incoming", f["incoming_states"], sc["incoming_states"], TOL)
+        parity.check_states("rank segments: outgoing", f["outgoing_states"], sc["outgoing_states"], TOL)
         # the whole range's map is its segments' composed in order; over a thousand tokens the
         # transition has decayed to (fp32) zero, so it is checked in absolute terms
         Mr, Ur = oracle.kda_segment_summary(cpu(w.k)[s:e], cpu(w.v)[s:e], cpu(w.raw_gate)[s:e],
                                             cpu(w.beta_logits)[s:e], cpu(w.a_log), cpu(w.dt_bias),
                                             np.array([0, e - s], np.int32))
         assert np.abs(cpu(sums[i][0]["range_transition"]).double().numpy() - Mr[0]).max() < 1e-6
-        assert rel_l2(sums[i][0]["range_contribution"], Ur[0]) < TOL
+        parity.check_states("rank map: U", sums[i][0]["range_contribution"], Ur[0], TOL)
 
 
 def test_safe_gate_fp32_output(cuda_device):
@@ -125,8 +126,8 @@ def test_safe_gate_fp32_output(cuda_device):
     out = torch.cat([f["out"] for f in fins])
     assert out.dtype == torch.float32
     o_ref, p_ref = straight(w, "K_FIRST", gate_mode="safe")
-    assert rel_l2(out, o_ref) < TOL
-    assert rel_l2(scan["final_state"], p_ref[0]) < TOL
+    parity.check_rows("emulated ranks, safe gate: out", out, o_ref, TOL)
+    parity.check_states("emulated ranks, safe gate: final", scan["final_state"], p_ref[0], TOL)
 
 
 def test_one_rank_equals_the_single_gpu_prefill(cuda_device):
@@ -150,8 +151,8 @@ def test_full_size_eight_ranks_sampled_heads(cuda_device):
     out = torch.cat([f["out"] for f in fins])
     heads = [0, 31]
     o_ref, p_ref = straight(w, "K_FIRST", heads=heads)
-    assert rel_l2(out[:, heads], o_ref) < TOL
-    assert rel_l2(scan["final_state"][heads], p_ref[0]) < TOL
+    parity.check_rows("long_T131072_H32 over 8 ranks: out", out[:, heads], o_ref, TOL)
+    parity.check_states("long_T131072_H32 over 8 ranks: final", scan["final_state"][heads], p_ref[0], TOL)
 
 
 def _free_port():
@@ -171,6 +172,6 @@ def test_distributed_entry_in_a_one_rank_nccl_group(cuda_device):
     finally:
         dist.destroy_process_group()
     o_ref, p_ref = straight(w, "K_FIRST")
-    assert rel_l2(res["out"], o_ref) < TOL
-    assert rel_l2(res["final_state"], p_ref[0]) < TOL
+    parity.check_rows("one-rank NCCL group: out", res["out"], o_ref, TOL)
+    parity.check_states("one-rank NCCL group: final", res["final_state"], p_ref[0], TOL)
     assert rel_l2(res["range_incoming"], w.state_pool[0]) == 0.0

@@ -3,13 +3,13 @@ pipelined with the kernels in segments.  Segment boundaries fall on chunk bounda
 outputs and the final state must equal the plain chunk kernel's on the whole sequence bit for
 bit (kda_chunk_fwd without a workspace); one
 case is also checked against the fp64 oracle (relative L2 1e-2, bf16 q/k/v)."""
-import numpy as np
 import pytest
 import torch
 
 import kda_workloads as W
 import kimi_delta_attention_23_b200 as kda
 import oracle
+import parity
 
 pytestmark = pytest.mark.gpu
 
@@ -60,9 +60,8 @@ def test_matches_oracle(cuda_device):
     _, _, res = run_both(w, 512)
     o_ref, p_ref = oracle.kda_forward(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens,
                                       w.state_pool, w.state_indices)
-    rel = lambda x, r: float(np.linalg.norm(x.double().numpy() - r) / np.linalg.norm(r))  # noqa: E731
-    assert rel(res["out"], o_ref) < 1e-2
-    assert rel(res["final_state"], p_ref[0]) < 1e-2
+    parity.check_rows("host-pipelined prefill: out", res["out"], o_ref, 1e-2)
+    parity.check_states("host-pipelined prefill: final", res["final_state"], p_ref[0], 1e-2)
 
 
 def test_empty_sequence_passes_the_state_through(cuda_device):

@@ -14,6 +14,7 @@ import torch
 import kda_workloads as W
 import kimi_delta_attention_23_b200 as kda
 import oracle
+import parity
 
 pytestmark = pytest.mark.gpu
 
@@ -55,7 +56,7 @@ def test_scan_only_matches_oracle_scan():
     cu = lambda x: torch.tensor(x, dtype=torch.float32, device="cuda")  # noqa: E731
     res = kda.kda_context_parallel(cu(M), cu(U), cu(S0))
     for key in ref:
-        assert rel_l2(res[key], ref[key]) < 1e-5, key
+        parity.check_states(f"scan only: {key}", res[key], ref[key], 1e-5)
 
 
 CASES = [
@@ -82,11 +83,12 @@ def test_segment_summaries_and_scan(dtype, d, layout, tol):
     M, U = oracle.kda_segment_summary(w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, offs,
                                       state_layout=layout)
     ref = oracle.kda_affine_scan(M, U, w.state_pool[0], state_layout=layout)
-    assert rel_l2(res["transition_matrices"], M) < tol
-    assert rel_l2(res["local_contributions"], U) < tol
-    assert rel_l2(res["incoming_states"], ref["incoming_states"]) < tol
-    assert rel_l2(res["outgoing_states"], ref["outgoing_states"]) < tol
-    assert rel_l2(res["final_state"], ref["final_state"]) < tol
+    lab = f"segment summaries {'fp32' if dtype == torch.float32 else 'bf16'}"
+    parity.check_maps(f"{lab}: M", res["transition_matrices"], M, tol)
+    parity.check_states(f"{lab}: U", res["local_contributions"], U, tol)
+    parity.check_states(f"{lab}: incoming", res["incoming_states"], ref["incoming_states"], tol)
+    parity.check_states(f"{lab}: outgoing", res["outgoing_states"], ref["outgoing_states"], tol)
+    parity.check_states(f"{lab}: final", res["final_state"], ref["final_state"], tol)
 
 
 def _cp_prefill(wd, offs, init, layout="K_FIRST", gate_mode="original", lb=-5.0):
@@ -109,11 +111,11 @@ def test_context_parallel_prefill_matches_straight_recurrence(layout):
     out, pool, res = _cp_prefill(wd, offs, wd.state_pool[0].contiguous(), layout)
     o_ref, p_ref = oracle.kda_forward(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens,
                                       w.state_pool, w.state_indices, state_layout=layout)
-    assert rel_l2(out, o_ref) < 1e-2
-    assert rel_l2(res["final_state"], p_ref[0]) < 1e-2
-    assert rel_l2(pool[-1], p_ref[0]) < 1e-2
+    parity.check_rows("two-pass context parallel: out", out, o_ref, 1e-2)
+    parity.check_states("two-pass context parallel: final", res["final_state"], p_ref[0], 1e-2)
+    parity.check_states("two-pass context parallel: final", pool[-1], p_ref[0], 1e-2)
     # the second pass ends every segment in the scan's outgoing state
-    assert rel_l2(pool, res["outgoing_states"].double().cpu().numpy()) < 1e-2
+    parity.check_states("two-pass: pass 2 vs scan outgoing", pool, res["outgoing_states"], 1e-2)
 
 
 def test_full_size_context_parallel_sampled_heads():
@@ -126,8 +128,8 @@ def test_full_size_context_parallel_sampled_heads():
                                       cpu(w.raw_gate)[:, heads], cpu(w.beta_logits)[:, heads], cpu(w.a_log)[heads],
                                       cpu(w.dt_bias)[heads], cpu(w.cu_seqlens), cpu(w.state_pool)[:, heads],
                                       cpu(w.state_indices))
-    assert rel_l2(out[:, heads], o_ref) < 1e-2
-    assert rel_l2(res["final_state"][heads], p_ref[0]) < 1e-2
+    parity.check_rows("long_T131072_H32_cp16 two-pass: out", out[:, heads], o_ref, 1e-2)
+    parity.check_states("long_T131072_H32_cp16 two-pass: final", res["final_state"][heads], p_ref[0], 1e-2)
 
 
 @pytest.mark.parametrize("layout,out_dtype", [("K_FIRST", torch.bfloat16), ("V_FIRST", torch.float32)])
@@ -144,16 +146,19 @@ def test_context_parallel_prefill_entry_point(layout, out_dtype):
     o_ref, p_ref = oracle.kda_forward(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens,
                                       w.state_pool, w.state_indices, state_layout=layout)
     assert res["out"].dtype == out_dtype
-    assert rel_l2(res["out"], o_ref) < 1e-2
-    assert rel_l2(res["final_state"], p_ref[0]) < 1e-2
+    parity.check_rows("context-parallel prefill: out", res["out"], o_ref, 1e-2)
+    parity.check_states("context-parallel prefill: final", res["final_state"], p_ref[0], 1e-2)
     M, U = oracle.kda_segment_summary(w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, offs.cpu(),
                                       state_layout=layout)
-    assert rel_l2(res["transition_matrices"], M) < 1e-2
-    assert rel_l2(res["local_contributions"], U) < 1e-2
+    parity.check_maps("context-parallel prefill: M", res["transition_matrices"], M, 1e-2)
+    parity.check_states("context-parallel prefill: U", res["local_contributions"], U, 1e-2)
 
 
 def test_full_size_context_parallel_prefill_sampled_heads():
-    """The benchmark's step: 131072 tokens, 32 heads, 16 segments, one entry point."""
+    """The benchmark's step: 131072 tokens, 32 heads, 16 segments, one entry point.  Besides the
+    outputs and the final state, every segment's M_i, U_i and its incoming and outgoing states
+    are compared with the oracle's own summaries (each segment replayed from I and from 0) and
+    its scan -- on the sampled heads, at full length."""
     w = W.make("long_T131072_H32_cp16", device="cuda")
     res = kda.kda_context_parallel_prefill(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias,
                                            w.seg_offsets, w.state_pool[0])
@@ -164,8 +169,17 @@ def test_full_size_context_parallel_prefill_sampled_heads():
                                       cpu(w.raw_gate)[:, heads], cpu(w.beta_logits)[:, heads], cpu(w.a_log)[heads],
                                       cpu(w.dt_bias)[heads], cpu(w.cu_seqlens), cpu(w.state_pool)[:, heads],
                                       cpu(w.state_indices))
-    assert rel_l2(res["out"][:, heads], o_ref) < 1e-2
-    assert rel_l2(res["final_state"][heads], p_ref[0]) < 1e-2
+    lab = "long_T131072_H32_cp16"
+    parity.check_rows(f"{lab}: out", res["out"][:, heads], o_ref, 1e-2)
+    parity.check_states(f"{lab}: final", res["final_state"][heads], p_ref[0], 1e-2)
+    M, U = oracle.kda_segment_summary(cpu(w.k)[:, heads], cpu(w.v)[:, heads], cpu(w.raw_gate)[:, heads],
+                                      cpu(w.beta_logits)[:, heads], cpu(w.a_log)[heads], cpu(w.dt_bias)[heads],
+                                      cpu(w.seg_offsets))
+    scan = oracle.kda_affine_scan(M, U, cpu(w.state_pool)[0, heads])
+    parity.check_maps(f"{lab}: M", res["transition_matrices"][:, heads], M, 1e-2)
+    parity.check_states(f"{lab}: U", res["local_contributions"][:, heads], U, 1e-2)
+    parity.check_states(f"{lab}: incoming", res["incoming_states"][:, heads], scan["incoming_states"], 1e-2)
+    parity.check_states(f"{lab}: outgoing", res["outgoing_states"][:, heads], scan["outgoing_states"], 1e-2)
 
 
 # ------------------------------------------------------------------------------------------
@@ -242,13 +256,14 @@ def test_split_prefill_matches_oracle_and_unsplit(layout):
     M, U = oracle.kda_segment_summary(w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, offs.cpu(),
                                       state_layout=layout)
     scan = oracle.kda_affine_scan(M, U, w.state_pool[0].double().numpy(), state_layout=layout)
-    for res in (split, whole):
-        assert rel_l2(res["out"], o_ref) < 1e-2
-        assert rel_l2(res["final_state"], p_ref[0]) < 1e-2
-        assert rel_l2(res["transition_matrices"], M) < 1e-2
-        assert rel_l2(res["local_contributions"], U) < 1e-2
-        assert rel_l2(res["incoming_states"], scan["incoming_states"]) < 1e-2
-        assert rel_l2(res["outgoing_states"], scan["outgoing_states"]) < 1e-2
+    for name, res in (("pieces", split), ("whole segments", whole)):
+        lab = f"context parallel ({name})"
+        parity.check_rows(f"{lab}: out", res["out"], o_ref, 1e-2)
+        parity.check_states(f"{lab}: final", res["final_state"], p_ref[0], 1e-2)
+        parity.check_maps(f"{lab}: M", res["transition_matrices"], M, 1e-2)
+        parity.check_states(f"{lab}: U", res["local_contributions"], U, 1e-2)
+        parity.check_states(f"{lab}: incoming", res["incoming_states"], scan["incoming_states"], 1e-2)
+        parity.check_states(f"{lab}: outgoing", res["outgoing_states"], scan["outgoing_states"], 1e-2)
     assert rel_l2(split["out"], whole["out"].double().cpu().numpy()) < 1e-2
 
 
@@ -276,4 +291,4 @@ def test_head_major_readouts_equal_token_major(out_dtype):
     assert torch.equal(oh, ot)
     o_ref, _ = oracle.kda_forward(w.q, w.k, w.v, w.raw_gate, w.beta_logits, w.a_log, w.dt_bias, w.cu_seqlens,
                                   w.state_pool, w.state_indices)
-    assert rel_l2(oh, o_ref) < 1e-2
+    parity.check_rows("head-major readouts: out", oh, o_ref, 1e-2)
