@@ -47,6 +47,48 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity
   }
 }
 
+// try_wait with a suspend-time hint: until the phase completes (or the hint's time passes) the
+// thread may be suspended instead of polling, so a waiting warp takes no issue slots from the
+// warps that work beside it
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity), "r"(10000000u)
+      : "memory");
+  return ok != 0;
+}
+// as mbar_wait_bounded, sleeping between the tests
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t addr, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait_sleep(addr, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_sleep(addr, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// as mbar_wait_bounded, with a short pause between the tests (a polling warp then takes few issue
+// slots from the warps that work beside it, and the pause adds at most that much latency)
+__device__ __forceinline__ bool mbar_wait_backoff(uint32_t addr, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(addr, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(32);
+    if (mbar_try_wait(addr, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// arrive once (release: the arriving thread's earlier writes are visible to a waiter that saw
+// the phase complete)
+__device__ __forceinline__ void mbar_arrive(uint32_t addr) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
 // expect `bytes` of asynchronous transactions on the barrier and arrive once
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t addr, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(bytes) : "memory");
@@ -257,6 +299,22 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[3
       "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
       "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
+}
+// 16 consecutive 32-bit columns of this thread's lane in one store
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+// 32 consecutive fp32 columns of this thread's lane in one store
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  uint32_t u[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(v[i]);
+  tmem_st32u(taddr, u);
 }
 // 64 consecutive 32-bit columns of this thread's lane in one store
 __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) {
