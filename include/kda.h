@@ -97,8 +97,11 @@ enum {
   KDA_FUSED = 1u << 3,         /* use_computebound: accepted; the bf16 path is always the fused kernel */
   KDA_SEG_SCAN_ONLY = 1u << 4, /* segment call: M and U are inputs, only the scan runs           */
   KDA_FORCE_SIMT = 1u << 5,    /* run the fp32 CUDA-core chunk kernel even for bf16 inputs       */
-  KDA_READOUT_HEAD_MAJOR = 1u << 6 /* readout_m / readout_u stored [Hv, T, 128] instead of
-                                      [T, Hv, 128] (calls that write or read readouts only)      */
+  KDA_READOUT_HEAD_MAJOR = 1u << 6, /* readout_m / readout_u stored [Hv, T, 128] instead of
+                                       [T, Hv, 128] (calls that write or read readouts only)     */
+  KDA_SCAN_LOGDEPTH = 1u << 7  /* segment call: the scan in log depth (needs the workspace of
+                                  kda_scan_workspace_size); without it the log-depth form is
+                                  chosen when that workspace is given and it is expected faster */
 };
 
 /*
@@ -198,6 +201,15 @@ KDA_API kda_status_t kda_decode(const void *q, const void *k, const void *v, kda
  *   transition readout_m[t] = q_t^T M_{<=t} and of the contribution readout_u[t] = q_t^T U_{<=t}
  *   ([T, Hv, 128] bf16 each; [Hv, T, 128] with KDA_READOUT_HEAD_MAJOR, which makes every
  *   head's rows contiguous for the apply), the inputs of kda_context_parallel_apply.
+ *
+ *   workspace (device, 256-byte aligned, nullable): with dk = 128 and dv a multiple of 32, at
+ *   least kda_scan_workspace_size(num_segments, num_v_heads, dk, dv) bytes let the scan run in
+ *   log depth ("KDA Context Parallelism", Compose segments in sequence order: the composition is
+ *   associative): ceil(log2 N) levels of P_i <- P_i o P_{i - 2^l}, then every prefix applied to
+ *   initial_state.  It is used with KDA_SCAN_LOGDEPTH (else KDA_ERR_WORKSPACE without the
+ *   workspace, KDA_ERR_UNSUPPORTED for other dk, dv or more than 65535 segments), or without
+ *   that flag where kda_scan_logdepth_preferred says it should finish first (few heads, many
+ *   segments).  Results equal the sequential scan's up to rounding (both fp32-accurate).
  */
 KDA_API kda_status_t kda_segment_summarize_and_scan(
     const void *k, const void *v, kda_dtype_t kv_dtype, const float *raw_gate,
@@ -207,6 +219,14 @@ KDA_API kda_status_t kda_segment_summarize_and_scan(
     float *outgoing, float *final_state, const void *q, void *readout_m, void *readout_u,
     uint32_t flags, float gate_lower_bound, void *workspace, size_t workspace_bytes,
     int32_t *device_status, void *stream);
+
+/* Workspace bytes of the log-depth scan: two sets of every segment's prefix map,
+ * 2 * N * H * (128 * 128 + 128 * dv) * 4 (0 where it does not apply: dk != 128, dv not a
+ * multiple of 32 up to 128, N < 1).  No counterpart on the pages beyond the associativity. */
+KDA_API size_t kda_scan_workspace_size(int32_t num_segments, int32_t num_v_heads, int32_t dk, int32_t dv);
+/* 1 if the log-depth scan is expected to finish before the sequential one on the current
+ * device (both counted in rounds of tile products over its SMs), else 0. */
+KDA_API int32_t kda_scan_logdepth_preferred(int32_t num_segments, int32_t num_v_heads, int32_t dv);
 
 /*
  * kda_context_parallel_apply -- outputs of every segment from its local readouts and its

@@ -44,6 +44,7 @@ FUSED = 1 << 3
 SEG_SCAN_ONLY = 1 << 4
 FORCE_SIMT = 1 << 5
 READOUT_HEAD_MAJOR = 1 << 6
+SCAN_LOGDEPTH = 1 << 7
 
 _F32, _BF16 = 0, 1
 _DTYPES = {torch.float32: _F32, torch.bfloat16: _BF16}
@@ -108,6 +109,10 @@ def load_library():
                                                vp, ctypes.c_int, fp, i64, u32, f32, vp, sz, ip, vp]
     lib.kda_workspace_size.restype = sz
     lib.kda_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32, i32, u32]
+    lib.kda_scan_workspace_size.restype = sz
+    lib.kda_scan_workspace_size.argtypes = [i32, i32, i32, i32]
+    lib.kda_scan_logdepth_preferred.restype = i32
+    lib.kda_scan_logdepth_preferred.argtypes = [i32, i32, i32]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_status_string.argtypes = [ctypes.c_int]
     lib.kda_version.restype = i32
@@ -335,7 +340,8 @@ def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, 
                                    *, M=None, U=None, incoming=None, outgoing=None, final_state=None,
                                    q=None, readout_m=None, readout_u=None, readout_layout="token_major",
                                    scan_only=False, gate_mode="original", beta_mode="logits", state_layout="K_FIRST",
-                                   gate_lower_bound=-5.0, device_status=None, stream=None):
+                                   gate_lower_bound=-5.0, workspace=None, scan_logdepth=False, device_status=None,
+                                   stream=None):
     """Segment summaries (M_i, U_i) of one sequence and the exclusive scan over them.
 
     Returns dict(incoming_states, outgoing_states, final_state, transition_matrices,
@@ -344,6 +350,8 @@ def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, 
     heads) the build also returns each token's readouts through the transition and of the
     contribution, the inputs of ``kda_context_parallel_apply``: [T, Hv, 128] each, or [Hv, T, 128]
     with ``readout_layout="head_major"`` (every head's rows contiguous; the apply reads them faster).
+    ``workspace`` (uint8 CUDA tensor of kda_scan_workspace_size bytes) lets the scan run in log
+    depth where that is expected to finish first; ``scan_logdepth`` forces the log-depth form.
     """
     lib = load_library()
     dev = initial_state.device
@@ -397,13 +405,18 @@ def kda_segment_summarize_and_scan(k, v, raw_gate, beta_logits, a_log, dt_bias, 
     flags = _flags(gate_mode, beta_mode, state_layout, scan_only=scan_only)
     if q is not None:
         flags |= _readout_flags(readout_layout)
+    if scan_logdepth:
+        flags |= SCAN_LOGDEPTH
+    if workspace is not None:
+        _dev(workspace, "workspace", torch.uint8, dev)
     rc = lib.kda_segment_summarize_and_scan(
         _ptr(k) if not scan_only else None, _ptr(v) if not scan_only else None, kv_dtype,
         _ptr(raw_gate) if not scan_only else None, _ptr(beta_logits) if not scan_only else None,
         _ptr(a_log) if not scan_only else None, _ptr(dt_bias) if not scan_only else None, T, Hk, Hv, dk, dv,
         _ptr(seg_offsets) if not scan_only else None, N, _ptr(initial_state), _ptr(M), _ptr(U),
         _ptr(incoming), _ptr(outgoing), _ptr(final_state), _ptr(q), _ptr(readout_m), _ptr(readout_u), flags,
-        float(gate_lower_bound), None, 0, _ptr(device_status), _stream(stream, dev))
+        float(gate_lower_bound), _ptr(workspace) if workspace is not None and workspace.numel() else None,
+        workspace.numel() if workspace is not None else 0, _ptr(device_status), _stream(stream, dev))
     own.launched()
     if rc != 0:
         raise KdaError(rc, "kda_segment_summarize_and_scan")
@@ -445,12 +458,14 @@ def kda_context_parallel_apply(readout_m, readout_u, incoming, seg_offsets, out=
 
 
 def kda_context_parallel(transition_matrices, local_contributions, initial_state, *, state_layout="K_FIRST",
-                         stream=None):
+                         method="auto", stream=None):
     """The exclusive affine scan alone ("KDA Context Parallelism", Requirements).
 
     transition_matrices (N, dk, dk), local_contributions (N, dk, dv), initial_state (dk, dv),
     fp32 CUDA tensors (a leading head axis after N is also accepted).  Returns a dict with
     exactly incoming_states, outgoing_states and final_state; no input is written.
+    ``method``: "sequential" (one step per segment), "logdepth" (the composition in log depth,
+    dk = 128 only) or "auto" (log depth where the library expects it to finish first).
     """
     M, U, S0 = transition_matrices, local_contributions, initial_state
     if M.dtype != torch.float32:
@@ -462,17 +477,42 @@ def kda_context_parallel(transition_matrices, local_contributions, initial_state
         M, U, S0 = M.unsqueeze(1), U.unsqueeze(1), S0.unsqueeze(0)
     if M.shape[0] < 1:
         raise ValueError("at least one segment is required")
+    if method not in ("auto", "sequential", "logdepth"):
+        raise ValueError(f"unknown scan method {method!r}")
     own = _Owned(stream, S0.device)
     Mc, Uc, Sc = own.keep(M.contiguous(), M), own.keep(U.contiguous(), U), own.keep(S0.contiguous(), S0)
+    N, H, dk = M.shape[0], M.shape[1], M.shape[-1]
+    dv = U.shape[-1] if state_layout == "K_FIRST" else U.shape[-2]
+    ws = None
+    if method == "logdepth" or (method == "auto" and kda_scan_logdepth_preferred(N, H, dv, device=S0.device)):
+        need = kda_scan_workspace_size(N, H, dk, dv)
+        if need == 0 and method == "logdepth":
+            raise ValueError("the log-depth scan needs dk = 128 and dv a multiple of 32 up to 128")
+        ws = own.empty(need, dtype=torch.uint8, device=S0.device) if need else None
     res = kda_segment_summarize_and_scan(None, None, None, None, None, None,
                                          torch.zeros(M.shape[0] + 1, dtype=torch.int32), Sc,
-                                         M=Mc, U=Uc, scan_only=True, state_layout=state_layout, stream=stream)
+                                         M=Mc, U=Uc, scan_only=True, state_layout=state_layout, workspace=ws,
+                                         scan_logdepth=method == "logdepth", stream=stream)
     own.launched()
     out = {k: res[k] for k in ("incoming_states", "outgoing_states", "final_state")}
     if squeeze:
         out = {"incoming_states": out["incoming_states"][:, 0], "outgoing_states": out["outgoing_states"][:, 0],
                "final_state": out["final_state"][0]}
     return out
+
+
+def kda_scan_workspace_size(num_segments, num_v_heads, dk=128, dv=128) -> int:
+    """Workspace bytes of the log-depth scan (0 where it does not apply)."""
+    return int(load_library().kda_scan_workspace_size(num_segments, num_v_heads, dk, dv))
+
+
+def kda_scan_logdepth_preferred(num_segments, num_v_heads, dv=128, device=None) -> bool:
+    """Whether the log-depth scan is expected to finish first on ``device`` (default: current)."""
+    lib = load_library()
+    if device is not None and torch.device(device).type == "cuda":
+        with torch.cuda.device(device):
+            return bool(lib.kda_scan_logdepth_preferred(num_segments, num_v_heads, dv))
+    return bool(lib.kda_scan_logdepth_preferred(num_segments, num_v_heads, dv))
 
 
 def kda_context_parallel_workspace_size(T, num_v_heads, dv=128) -> int:

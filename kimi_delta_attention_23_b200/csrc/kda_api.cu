@@ -17,7 +17,7 @@ bool fused_available();
 namespace {
 
 constexpr uint32_t kKnownFlags = KDA_GATE_SAFE | KDA_BETA_PROB | KDA_STATE_V_FIRST | KDA_FUSED |
-                                 KDA_SEG_SCAN_ONLY | KDA_FORCE_SIMT | KDA_READOUT_HEAD_MAJOR;
+                                 KDA_SEG_SCAN_ONLY | KDA_FORCE_SIMT | KDA_READOUT_HEAD_MAJOR | KDA_SCAN_LOGDEPTH;
 
 bool dtype_ok(kda_dtype_t t) { return t == KDA_F32 || t == KDA_BF16; }
 
@@ -331,8 +331,6 @@ extern "C" kda_status_t kda_segment_summarize_and_scan(
     float* M, float* U, float* incoming, float* outgoing, float* final_state, const void* q, void* readout_m,
     void* readout_u, uint32_t flags, float gate_lower_bound, void* workspace, size_t workspace_bytes,
     int32_t* device_status, void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   if (num_segments < 1 || num_v_heads <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
   const bool readouts = q || readout_m || readout_u;
   if (readouts && (!q || !readout_m || !readout_u)) return KDA_ERR_INVALID_ARG;
@@ -340,6 +338,17 @@ extern "C" kda_status_t kda_segment_summarize_and_scan(
   if ((flags & ~kKnownFlags) != 0) return KDA_ERR_INVALID_ARG;
   if (!initial_state || !M || !U || !incoming || !outgoing || !final_state) return KDA_ERR_INVALID_ARG;
   if (dk > 128 || dv > 128) return KDA_ERR_UNSUPPORTED;
+  // the scan's form: log depth when forced (and possible) or when given its workspace and expected
+  // to finish first; the checks come before any launch
+  const size_t log_need = kda::logdepth_scan_bytes(num_segments, num_v_heads, dk, dv);
+  const bool log_possible = log_need > 0 && num_segments <= 65535;
+  const bool log_ws = workspace && workspace_bytes >= log_need && !(reinterpret_cast<uintptr_t>(workspace) & 255u);
+  if (flags & KDA_SCAN_LOGDEPTH) {
+    if (!log_possible) return KDA_ERR_UNSUPPORTED;
+    if (!log_ws) return KDA_ERR_WORKSPACE;
+  }
+  const bool use_log = log_possible && log_ws &&
+                       ((flags & KDA_SCAN_LOGDEPTH) || kda::logdepth_scan_preferred(num_segments, num_v_heads, dv));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int v_first = (flags & KDA_STATE_V_FIRST) ? 1 : 0;
   if (!(flags & KDA_SEG_SCAN_ONLY)) {
@@ -438,7 +447,19 @@ extern "C" kda_status_t kda_segment_summarize_and_scan(
   sa.incoming = incoming;
   sa.outgoing = outgoing;
   sa.final_state = final_state;
+  if (use_log)
+    return kda::launch_affine_scan_logdepth(sa, reinterpret_cast<float*>(workspace), s) == cudaSuccess ? KDA_OK
+                                                                                                      : KDA_ERR_CUDA;
   return kda::launch_affine_scan(sa, s) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" size_t kda_scan_workspace_size(int32_t num_segments, int32_t num_v_heads, int32_t dk, int32_t dv) {
+  return kda::logdepth_scan_bytes(num_segments, num_v_heads, dk, dv);
+}
+
+extern "C" int32_t kda_scan_logdepth_preferred(int32_t num_segments, int32_t num_v_heads, int32_t dv) {
+  if (num_segments < 1 || num_segments > 65535 || num_v_heads < 1 || dv < 32 || dv > 128 || dv % 32) return 0;
+  return kda::logdepth_scan_preferred(num_segments, num_v_heads, dv) ? 1 : 0;
 }
 
 extern "C" size_t kda_context_parallel_workspace_size(int64_t T, int32_t num_v_heads, int32_t dv) {

@@ -47,6 +47,15 @@ struct ScanArgs {
   float* final_state;
 };
 
+// One level of the log-depth scan over the maps' prefixes.
+struct ScanLevelArgs {
+  const float* M;   // [N][H][128][128] the level's input prefixes (row-major)
+  const float* U;   // [N][H][state]
+  float* M_out;     // the level's output prefixes
+  float* U_out;
+  int32_t N, H, dv, v_first, stride;
+};
+
 // Fused tensor-core chunk kernel (bf16 q/k/v, dk = dv = 128).
 struct FusedArgs {
   const void* q;            // bf16 [T,Hk,128]
@@ -177,6 +186,11 @@ cudaError_t launch_pool_scan(const PoolScanArgs& a, cudaStream_t stream);
 cudaError_t launch_cp_apply(const ApplyArgs& a, cudaStream_t stream);
 cudaError_t launch_simt_chunk(const SimtArgs& a, cudaStream_t stream);
 cudaError_t launch_affine_scan(const ScanArgs& a, cudaStream_t stream);
+// the log-depth form (dk = 128, dv a multiple of 32 up to 128); `work` holds
+// logdepth_scan_bytes(N, H, dk, dv) bytes
+size_t logdepth_scan_bytes(int N, int H, int dk, int dv);
+bool logdepth_scan_preferred(int N, int H, int dv);
+cudaError_t launch_affine_scan_logdepth(const ScanArgs& a, float* work, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace kda

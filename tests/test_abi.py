@@ -222,3 +222,14 @@ def test_token_counts_beyond_int32_are_refused(lib):
     # the sizes say that no workspace can serve such a call
     assert kda.kda_context_parallel_workspace_size(big, 32, 128) == 2 ** 64 - 1
     assert kda.kda_context_parallel_workspace_preferred(big, 16, 32, 128) == 2 ** 64 - 1
+
+
+def test_logdepth_scan_sizes_and_host_checks(lib):
+    # two sets of every segment's prefix map: 2 * N * H * (128 * 128 + 128 * dv) floats
+    assert kda.kda_scan_workspace_size(17, 3, 128, 64) == 2 * 17 * 3 * (128 * 128 + 128 * 64) * 4
+    assert kda.kda_scan_workspace_size(17, 3, 64, 64) == 0    # dk must be 128
+    assert kda.kda_scan_workspace_size(17, 3, 128, 48) == 0   # dv a multiple of 32
+    assert lib.kda_scan_logdepth_preferred(1, 4, 128) == 0    # one segment: nothing to compose
+    # forced without a workspace, or where it cannot run: refused before any launch
+    assert _seg(lib, flags=kda.SEG_SCAN_ONLY | kda.SCAN_LOGDEPTH) == 3            # KDA_ERR_WORKSPACE
+    assert _seg(lib, flags=kda.SEG_SCAN_ONLY | kda.SCAN_LOGDEPTH, dk=64) == 2     # KDA_ERR_UNSUPPORTED
