@@ -21,7 +21,7 @@
 // Two warp teams share the CTA (512 threads) and work one chunk apart:
 //   * the key team (warps 0-7) does everything that does not touch the state.  It reads a
 //     chunk's raw gates, keys and queries from global memory straight into registers (an L2
-//     prefetch runs two chunks ahead), forms the decays, the 8x8 diagonal score blocks on CUDA
+//     prefetch runs one or two chunks ahead), forms the decays, the 8x8 diagonal score blocks on CUDA
 //     cores (a product recursion along the rows), the operand tiles, the off-diagonal scores
 //     with mma.sync on operands scaled by a reference point that sits between rows and columns
 //     (both factors <= 1), and the inverses of the 8x8 diagonal blocks;
@@ -360,7 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     const __nv_bfloat16* k_base = reinterpret_cast<const __nv_bfloat16*>(a.k) + (size_t)kh * D + ch;
     const __nv_bfloat16* q_base = reinterpret_cast<const __nv_bfloat16*>(qb ? a.q : a.k) + (size_t)kh * D + ch;
     // a chunk's raw gates, keys and queries of this thread's rows and channels, read straight
-    // into registers (rows past the sequence's end read as zero and are never used)
+    // into registers (rows past the sequence's end read as zero and are never used); an L2
+    // prefetch of a later chunk's inputs runs ahead of these loads
     float4 rw[8];
     uint2 k2[8], q2[8];
     float beta_raw = 0.f;  // beta of one row (lanes 0..7)
@@ -393,8 +394,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         if (qb) tma_prefetch_l2_3d(&tm.q, 0, kh, c0n);
       }
     };
+    // L2 prefetch distance in chunks (measured: the prefill 1.90 -> 1.80 ms with one chunk on the
+    // 64 x 2048-token batch; the segment build 4.79 -> 4.90 ms, so it keeps two)
+    constexpr int kAhead = kBuild ? 2 : 1;
     if (t1 > t0) {
-      prefetch_l2(t0 + C);
+      if (kAhead > 1) prefetch_l2(t0 + C);
       load_raw(t0);
       load_beta(t0);
     }
@@ -405,8 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       const uint32_t par = ci & 1u;
       uint8_t* sP = sm + OFF_P + par * 8192;
       float* sBetaC = sBeta + par * 64;
-      load_kq(c0);
-      prefetch_l2(c0 + 2 * C);
+      // the keys and queries: issued before the gates in the prefill, after them in the build
+      // (measured: the build's gates run faster with those registers free, 4.79 -> 4.75 ms on
+      // the benchmark step; the prefill's part 1 waits on them instead, 1.80 -> 1.82 ms)
+      if constexpr (!kBuild) load_kq(c0);
+      prefetch_l2(c0 + kAhead * C);
 
       // ---- gates of this chunk: alpha = exp(g), 1 past the sequence end
       float al[8][4];
@@ -451,6 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         sBetaC[row] = row < L ? beta_f32(beta_raw, prob) : 0.f;
       }
 
+      if constexpr (kBuild) load_kq(c0);
       // ---- part 1: in-block products.  k and q of my rows stay packed in registers (two bf16
       // per word) and are widened where they are used: widening is one instruction per value,
       // and the fp32 copies would hold 64 more registers through part 1 and the tiles
