@@ -95,15 +95,21 @@ constexpr int OFF_TAU = OFF_A + 17408;      // fp32 [8][128] decay product of ea
 constexpr int OFF_MP = OFF_TAU + 4096;      // bf16x2 [6][64] decay between 16-blocks of a pair
 constexpr int OFF_BETA = OFF_MP + 1536;     // fp32 [2][64] beta (chunk parity)
 constexpr int OFF_GC = OFF_BETA + 512;      // fp32 [2][128] Gamma of the last row (chunk parity)
-constexpr int OFF_BAR = OFF_GC + 1024;      // mbarriers (+0..+71), TMEM base (+72), abort flag (+76)
+constexpr int OFF_BAR = OFF_GC + 1024;      // mbarriers (+0..+71), TMEM base (+72), abort flag (+76),
+                                            // the staged inputs' mbarrier (+80)
 constexpr int kSmemBytes = OFF_BAR + 128;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for aligning the base to 1024
-// the state team's inverse works in the score tiles, free once the key team's scores are done
-// (the key team rewrites them only after the inverse has signalled)
-constexpr int OFF_XI = OFF_KPI;             // fp32 [64][68] inverse
-constexpr int OFF_Y = OFF_KPI8;             // fp32 inverse temporaries: [4][8][8] and [4][16][8], then
+// Once the key team's scores of a chunk are done, the score tiles' region serves two users until
+// the key team's next tiles: the state team's inverse works at its end, and the next chunk's raw
+// gates and keys arrive at its start by tensor copies (the key team reads them there for its
+// gates and in-block products)
+constexpr int OFF_STG = OFF_KPI;            // raw gates, fp32 [64][128] (token rows)
+constexpr int OFF_STG_K = OFF_STG + 32768;  // keys, bf16 [64][128]
+constexpr int OFF_Y = OFF_A - 6144;         // fp32 inverse temporaries: [4][8][8] and [4][16][8], then
                                             // [32][32] after them
-static_assert(OFF_XI + 17408 <= OFF_KC && OFF_Y + 6144 <= OFF_QPI8, "inverse scratch overlaps live tiles");
+constexpr int OFF_XI = OFF_Y - 17408;       // fp32 [64][68] inverse
+static_assert(OFF_STG_K + 16384 <= OFF_XI && OFF_XI >= OFF_KPI && OFF_XI % 1024 == 0,
+              "staged inputs overlap the inverse's scratch");
 constexpr int kLdA = 68;                    // row stride of the fp32 [64][*] arrays
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
@@ -246,9 +252,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   // bar0..bar4: completions of the chunk's product groups (bar3: the issuing threads' final
   // commits when a chunk loop is abandoned); bar_v: V's tensor copy; bar_tiles, bar_scores:
   // the key team's operand tiles and scores of a chunk are in place; bar_inv: the state team's
-  // inverse of a chunk is done (sA and the inverse's scratch in the score tiles are free)
+  // inverse of a chunk is done (sA and the inverse's scratch in the score tiles are free); bar_stg:
+  // a chunk's raw gates and keys have been copied in
   const uint32_t bar0 = sbase + OFF_BAR, bar1 = bar0 + 8, bar2 = bar0 + 16, bar3 = bar0 + 24, bar4 = bar0 + 32;
   const uint32_t bar_v = bar0 + 40, bar_tiles = bar0 + 48, bar_scores = bar0 + 56, bar_inv = bar0 + 64;
+  const uint32_t bar_stg = bar0 + 80;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_BAR + 72);
   volatile int* s_abort = reinterpret_cast<volatile int*>(sm + OFF_BAR + 76);
   float* sA = reinterpret_cast<float*>(sm + OFF_A);
@@ -267,6 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     mbar_init(bar_tiles, 1);
     mbar_init(bar_scores, 1);
     mbar_init(bar_inv, 1);
+    mbar_init(bar_stg, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -355,29 +364,31 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     const float cexp = expf(a.a_log[h]);
     const float alpha_floor = safe ? expf(a.lb) : 0.f;
     const int b16 = kw >> 1, upper = kw & 1;
-    const float* raw_base = a.raw_gate + (size_t)h * D + ch;
-    const size_t raw_stride = (size_t)a.Hv * D, kq_stride = (size_t)a.Hk * D;
-    const __nv_bfloat16* k_base = reinterpret_cast<const __nv_bfloat16*>(a.k) + (size_t)kh * D + ch;
+    const size_t kq_stride = (size_t)a.Hk * D;
     const __nv_bfloat16* q_base = reinterpret_cast<const __nv_bfloat16*>(qb ? a.q : a.k) + (size_t)kh * D + ch;
-    // a chunk's raw gates, keys and queries of this thread's rows and channels, read straight
-    // into registers (rows past the sequence's end read as zero and are never used); an L2
-    // prefetch of a later chunk's inputs runs ahead of these loads
-    float4 rw[8];
+    // A chunk's raw gates and keys arrive in shared memory by tensor copies, issued once the
+    // previous chunk's scores are done (the copies then run under its state tiles); the queries
+    // of this thread's rows and channels are read straight into registers.  Rows past the
+    // sequence's end read as zero (keys, queries) or are never used (gates).  An L2 prefetch of
+    // a later chunk's inputs runs ahead of both.
     uint2 k2[8], q2[8];
     float beta_raw = 0.f;  // beta of one row (lanes 0..7)
-    auto load_raw = [&](int c0n) {
+    auto issue_stage = [&](int c0n) {  // one thread
+      mbar_arrive_expect_tx(bar_stg, 32768u + 16384u);
+      tma_load_3d(sbase + OFF_STG, &tm.raw, 0, h, c0n, bar_stg);
+      tma_load_3d(sbase + OFF_STG_K, &tm.k, 0, kh, c0n, bar_stg);
+    };
+    auto read_k = [&](int L) {
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        const int t = c0n + kw * 8 + r;
-        rw[r] = t < t1 ? __ldg(reinterpret_cast<const float4*>(raw_base + (size_t)t * raw_stride))
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int row = kw * 8 + r;
+        k2[r] = row < L ? *reinterpret_cast<const uint2*>(sm + OFF_STG_K + (row * D + ch) * 2) : make_uint2(0u, 0u);
       }
     };
-    auto load_kq = [&](int c0n) {
+    auto load_q = [&](int c0n) {
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         const int t = c0n + kw * 8 + r;
-        k2[r] = t < t1 ? __ldg(reinterpret_cast<const uint2*>(k_base + (size_t)t * kq_stride)) : make_uint2(0u, 0u);
         q2[r] = (qb && t < t1) ? __ldg(reinterpret_cast<const uint2*>(q_base + (size_t)t * kq_stride))
                                : make_uint2(0u, 0u);
       }
@@ -397,10 +408,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
     // L2 prefetch distance in chunks (measured: the prefill 1.90 -> 1.80 ms with one chunk on the
     // 64 x 2048-token batch; the segment build 4.79 -> 4.90 ms, so it keeps two)
     constexpr int kAhead = kBuild ? 2 : 1;
+    bool stg_pending = false;  // a staging copy issued whose completion was not yet observed
+    uint32_t stg_parity = 0;   // parity of the next completion on bar_stg
     if (t1 > t0) {
       if (kAhead > 1) prefetch_l2(t0 + C);
-      load_raw(t0);
-      load_beta(t0);
+      if (tid == 0) issue_stage(t0);
+      stg_pending = true;
     }
     uint32_t ci = 0;  // chunk index
 #pragma unroll 1
@@ -409,11 +422,19 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       const uint32_t par = ci & 1u;
       uint8_t* sP = sm + OFF_P + par * 8192;
       float* sBetaC = sBeta + par * 64;
-      // the keys and queries: issued before the gates in the prefill, after them in the build
-      // (measured: the build's gates run faster with those registers free, 4.79 -> 4.75 ms on
-      // the benchmark step; the prefill's part 1 waits on them instead, 1.80 -> 1.82 ms)
-      if constexpr (!kBuild) load_kq(c0);
+      // the queries: issued before the gates in the prefill, after them in the build (measured:
+      // the build's gates run faster with those registers free, the prefill's part 1 waits on
+      // them instead)
+      load_beta(c0);
+      if constexpr (!kBuild) load_q(c0);
       prefetch_l2(c0 + kAhead * C);
+      // this chunk's staged raw gates and keys
+      if (!mbar_wait_bounded(bar_stg, stg_parity, kWaitLimitNs)) {
+        *s_abort = 1;
+        report(a.status, KDA_ERR_DEVICE_TIMEOUT);
+      }
+      stg_pending = false;
+      stg_parity ^= 1u;
 
       // ---- gates of this chunk: alpha = exp(g), 1 past the sequence end
       float al[8][4];
@@ -423,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
 #pragma unroll
         for (int c = 0; c < 4; ++c) al[r][c] = 1.f;
         if (row < L) {
-          const float4 raw = rw[r];
+          const float4 raw = *reinterpret_cast<const float4*>(sm + OFF_STG + (row * D + ch) * 4);
           // softplus(x) in log2 units, log2(1 + 2^(x log2 e)), then alpha = exp(-exp(a_log)
           // softplus(x)) = 2^(-c sp2); the limits come out right on both sides (x large: the power
           // overflows to inf and alpha = 0; x very negative: it flushes to 0 and alpha = 1).  In the
@@ -458,7 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         sBetaC[row] = row < L ? beta_f32(beta_raw, prob) : 0.f;
       }
 
-      if constexpr (kBuild) load_kq(c0);
+      read_k(L);
+      if constexpr (kBuild) load_q(c0);
       // ---- part 1: in-block products.  k and q of my rows stay packed in registers (two bf16
       // per word) and are widened where they are used: widening is one instruction per value,
       // and the fp32 copies would hold 64 more registers through part 1 and the tiles
@@ -675,11 +697,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       }
       group_sync(kKeyBar, kTeam);  // (2) score tiles, pair decays and diagonal scores in place
 
-      // the next chunk's raw gates and beta, read now: the score phase hides their latency
-      if (c0 + C < t1) {
-        load_raw(c0 + C);
-        load_beta(c0 + C);
-      }
 
       // ---- part 2: off-diagonal scores on mma.sync
       {
@@ -776,7 +793,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       }
       fence_async_smem();          // P is read by the tensor cores
       group_sync(kKeyBar, kTeam);  // (3) A, P and the 8x8 block inverses complete
-      if (tid == 0) mbar_arrive(bar_scores);
+      // the score tiles have been read: the next chunk's raw gates and keys may come in (every
+      // thread's reads were ordered before the copies by its proxy fence and the barrier)
+      if (tid == 0) {
+        mbar_arrive(bar_scores);
+        if (c0 + C < t1) issue_stage(c0 + C);
+      }
+      stg_pending = c0 + C < t1;
 
       // ---- the state side's tiles, once the previous chunk's products that read them completed:
       // its state updates (K') and its readout / output products (the K o Gamma and Q o Gamma
@@ -848,6 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         if (tid == 0) mbar_arrive(bar_tiles);
       }
     }
+    if (stg_pending) mbar_wait_bounded(bar_stg, stg_parity, kWaitLimitNs);  // a copy still in flight
     regs_decrease<kLaunchRegs>();  // back to the launch's share before the teams join
   } else {
     regs_decrease<RegSplit<kBuild>::state>();
