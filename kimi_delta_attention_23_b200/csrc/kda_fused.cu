@@ -422,11 +422,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       const uint32_t par = ci & 1u;
       uint8_t* sP = sm + OFF_P + par * 8192;
       float* sBetaC = sBeta + par * 64;
-      // the queries: issued before the gates in the prefill, after them in the build (measured:
-      // the build's gates run faster with those registers free, the prefill's part 1 waits on
-      // them instead)
+      // this chunk's beta and queries, read into registers: the gates hide their latency
+      // (measured: with the keys staged, the benchmark step 4.635 -> 4.585 ms against issuing the
+      // build's queries after the gates)
       load_beta(c0);
-      if constexpr (!kBuild) load_q(c0);
+      load_q(c0);
       prefetch_l2(c0 + kAhead * C);
       // this chunk's staged raw gates and keys
       if (!mbar_wait_bounded(bar_stg, stg_parity, kWaitLimitNs)) {
@@ -480,7 +480,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       }
 
       read_k(L);
-      if constexpr (kBuild) load_q(c0);
       // ---- part 1: in-block products.  k and q of my rows stay packed in registers (two bf16
       // per word) and are widened where they are used: widening is one instruction per value,
       // and the fp32 copies would hold 64 more registers through part 1 and the tiles
@@ -901,9 +900,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       const float* sBetaC = sBeta + par * 64;
       const float* sGCc = sGC + par * 128;
 
-      // ---- the first product(s) once the key team's tiles are in place; the bf16 state copies
-      // (this team's, at the end of the previous chunk) have landed
-      if (st == kIssueFirst) {
+      // the first product(s), once the key team's tiles are in place (the bf16 state copies, this
+      // team's, landed at the end of the previous chunk); one thread
+      auto issue_first = [&]() {
         if (!mbar_wait_bounded(bar_tiles, par, kWaitLimitNs)) {
           *s_abort = 1;
           report(a.status, KDA_ERR_DEVICE_TIMEOUT);
@@ -929,7 +928,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           }
           mma_commit(bar0);
         }
-      }
+      };
+      // The build issues them here; the prefill inside the inverse's first level, where its
+      // epilogue runs (measured: the prefill 1.705 -> 1.67 ms on the 64 x 2048-token batch; the
+      // build slower, 4.62 -> 4.89 ms on the benchmark step, as its later products then meet the
+      // key team's tile stores)
+      if (kBuild && st == kIssueFirst) issue_first();
       // the previous chunk's staged outputs have been read by their tensor store (the staging
       // tiles are rewritten below)
       if (st == kCopyThread) bulk_wait_read_all();
@@ -993,6 +997,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           // product's epilogue; warp -> TMEM lane quadrant sw % 4, all 64 columns.  Y^T[j][r] =
           // -((K o Gamma) S0)^T into the X tile(s) (in the build the products computed it negated;
           // the prefill's one N = 128 product negates here); V enters in the next product
+          if (!kBuild && st == kIssueFirst) issue_first();
+          __syncwarp();
           if (!mbar_wait_bounded(bar0, par, kWaitLimitNs)) {
             *s_abort = 1;
             report(a.status, KDA_ERR_DEVICE_TIMEOUT);
