@@ -800,6 +800,71 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       }
       stg_pending = c0 + C < t1;
 
+      // ---- prefill: the state side's tiles.  K o Gamma and Q o Gamma were read only by the previous
+      // chunk's first product, which completed before its inverse signalled (observed at (1)), so
+      // they are written at once.  K' waits for the previous chunk's state update, and the wait
+      // also covers its output product: it read the score tile P of that chunk's parity, which
+      // the next chunk's in-block products rewrite before their first barrier.
+      if constexpr (!kBuild) {
+        float p8[8][4], s8[8][4];
+        block_products(p8, s8);
+        float pre[4], suf[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          pre[c] = 1.f;
+          suf[c] = 1.f;
+        }
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          const float4 t4 = *reinterpret_cast<const float4*>(sTau + w * D + ch);
+          const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            if (w < kw) pre[c] *= tv[c];
+            if (w > kw) suf[c] *= tv[c];
+          }
+        }
+        if (kw == 0) {
+          *reinterpret_cast<float4*>(sGC + par * 128 + ch) =
+              make_float4(p8[7][0] * suf[0], p8[7][1] * suf[1], p8[7][2] * suf[2], p8[7][3] * suf[3]);
+        }
+        const float2 pre01 = make_float2(pre[0], pre[1]), pre23 = make_float2(pre[2], pre[3]);
+        const float2 suf01 = make_float2(suf[0], suf[1]), suf23 = make_float2(suf[2], suf[3]);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int row = kw * 8 + r;
+          const float2 p01 = make_float2(p8[r][0], p8[r][1]), p23 = make_float2(p8[r][2], p8[r][3]);
+          const float2 kp01 = mul_f32x2(klo(r), p01), kp23 = mul_f32x2(khi(r), p23);
+          const float2 qp01 = mul_f32x2(qlo(r), p01), qp23 = mul_f32x2(qhi(r), p23);
+          *reinterpret_cast<uint2*>(sm + OFF_KQ + sw_off(row, ch, 128)) =
+              pack4(mul_f32x2(kp01, pre01), mul_f32x2(kp23, pre23));
+          *reinterpret_cast<uint2*>(sm + OFF_KQ + sw_off(64 + row, ch, 128)) =
+              pack4(mul_f32x2(qp01, pre01), mul_f32x2(qp23, pre23));
+        }
+        bool bad = false;
+        if (ci > 0 && tid == 0) {
+          bad = !mbar_wait_bounded(bar4, par ^ 1u, kWaitLimitNs) || !mbar_wait_bounded(bar2, par ^ 1u, kWaitLimitNs);
+          if (bad) {
+            *s_abort = 1;
+            report(a.status, KDA_ERR_DEVICE_TIMEOUT);
+          }
+        }
+        if (group_sync_any(kKeyBar, kTeam, bad || *s_abort != 0)) {  // (4)
+          aborted = true;
+          break;
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int row = kw * 8 + r;
+          const float2 s01 = make_float2(s8[r][0], s8[r][1]), s23 = make_float2(s8[r][2], s8[r][3]);
+          const float2 ks01 = mul_f32x2(klo(r), s01), ks23 = mul_f32x2(khi(r), s23);
+          *reinterpret_cast<uint2*>(sm + OFF_KPT + sw_off(row, ch, 64)) =
+              pack4(mul_f32x2(ks01, suf01), mul_f32x2(ks23, suf23));
+        }
+        fence_async_smem();  // the state tiles are read by the tensor cores
+        group_sync(kKeyBar, kTeam);  // (5) state tiles in place (and every read of sTau done)
+        if (tid == 0) mbar_arrive(bar_tiles);
+      } else
       // ---- the state side's tiles, once the previous chunk's products that read them completed:
       // its state updates (K') and its readout / output products (the K o Gamma and Q o Gamma
       // tile).  This is the only place the key team waits on those products, so its gates,
