@@ -99,9 +99,16 @@ enum {
   KDA_FORCE_SIMT = 1u << 5,    /* run the fp32 CUDA-core chunk kernel even for bf16 inputs       */
   KDA_READOUT_HEAD_MAJOR = 1u << 6, /* readout_m / readout_u stored [Hv, T, 128] instead of
                                        [T, Hv, 128] (calls that write or read readouts only)     */
-  KDA_SCAN_LOGDEPTH = 1u << 7  /* segment call: the scan in log depth (needs the workspace of
+  KDA_SCAN_LOGDEPTH = 1u << 7, /* segment call: the scan in log depth (needs the workspace of
                                   kda_scan_workspace_size); without it the log-depth form is
                                   chosen when that workspace is given and it is expected faster */
+  KDA_DEBUG_WITHHOLD_HANDOFF = 1u << 8 /* test hook for the bounded waits (kda_chunk_fwd): the bf16
+                                  kernel withholds one "scores ready" signal between its two
+                                  warp teams in every chain's first chunk, so the waiting team
+                                  gives up after its limit (about one second).  device_status
+                                  then reads KDA_ERR_DEVICE_TIMEOUT, the outputs and the pool
+                                  slots are unspecified, and the context stays usable.  No
+                                  effect on the fp32 kernel. */
 };
 
 /*

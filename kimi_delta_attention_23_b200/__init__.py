@@ -45,6 +45,10 @@ SEG_SCAN_ONLY = 1 << 4
 FORCE_SIMT = 1 << 5
 READOUT_HEAD_MAJOR = 1 << 6
 SCAN_LOGDEPTH = 1 << 7
+DEBUG_WITHHOLD_HANDOFF = 1 << 8  # test hook: see include/kda.h
+# device_status values (kda_status_t in include/kda.h) that callers test for
+ERR_DEVICE_CHECK = 5
+ERR_DEVICE_TIMEOUT = 6
 
 _F32, _BF16 = 0, 1
 _DTYPES = {torch.float32: _F32, torch.bfloat16: _BF16}
@@ -221,7 +225,7 @@ class _Owned:
 def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, state_pool, state_indices,
                   out=None, *, output_dtype=None, use_computebound=False, gate_mode="original",
                   beta_mode="logits", state_layout="K_FIRST", gate_lower_bound=-5.0, force_simt=False,
-                  workspace=None, device_status=None, stream=None):
+                  workspace=None, device_status=None, stream=None, _debug_flags=0):
     """Chunk-parallel KDA prefill (``max.nn.state_space.kda_chunk`` semantics).
 
     Shapes: q,k [T,Hk,dk]; v [T,Hv,dv]; raw_gate [T,Hv,dk] f32; beta_logits [T,Hv] f32;
@@ -230,6 +234,7 @@ def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, st
     Returns out [T,Hv,dv] in ``output_dtype`` (default: the dtype of v).  ``workspace`` (uint8
     CUDA tensor) enables the split route for batches of few or uneven sequences; it is
     allocated at kda_workspace_size bytes when not given (pass an empty tensor to disable).
+    ``_debug_flags`` is OR-ed into the call's flags (tests pass ``DEBUG_WITHHOLD_HANDOFF``).
     """
     lib = load_library()
     dev = q.device
@@ -264,7 +269,7 @@ def kda_chunk_fwd(q, k, v, raw_gate, beta_logits, a_log, dt_bias, cu_seqlens, st
     _shape(_dev(out, "out", output_dtype, dev), "out", (T, Hv, dv))
     if device_status is not None:
         _shape(_dev(device_status, "device_status", torch.int32, dev), "device_status", (1,))
-    flags = _flags(gate_mode, beta_mode, state_layout, use_computebound, force_simt)
+    flags = _flags(gate_mode, beta_mode, state_layout, use_computebound, force_simt) | int(_debug_flags)
     if workspace is None:
         need = 0
         if q.dtype == torch.bfloat16 and not force_simt:

@@ -17,7 +17,8 @@ bool fused_available();
 namespace {
 
 constexpr uint32_t kKnownFlags = KDA_GATE_SAFE | KDA_BETA_PROB | KDA_STATE_V_FIRST | KDA_FUSED |
-                                 KDA_SEG_SCAN_ONLY | KDA_FORCE_SIMT | KDA_READOUT_HEAD_MAJOR | KDA_SCAN_LOGDEPTH;
+                                 KDA_SEG_SCAN_ONLY | KDA_FORCE_SIMT | KDA_READOUT_HEAD_MAJOR | KDA_SCAN_LOGDEPTH |
+                                 KDA_DEBUG_WITHHOLD_HANDOFF;
 
 bool dtype_ok(kda_dtype_t t) { return t == KDA_F32 || t == KDA_BF16; }
 

@@ -795,7 +795,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
       // the score tiles have been read: the next chunk's raw gates and keys may come in (every
       // thread's reads were ordered before the copies by its proxy fence and the barrier)
       if (tid == 0) {
-        mbar_arrive(bar_scores);
+        // (the test hook withholds the first chunk's signal: the state team's bounded wait then
+        // gives up and both teams leave through the abort flag)
+        if (!((a.flags & KDA_DEBUG_WITHHOLD_HANDOFF) && ci == 0)) mbar_arrive(bar_scores);
         if (c0 + C < t1) issue_stage(c0 + C);
       }
       stg_pending = c0 + C < t1;

@@ -233,3 +233,22 @@ def test_logdepth_scan_sizes_and_host_checks(lib):
     # forced without a workspace, or where it cannot run: refused before any launch
     assert _seg(lib, flags=kda.SEG_SCAN_ONLY | kda.SCAN_LOGDEPTH) == 3            # KDA_ERR_WORKSPACE
     assert _seg(lib, flags=kda.SEG_SCAN_ONLY | kda.SCAN_LOGDEPTH, dk=64) == 2     # KDA_ERR_UNSUPPORTED
+
+
+def test_python_constants_match_the_header():
+    """The binding's flag and status constants are the header's values."""
+    text = open(HEADER).read()
+
+    def enum_value(name):
+        m = re.search(rf"\b{name}\s*=\s*(1u\s*<<\s*(\d+)|\d+)", text)
+        assert m, name
+        return (1 << int(m.group(2))) if m.group(2) else int(m.group(1))
+
+    for py, c in (("GATE_SAFE", "KDA_GATE_SAFE"), ("BETA_PROB", "KDA_BETA_PROB"),
+                  ("STATE_V_FIRST", "KDA_STATE_V_FIRST"), ("FUSED", "KDA_FUSED"),
+                  ("SEG_SCAN_ONLY", "KDA_SEG_SCAN_ONLY"), ("FORCE_SIMT", "KDA_FORCE_SIMT"),
+                  ("READOUT_HEAD_MAJOR", "KDA_READOUT_HEAD_MAJOR"), ("SCAN_LOGDEPTH", "KDA_SCAN_LOGDEPTH"),
+                  ("DEBUG_WITHHOLD_HANDOFF", "KDA_DEBUG_WITHHOLD_HANDOFF"),
+                  ("ERR_DEVICE_CHECK", "KDA_ERR_DEVICE_CHECK"), ("ERR_DEVICE_TIMEOUT", "KDA_ERR_DEVICE_TIMEOUT")):
+        assert getattr(kda, py) == enum_value(c), (py, c)
+    assert kda.kda_status_string(kda.ERR_DEVICE_TIMEOUT).startswith("KDA_ERR_DEVICE_TIMEOUT")
