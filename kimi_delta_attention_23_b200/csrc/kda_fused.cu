@@ -288,9 +288,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   // TMEM columns.  prefill: D1 [0,128) (X/Delta part, then O part), S fp32 [128,256), S bf16
-  // [256,320).  build: D1 of M [0,64) and of U [64,128), S_M [128,256), S_U [256,384), bf16
-  // copies [384,448) and [448,512).
+  // [256,320), Delta^T bf16 [320,352) (the A operand of the output product and the update).
+  // build: D1 of M [0,64) and of U [64,128), S_M [128,256), S_U [256,384), bf16 copies [384,448)
+  // and [448,512).
   const uint32_t tmD1 = tmem, tmS = tmem + 128, tmSb = kBuild ? tmem + 384 : tmem + 256;
+  const uint32_t tmDb = tmem + 320;
   const uint32_t tmD1u = tmem + 64, tmSu = tmem + 256, tmSbu = tmem + 448;
   const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   constexpr bool qb = kRead;
@@ -1217,14 +1219,15 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
             report(a.status, KDA_ERR_DEVICE_TIMEOUT);
           } else {
             tc_fence_after();
+            // Delta^T stays in TMEM as bf16 (two tokens per column), the A operand of the two
+            // products below: no shared-memory round trip for it (measured: see the products)
             float d[32];
             tmem_ld16n<2>(tmD1 + lane_base + 32 * ehalf, d);
             tmem_wait_ld();
+            uint32_t pk[16];
 #pragma unroll
-            for (int r0 = 0; r0 < 32; r0 += 8)
-              *reinterpret_cast<uint4*>(sm + OFF_X + sw_off(ej, 32 * ehalf + r0, 128)) =
-                  make_uint4(pack_bf16(d[r0], d[r0 + 1]), pack_bf16(d[r0 + 2], d[r0 + 3]),
-                             pack_bf16(d[r0 + 4], d[r0 + 5]), pack_bf16(d[r0 + 6], d[r0 + 7]));
+            for (int u = 0; u < 16; ++u) pk[u] = pack_bf16(d[2 * u], d[2 * u + 1]);
+            tmem_st16u(tmDb + lane_base + 16 * ehalf, pk);
           }
           tmem_wait_st();
           fence_async_smem();
@@ -1244,27 +1247,27 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           v_pending = has_v;
         }
 
-        // D1[:, 64:128] += Delta^T P^T ;  S^T += Delta^T K'   (accumulate; two issuing threads)
+        // D1[:, 64:128] += Delta^T P^T ;  S^T += Delta^T K'   (accumulate; two issuing threads; A is
+        // Delta^T in TMEM, 8 columns per 16 tokens)
         if (st == kIssueRead) {
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmD1 + 64, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128(sbase + pofs + kk * 32),
-                     idesc_bf16_f32(64), 1);
+            mma_bf16_ts(tmD1 + 64, tmDb + 8 * kk, desc_sw128(sbase + pofs + kk * 32), idesc_bf16_f32(64), 1);
           mma_commit(bar2);
         }
         if (st == kIssueUpdate) {
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmS, desc_sw128(sbase + OFF_X + kk * 32), desc_sw128_mn(sbase + OFF_KPT + kk * 2048, 8192),
-                     idesc_bf16_f32(128, false, true), 1);
+            mma_bf16_ts(tmS, tmDb + 8 * kk, desc_sw128_mn(sbase + OFF_KPT + kk * 2048, 8192),
+                        idesc_bf16_f32(128, false, true), 1);
           mma_commit(bar4);
         }
         {
           // the outputs are staged while the state update still runs: bf16 in the XM tile (no
-          // product reads it in the prefill); fp32 from the X tile on, once the update (which
-          // reads X) has completed
+          // product reads it in the prefill); fp32 from the X tile on (free once the second
+          // product completed), after the update too
           const bool out_done = mbar_wait_bounded(bar2, par, kWaitLimitNs);
           const bool upd_done = out_done && (a.out_bf16 || !a.out || mbar_wait_bounded(bar4, par, kWaitLimitNs));
           if (out_done && upd_done) {
