@@ -1454,17 +1454,33 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
         } else {
           tc_fence_after();
           if constexpr (kRead) {
+            // staged for the tensor stores as two token-row [64][64 channels] bf16 halves with the
+            // 128-byte swizzle: a 16 x 256-bit TMEM load hands each thread two adjacent tokens of
+            // two channels, and transposing matrix stores write them as 8 x 8 blocks of token rows
+            // (8 channels, 16 bytes each)
+            const int q4 = warp & 3, jm = lane >> 3, rr = lane & 7;
 #pragma unroll 1
             for (int stt = 0; stt < 2; ++stt) {
-              float d[32];
-              tmem_ld16n<2>((stt ? tmD1u : tmD1) + lane_base + 32 * ehalf, d);
-              tmem_wait_ld();
-              uint8_t* stage = sm + (stt ? OFF_X : OFF_XM);
+              const uint32_t stage = sbase + (stt ? OFF_X : OFF_XM);
 #pragma unroll
-              for (int u = 0; u < 32; u += 2) {  // one conversion per row pair, two 16-bit stores
-                const uint32_t pk = pack_bf16(d[u], d[u + 1]);
-                *reinterpret_cast<uint16_t*>(stage + ((32 * ehalf + u) * D + ej) * 2) = (uint16_t)(pk & 0xffffu);
-                *reinterpret_cast<uint16_t*>(stage + ((32 * ehalf + u + 1) * D + ej) * 2) = (uint16_t)(pk >> 16);
+              for (int hh = 0; hh < 2; ++hh) {
+                uint32_t r[16];
+                tmem_ld16x256b_x4((stt ? tmD1u : tmD1) + ((uint32_t)(32 * q4 + 16 * hh) << 16) + 32 * ehalf, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k2 = 0; k2 < 2; ++k2) {
+                  // matrix jm: tokens 32 ehalf + 16 k2 + 8 (jm / 2) .., channels 32 q4 + 16 hh + 8 (jm % 2) ..;
+                  // this lane addresses its token row rr
+                  const int tok = 32 * ehalf + 16 * k2 + 8 * (jm >> 1) + rr;
+                  const int chn = 32 * q4 + 16 * hh + 8 * (jm & 1);
+                  const uint32_t addr =
+                      stage + (chn >> 6) * 8192 + tok * 128 + ((((chn & 63) >> 3) ^ (tok & 7)) << 4);
+                  const uint32_t* v = r + 8 * k2;
+                  stsm_x4_trans(addr, pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                                pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                                pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                                pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7])));
+                }
               }
             }
           }
@@ -1489,13 +1505,15 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           break;
         }
         if constexpr (kRead) {
-          // full chunks leave through two tensor stores (sources read before the next chunk's first
-          // epilogue rewrites them)
+          // full chunks leave through four tensor stores, a 64-channel half each (sources read before
+          // the next chunk's first epilogue rewrites them)
           if (L == C) {
             if (st == kCopyThread) {
               const int y = a.readout_hm ? (int)c0 : h, z = a.readout_hm ? h : (int)c0;
               tma_store_3d(&tm.out, sbase + OFF_XM, 0, y, z);
+              tma_store_3d(&tm.out, sbase + OFF_XM + 8192, 64, y, z);
               tma_store_3d(&tm.out2, sbase + OFF_X, 0, y, z);
+              tma_store_3d(&tm.out2, sbase + OFF_X + 8192, 64, y, z);
               bulk_commit();
             }
           } else {
@@ -1505,7 +1523,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
                 *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(sti ? a.out2 : a.out) +
                                           (a.readout_hm ? (size_t)h * a.total_tokens + c0 + row
                                                         : (size_t)(c0 + row) * a.Hv + h) * D + cc * 8) =
-                    *reinterpret_cast<const uint4*>(sm + (sti ? OFF_X : OFF_XM) + row * 256 + cc * 16);
+                    *reinterpret_cast<const uint4*>(sm + (sti ? OFF_X : OFF_XM) + (cc >> 3) * 8192 + row * 128 +
+                                                    (((cc & 7) ^ (row & 7)) << 4));
             }
           }
         }
@@ -1618,12 +1637,15 @@ cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream) {
                   encode_rows(&tm.q, a.q ? a.q : a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hk) &&
                   encode_rows(&tm.v, a.v ? a.v : a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv, 64,
                               CU_TENSOR_MAP_SWIZZLE_128B);
-  // bf16 outputs (the prefill output, or both readouts of the build) leave through tensor stores
+  // bf16 outputs (the prefill output, or both readouts of the build) leave through tensor stores;
+  // the build stages its readouts as 64-channel halves with the 128-byte swizzle
+  const uint32_t out_box = a.build ? 64u : (uint32_t)D;
+  const CUtensorMapSwizzle out_swz = a.build ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
   const bool out_ok = rows == 0 || !a.out || !a.out_bf16 ||
-                      (encode_rows(&tm.out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv, D,
-                                   CU_TENSOR_MAP_SWIZZLE_NONE, a.build && a.readout_hm) &&
-                       (!a.out2 || encode_rows(&tm.out2, a.out2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv, D,
-                                               CU_TENSOR_MAP_SWIZZLE_NONE, a.build && a.readout_hm)));
+                      (encode_rows(&tm.out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv, out_box, out_swz,
+                                   a.build && a.readout_hm) &&
+                       (!a.out2 || encode_rows(&tm.out2, a.out2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv,
+                                               out_box, out_swz, a.build && a.readout_hm)));
   if (!ok || !out_ok) return cudaErrorInvalidValue;
   dim3 grid(a.Hv, a.batch);
   if (a.build && a.out)

@@ -241,6 +241,16 @@ __device__ __forceinline__ void tmem_ld16n(uint32_t taddr, float (&v)[16 * N]) {
     for (int i = 0; i < 16; ++i) v[16 * q + i] = __uint_as_float(r[i]);
   }
 }
+// 16 lanes x 256 bits, four repetitions along the columns (32 columns): thread t holds, per
+// repetition k (columns 8k .. 8k + 7 from taddr), r[4k], r[4k + 1] = lane t / 4, columns 8k + 2 (t % 4)
+// and + 1, and r[4k + 2], r[4k + 3] = lane t / 4 + 8, the same columns (the mma accumulator layout)
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 // 32 lanes x 32-bit, 64 consecutive columns in one load
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   uint32_t r[64];
@@ -358,6 +368,13 @@ __device__ __forceinline__ void regs_decrease() {
 }
 
 // ---------------------------------------------------------------- legacy warp-level MMA
+// four 8 x 8 bf16 matrices stored transposed: thread t holds, in r_j, row t / 4 and columns 2 (t % 4),
+// + 1 of matrix j; the shared address of thread 8 j + i receives column i of matrix j (16 bytes)
+__device__ __forceinline__ void stsm_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r0), "r"(r1),
+               "r"(r2), "r"(r3)
+               : "memory");
+}
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
