@@ -1272,21 +1272,34 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           const bool upd_done = out_done && (a.out_bf16 || !a.out || mbar_wait_bounded(bar4, par, kWaitLimitNs));
           if (out_done && upd_done) {
             tc_fence_after();
-            if (a.out) {
+            if (a.out && a.out_bf16) {
+              // two token-row [64][64 channels] halves with the 128-byte swizzle, written by
+              // transposing matrix stores from a 16 x 256-bit TMEM load (as the build's readouts)
+              const int q4 = warp & 3, jm = lane >> 3, rr = lane & 7;
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                uint32_t r[16];
+                tmem_ld16x256b_x4(tmD1 + 64 + ((uint32_t)(32 * q4 + 16 * hh) << 16) + 32 * ehalf, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k2 = 0; k2 < 2; ++k2) {
+                  const int tok = 32 * ehalf + 16 * k2 + 8 * (jm >> 1) + rr;
+                  const int chn = 32 * q4 + 16 * hh + 8 * (jm & 1);
+                  const uint32_t addr =
+                      sbase + OFF_XM + (chn >> 6) * 8192 + tok * 128 + ((((chn & 63) >> 3) ^ (tok & 7)) << 4);
+                  const uint32_t* v = r + 8 * k2;
+                  stsm_x4_trans(addr, pack_bf16(__uint_as_float(v[0]), __uint_as_float(v[1])),
+                                pack_bf16(__uint_as_float(v[2]), __uint_as_float(v[3])),
+                                pack_bf16(__uint_as_float(v[4]), __uint_as_float(v[5])),
+                                pack_bf16(__uint_as_float(v[6]), __uint_as_float(v[7])));
+                }
+              }
+            } else if (a.out) {
               float d[32];
               tmem_ld16n<2>(tmD1 + lane_base + 64 + 32 * ehalf, d);
               tmem_wait_ld();
-              if (a.out_bf16) {
 #pragma unroll
-                for (int u = 0; u < 32; u += 2) {  // one conversion per row pair, two 16-bit stores
-                  const uint32_t pk = pack_bf16(d[u], d[u + 1]);
-                  *reinterpret_cast<uint16_t*>(sm + OFF_XM + ((32 * ehalf + u) * D + ej) * 2) = (uint16_t)(pk & 0xffffu);
-                  *reinterpret_cast<uint16_t*>(sm + OFF_XM + ((32 * ehalf + u + 1) * D + ej) * 2) = (uint16_t)(pk >> 16);
-                }
-              } else {
-#pragma unroll
-                for (int u = 0; u < 32; ++u) reinterpret_cast<float*>(sm + OFF_X)[(32 * ehalf + u) * D + ej] = d[u];
-              }
+              for (int u = 0; u < 32; ++u) reinterpret_cast<float*>(sm + OFF_X)[(32 * ehalf + u) * D + ej] = d[u];
             }
           }
           if (!out_done || !upd_done || !mbar_wait_bounded(bar4, par, kWaitLimitNs)) {
@@ -1315,12 +1328,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
           break;
         }
         // flush the staged output rows of this chunk: a full chunk of a bf16 output leaves through
-        // one tensor store (its source is read before the next chunk's staging); otherwise row by
-        // row, so that no row of the next sequence is touched
+        // two tensor stores, a 64-channel half each (the source is read before the next chunk's
+        // staging); otherwise row by row, so that no row of the next sequence is touched
         if (!a.out) {
         } else if (a.out_bf16 && L == C) {
           if (st == kCopyThread) {
             tma_store_3d(&tm.out, sbase + OFF_XM, 0, h, (int)c0);
+            tma_store_3d(&tm.out, sbase + OFF_XM + 8192, 64, h, (int)c0);
             bulk_commit();
           }
         } else if (a.out_bf16) {
@@ -1328,7 +1342,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_chunk_kernel(const FusedArg
             const int row = e >> 4, cc = e & 15;
             if (row < L)
               *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)(c0 + row) * a.Hv + h) * D +
-                                        cc * 8) = *reinterpret_cast<const uint4*>(sm + OFF_XM + row * 256 + cc * 16);
+                                        cc * 8) =
+                  *reinterpret_cast<const uint4*>(sm + OFF_XM + (cc >> 3) * 8192 + row * 128 + (((cc & 7) ^ (row & 7)) << 4));
           }
         } else {
           for (int e = st; e < C * 32; e += kTeam) {
@@ -1637,10 +1652,10 @@ cudaError_t launch_fused_chunk(const FusedArgs& a, cudaStream_t stream) {
                   encode_rows(&tm.q, a.q ? a.q : a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hk) &&
                   encode_rows(&tm.v, a.v ? a.v : a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv, 64,
                               CU_TENSOR_MAP_SWIZZLE_128B);
-  // bf16 outputs (the prefill output, or both readouts of the build) leave through tensor stores;
-  // the build stages its readouts as 64-channel halves with the 128-byte swizzle
-  const uint32_t out_box = a.build ? 64u : (uint32_t)D;
-  const CUtensorMapSwizzle out_swz = a.build ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  // bf16 outputs (the prefill output, or both readouts of the build) leave through tensor stores,
+  // staged as 64-channel halves with the 128-byte swizzle
+  const uint32_t out_box = 64u;
+  const CUtensorMapSwizzle out_swz = CU_TENSOR_MAP_SWIZZLE_128B;
   const bool out_ok = rows == 0 || !a.out || !a.out_bf16 ||
                       (encode_rows(&tm.out, a.out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, a.Hv, out_box, out_swz,
                                    a.build && a.readout_hm) &&
